@@ -1,0 +1,468 @@
+#!/usr/bin/env python
+"""Throughput of the SEED decode hot path on B200: head-steps/s and HBM GB/s.
+
+A step is one pass of the whole hot path over one batch: seed_decode_step for
+every layer (one launch per layer), and seed_compress over all layers after the
+step that fills R + W columns.  Default workload: 36 GDN layers x 48 heads of
+128 x 128, R = W = 16, batch 256 requests per GPU (the full recurrent stack).
+
+Timing: W untimed warm-up steps, then K steps between barriers and device
+synchronisations, CUDA events on the launching stream (max over ranks).  Inputs
+(q, k, v, alpha, beta of a pool of distinct steps) are generated on the device
+before the timed region and are larger than L2, as is the 15 GB state.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun), every rank runs its own requests (weak scaling, no
+collective on the data path).  Prints one JSON line on rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode head-steps/s and achieved HBM GB/s (% of B200 peak) at R=16,W=16"
+UNIT = "head-steps/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=320)
+    ap.add_argument("--warmup", type=int, default=16)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", type=int, default=2, help="workload id (2: the full GDN stack)")
+    ap.add_argument("--batch", type=int, default=None, help="requests per GPU (default: the workload's)")
+    ap.add_argument("--prefill", type=int, default=None, help="prefill tokens (default: the workload's)")
+    ap.add_argument("--input-steps", type=int, default=16, help="distinct pre-generated input steps")
+    ap.add_argument("--dense-steps", type=int, default=8)
+    ap.add_argument("--e2e-steps", type=int, default=8)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        backend = os.environ.get("SEED_BENCH_BACKEND", "nccl")
+        kw = {"timeout": datetime.timedelta(seconds=180)}
+        if backend == "nccl":
+            import torch
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, **kw)
+    return world, rank, local
+
+
+def shard(batch_per_rank: int, rank: int) -> int:
+    """First global request index of this rank's shard (requests are independent)."""
+    return rank * batch_per_rank
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None) -> None:
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and device != "cpu":
+            dist.barrier(device_ids=[device.index if hasattr(device, "index") else int(device)])
+        else:
+            dist.barrier()
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, enabled: bool = True):
+        self.proc = None
+        self.gpu_index = gpu_index
+        self.enabled = enabled
+
+    def __enter__(self):
+        if self.enabled:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
+                     "--format=csv,noheader,nounits", "-lms", "100"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except (OSError, ValueError):
+                self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self) -> dict | None:
+        rows = []
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[4:8]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        load = [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ peaks
+
+def measured_peak_hbm():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------ CPU (oracle) arm
+
+def cpu_oracle_rate(cfg, seconds: float, rank_seed: int = 0) -> dict:
+    """Time the fp64 oracle's decode step + compression on a sample of units."""
+    import numpy as np
+
+    from oracle import compress as ocomp
+    from oracle import convert as oconv
+    from oracle import factored, recurrences
+    from workloads import philox
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:   # pragma: no cover - reporting only
+        threads = 1
+    rng = np.random.default_rng(1234 + rank_seed)
+    n = 96
+    u = rng.choice(cfg.units, size=n, replace=False)
+    b, rem = np.divmod(u, cfg.layers * cfg.heads)
+    l, h = np.divmod(rem, cfg.heads)
+    n_pre = 256
+    S0 = recurrences.dense_prefill(cfg, b, l, h, n_pre)
+    vb = philox.vbar(cfg, l, h).astype(np.float64)
+    a, U, V, _ = oconv.convert(S0, vb, cfg.R)
+    inputs = [recurrences.f64(philox.token_inputs(cfg, b, l, h, t, philox.PHASE_DECODE))
+              for t in range(cfg.W)]
+    steps = 0
+    c = cfg.R
+    t0 = time.perf_counter()
+    while True:
+        for t in range(cfg.W):
+            inp = inputs[t]
+            a, U, V, _o = factored.step(cfg.form, a, U, V, vb, inp["q"], inp["k"], inp["v"],
+                                        inp["alpha"], inp["beta"])
+            c += 1
+            if c == cfg.R + cfg.W:
+                U, V, _s = ocomp.truncate_qr_core(U, V, cfg.R)
+                c = cfg.R
+            steps += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": steps * n / dt, "unit": UNIT, "cores": int(threads), "kind": "oracle",
+            "sample": (f"{n} sampled units of the workload, {steps} decode steps each "
+                       f"({steps // cfg.W} compressions), fp64 NumPy, {dt:.1f} s; "
+                       f"state from a {n_pre}-token oracle prefill (untimed)"),
+            "affinity_cores": len(os.sched_getaffinity(0))}
+
+
+def config_obj(cfg, batch, world, prefill):
+    return {"workload": f"{cfg.name}: {cfg.layers} GDN layers x {cfg.heads} heads, "
+                        f"d_k=d_v={cfg.d_k}, R={cfg.R}, W={cfg.W}" if cfg.form == 0 else cfg.name,
+            "form": {0: "gdn", 1: "kda", 2: "mamba2"}[cfg.form], "layers": cfg.layers,
+            "heads": cfg.heads, "d_k": cfg.d_k, "d_v": cfg.d_v, "R": cfg.R, "W": cfg.W,
+            "batch_per_gpu": batch, "global_batch": batch * world, "prefill_tokens": prefill,
+            "parallelism": f"dp{world} (requests sharded, no collective)",
+            "l2": "inputs and state larger than L2 (no flush needed)"}
+
+
+def run_reference(args, world, rank):
+    from workloads import config
+    cfg = config(args.config)
+    if args.batch:
+        cfg = cfg.replace(batch=args.batch)
+    if rank != 0:
+        return 0
+    per = max(1.0, args.cpu_seconds)
+    res = cpu_oracle_rate(cfg, per)
+    line = {"metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded Philox4x32-10 inputs)", "impl": "reference",
+            "config": config_obj(cfg, cfg.batch, world, 256),
+            "cpu_baseline": res,
+            "e2e": {"value": res["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    line["ms_per_step"] = cfg.units / res["value"] * 1e3
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    from rank_recurrent_state_b200 import build as build_mod
+    from rank_recurrent_state_b200 import roofline
+    from rank_recurrent_state_b200 import seed as S
+    from rank_recurrent_state_b200.pipeline import DeviceRun
+    from workloads import config
+
+    if rank == 0 or not os.path.exists(build_mod.LIB):
+        build_mod.build()
+    if world > 1:
+        barrier(world, None)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    cfg = config(args.config)
+    if args.batch:
+        cfg = cfg.replace(batch=args.batch)
+    B = cfg.batch
+    prefill = cfg.n_prefill if args.prefill is None else args.prefill
+    run = DeviceRun(cfg, b0=shard(B, rank), device=str(dev), n_prefill=prefill,
+                    keep_dense=not args.no_dense)
+    d = run.dims
+    t_setup = time.perf_counter()
+    run.prefill_and_convert()
+    torch.cuda.synchronize()
+    t_setup = time.perf_counter() - t_setup
+
+    # ---- input pool: P distinct steps x L layers, generated on the device
+    P, L, BH = args.input_steps, d.layers, d.batch * d.heads
+    BHp = (BH + 3) // 4 * 4
+    f32 = dict(dtype=torch.float32, device=dev)
+    q = torch.empty(P, L, BH, d.d_k, **f32)
+    k = torch.empty(P, L, BH, d.d_k, **f32)
+    v = torch.empty(P, L, BH, d.d_v, **f32)
+    kda = d.form == S.SEED_KDA
+    alpha = torch.empty(P, L, BH, d.d_k, **f32) if kda else torch.empty(P, L, BHp, **f32)
+    beta = torch.empty(P, L, BHp, **f32)
+    for t in range(P):
+        for l in range(L):
+            al = alpha[t, l] if kda else alpha[t, l, :BH]
+            S.seed_synth_token_inputs(d, run.key, S.SEED_PHASE_DECODE, t, l, run.vbar, q[t, l], k[t, l],
+                                      v[t, l], al, beta[t, l, :BH])
+    o = torch.empty(L, BH, d.d_v, **f32)
+    stream = torch.cuda.current_stream(dev)
+
+    def inputs(t, l):
+        return (q[t, l], k[t, l], v[t, l], alpha[t, l] if kda else alpha[t, l, :BH], beta[t, l, :BH])
+
+    def one_step(s, ev=None):
+        t = s % P
+        for l in range(L):
+            qq, kk, vv, aa, bb = inputs(t, l)
+            if ev is not None:
+                ev["dec"].append((torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+                                  run.c))
+                ev["dec"][-1][0].record(stream)
+            S.seed_decode_step(d, run.state, l, qq, kk, vv, aa, bb, o[l], run.ws, stream)
+            if ev is not None:
+                ev["dec"][-1][1].record(stream)
+        run.c += 1
+        if run.c == d.m:
+            if ev is not None:
+                ev["cmp"].append((torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)))
+                ev["cmp"][-1][0].record(stream)
+            S.seed_compress(d, run.state, S.SEED_ALL_LAYERS, run.ws, stream=stream)
+            if ev is not None:
+                ev["cmp"][-1][1].record(stream)
+            run.c = d.R
+
+    for s in range(args.warmup):
+        one_step(s)
+    torch.cuda.synchronize()
+    flags_warm = S.seed_get_status(run.ws)
+
+    ev = {"dec": [], "cmp": []}
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    visible = [x for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
+    gpu_index = int(visible[local]) if len(visible) > local and visible[local].isdigit() else local
+    barrier(world, dev)
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_index, enabled=not args.no_clocks) as clk:
+        start.record(stream)
+        for s in range(args.steps):
+            one_step(args.warmup + s, ev)
+        end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world, dev)
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), world, dev)
+    flags = S.seed_get_status(run.ws)
+
+    units = d.units
+    value = args.steps * units * world / (elapsed_ms / 1e3)
+    dec_ms = [a.elapsed_time(b) for a, b, _ in ev["dec"]]
+    dec_bytes = [BH * roofline.lazy_bytes(d.form, d.d_k, d.d_v, c) for _, _, c in ev["dec"]]
+    cmp_ms = [a.elapsed_time(b) for a, b in ev["cmp"]]
+    dec_gbs = sum(dec_bytes) / (sum(dec_ms) / 1e3) / 1e9
+    peak, peak_kind = measured_peak_hbm()
+    cbar = roofline.mean_columns(d.R, d.W)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded Philox4x32-10 inputs and prefill, generated on the device)",
+        "config": config_obj(cfg, B, world, prefill),
+        "roofline": {"bound": "hbm", "kernel": "decode_step_kernel", "achieved": dec_gbs, "peak": peak,
+                     "unit": "GB/s", "frac": dec_gbs / peak, "peak_source": f"{peak_kind} copy bandwidth",
+                     "frac_of_nominal_8TBs": dec_gbs / NOMINAL_HBM_GBS, "traffic": None,
+                     "algorithmic_bytes_per_head_step_mean": roofline.lazy_bytes(d.form, d.d_k, d.d_v, cbar),
+                     "avg_launch_us": 1e3 * sum(dec_ms) / len(dec_ms), "launches": len(dec_ms)},
+        "decode_only": {"head_steps_per_s": len(dec_ms) * BH * world / (sum(dec_ms) / 1e3),
+                        "GBps": dec_gbs},
+        "compress": {"launches": len(cmp_ms), "ms_per_launch": (sum(cmp_ms) / len(cmp_ms)) if cmp_ms else None,
+                     "ns_per_head_step_amortized": 1e6 * sum(cmp_ms) / (args.steps * units) if cmp_ms else 0.0,
+                     "share_of_step": sum(cmp_ms) / elapsed_ms},
+        "gpu_launches": len(dec_ms) + len(cmp_ms),
+        "status_flags": flags | flags_warm,
+        "setup_s": t_setup,
+    }
+    clocks = clk.summary()
+    line["clocks"] = clocks
+
+    # ---- dense comparison on the same inputs
+    if not args.no_dense and run.dense is not None:
+        dev_ms = []
+        od = torch.empty(BH, d.d_v, **f32)
+        for s in range(2):
+            for l in range(L):
+                S.seed_dense_step(d, run.dense, l, *inputs(s % P, l), od, run.ws, stream)
+        torch.cuda.synchronize()
+        for s in range(args.dense_steps):
+            for l in range(L):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                S.seed_dense_step(d, run.dense, l, *inputs(s % P, l), od, run.ws, stream)
+                e1.record(stream)
+                dev_ms.append((e0, e1))
+        torch.cuda.synchronize()
+        dms = [a.elapsed_time(b) for a, b in dev_ms]
+        dense_hs = len(dms) * BH / (sum(dms) / 1e3)
+        dense_gbs = len(dms) * BH * roofline.dense_bytes(d.d_k, d.d_v) / (sum(dms) / 1e3) / 1e9
+        line["dense"] = {"head_steps_per_s": dense_hs * world, "GBps": dense_gbs, "frac": dense_gbs / peak,
+                         "bytes_per_head_step": roofline.dense_bytes(d.d_k, d.d_v)}
+        line["speedup_vs_dense"] = {
+            "decode_only": line["decode_only"]["head_steps_per_s"] / line["dense"]["head_steps_per_s"],
+            "with_compress": value / line["dense"]["head_steps_per_s"],
+            "byte_ratio_lazy": roofline.dense_bytes(d.d_k, d.d_v) / roofline.lazy_bytes(d.form, d.d_k, d.d_v, cbar),
+            "byte_ratio_explicit": roofline.dense_bytes(d.d_k, d.d_v) / roofline.explicit_bytes(d.d_k, d.d_v, cbar)}
+        del run.dense
+        run.dense = None
+        torch.cuda.empty_cache()
+
+    # ---- end to end: host inputs in pinned memory, copies inside the timed region
+    if not args.no_e2e:
+        Ph = 2
+        hq = torch.empty(Ph, L, BH, d.d_k, dtype=torch.float32, pin_memory=True)
+        hk = torch.empty_like(hq, pin_memory=True)
+        hv = torch.empty(Ph, L, BH, d.d_v, dtype=torch.float32, pin_memory=True)
+        ha = torch.empty(Ph, *alpha.shape[1:], dtype=torch.float32, pin_memory=True)
+        hb = torch.empty(Ph, *beta.shape[1:], dtype=torch.float32, pin_memory=True)
+        for t in range(Ph):
+            hq[t].copy_(q[t]); hk[t].copy_(k[t]); hv[t].copy_(v[t]); ha[t].copy_(alpha[t]); hb[t].copy_(beta[t])
+        ho = torch.empty(L, BH, d.d_v, dtype=torch.float32, pin_memory=True)
+        sq, sk, sv = torch.empty_like(q[0, 0]), torch.empty_like(k[0, 0]), torch.empty_like(v[0, 0])
+        sa, sb = torch.empty_like(alpha[0, 0]), torch.empty_like(beta[0, 0])
+        h2d = L * (sq.numel() + sk.numel() + sv.numel() + sa.numel() + sb.numel()) * 4   # as copied
+        d2h = o.numel() * 4
+        torch.cuda.synchronize()
+        barrier(world, dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for s in range(args.e2e_steps):
+            t = s % Ph
+            for l in range(L):
+                sq.copy_(hq[t, l], non_blocking=True); sk.copy_(hk[t, l], non_blocking=True)
+                sv.copy_(hv[t, l], non_blocking=True); sa.copy_(ha[t, l], non_blocking=True)
+                sb.copy_(hb[t, l], non_blocking=True)
+                S.seed_decode_step(d, run.state, l, sq, sk, sv, sa if kda else sa[:BH], sb[:BH], o[l],
+                                   run.ws, stream)
+            run.c += 1
+            if run.c == d.m:
+                S.seed_compress(d, run.state, S.SEED_ALL_LAYERS, run.ws, stream=stream)
+                run.c = d.R
+            ho.copy_(o, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world, dev)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        line["e2e"] = {"value": args.e2e_steps * units * world / (e2e_ms / 1e3), "unit": UNIT,
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                       "note": "pinned host buffers; every step copies its inputs in and its o out"}
+        line["status_flags"] |= S.seed_get_status(run.ws)
+
+    if rank == 0 and world == 1 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_oracle_rate(cfg, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None) -> int:
+    args = parse_args(argv)
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            return run_reference(args, world, rank)
+        return run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            if dist.is_initialized():
+                dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

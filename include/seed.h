@@ -1,0 +1,194 @@
+/*
+ * seed.h -- C ABI of the sink-plus-low-rank recurrent-state decode path (libseed.so).
+ *
+ * What the library computes ("Shallow Encoding Emits Deep Memories", SEED):
+ * each per-head d_k x d_v recurrent state of a Gated DeltaNet, Kimi Delta
+ * Attention or Mamba-2 layer is stored as
+ *
+ *     S = a vbar^T + U V^T                                              (1)
+ *
+ * (SEED summary (picx.dev), Methodology, "SEED Architecture": decode, shallow in
+ * representation), where vbar (d_v) is a fixed per-head direction shared by all
+ * requests, a (d_k) the sink coefficient and U (d_k x c), V (d_v x c) the content
+ * factors.  A decode step reads out o = S^T q, applies the exact factored update
+ * (same page, "Exact Update (Lemma 2)"; the sink split of Lemma 1 under
+ * "Theoretical and Practical Implications"), and appends one column pair; every
+ * W steps the factors are compressed back to rank R (SEED figures & tables
+ * (thelatestinai.com), Figure 1(b) and Table 1).
+ *
+ * Conventions shared by every entry point
+ *  - Memory: every pointer is a DEVICE pointer owned by the caller.  The library
+ *    never allocates, frees or keeps a pointer after a call returns.
+ *  - Alignment: every array pointer must be 16-byte aligned (float4 access).
+ *  - Streams: `stream` is a cudaStream_t (NULL = the legacy default stream).
+ *    Calls only enqueue work and return; they never synchronise, except
+ *    seed_get_status.
+ *  - Errors: arguments are validated on the host before anything is enqueued;
+ *    a negative seed_status is returned and nothing is launched.  Conditions
+ *    that only the device can see set bits in the status word that lives in the
+ *    caller's workspace; kernels never trap.  Read them with seed_get_status.
+ *  - Units: one unit is one (request b, layer l, head h).  State arrays are
+ *    request-major: unit index u = ((b * layers) + l) * heads + h.
+ *  - Precision: float32 storage and arithmetic throughout.
+ */
+#ifndef SEED_H_
+#define SEED_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Recurrent-layer forms.  Dense recurrences (orientation d_k x d_v, o = S^T q):
+ *   SEED_GDN     S+ = g (I - beta k k^T) S + beta k v^T
+ *   SEED_KDA     S+ = (I - beta k k^T) Diag(alpha) S + beta k v^T
+ *   SEED_MAMBA2  S+ = alpha S + Delta k v^T   (k = B_t, v = x_t; d_k = d_state, d_v = headdim,
+ *                the orientation of SEED figures & tables, Table 17)                         */
+typedef enum { SEED_GDN = 0, SEED_KDA = 1, SEED_MAMBA2 = 2 } seed_form;
+
+/* Host-side return codes. */
+typedef enum {
+  SEED_OK = 0,
+  SEED_ERR_INVALID_ARG = -1, /* null pointer, bad enum, non-positive size, layer out of range */
+  SEED_ERR_SHAPE = -2,       /* unsupported d_k / d_v / R / W combination                    */
+  SEED_ERR_ALIGN = -3,       /* a pointer is not 16-byte aligned                             */
+  SEED_ERR_CUDA = -4,        /* a CUDA runtime call or kernel launch failed                  */
+  SEED_ERR_WORKSPACE = -5    /* workspace missing or smaller than seed_workspace_bytes       */
+} seed_status;
+
+/* Device-side status bits, accumulated in the workspace, read by seed_get_status. */
+#define SEED_FLAG_FULL 0x1u       /* decode_step met a unit already holding R+W columns;
+                                     that unit was left unchanged and its o not written    */
+#define SEED_FLAG_NONFINITE 0x2u  /* a non-finite value was produced                       */
+#define SEED_FLAG_NOCONVERGE 0x4u /* a Jacobi SVD reached its sweep cap                     */
+#define SEED_FLAG_BADCOLS 0x8u    /* a unit's column count was outside [0, R+W]            */
+#define SEED_FLAG_ZERO_VBAR 0x10u /* a head's vbar has zero norm; its units were left
+                                     unchanged (decode_step also leaves o unwritten)      */
+#define SEED_FLAG_BADINDEX 0x20u  /* seed_state_to_dense met a unit index outside the scope;
+                                     that output slab was not written                      */
+#define SEED_FLAG_TIMEOUT 0x40u   /* a bounded wait for a bulk copy gave up (1 s); the unit
+                                     was left unchanged                                    */
+
+/* Supported shapes: (d_k, d_v) equal and in {16, 32, 64, 128}, or (128, 64), or
+ * (64, 128); R >= 1, W >= 1, R + W <= SEED_MAX_COLS and R + W <= min(d_k, d_v).
+ * Anything else returns SEED_ERR_SHAPE. */
+#define SEED_MAX_COLS 96
+#define SEED_ALL_LAYERS (-1)
+
+/* Problem dimensions: batch of requests x layers x heads, head dims, rank, window. */
+typedef struct {
+  int32_t form;   /* seed_form */
+  int32_t batch;  /* requests B */
+  int32_t layers; /* recurrent layers L */
+  int32_t heads;  /* heads per layer H */
+  int32_t d_k;    /* key / state dimension */
+  int32_t d_v;    /* value dimension */
+  int32_t R;      /* rank kept after a compression */
+  int32_t W;      /* steps between compressions; a unit holds at most R + W columns */
+} seed_dims;
+
+/* The stored state of all B x L x H units (device pointers, caller-owned).
+ *   a      [B][L][H][d_k]            sink coefficient a
+ *   U      [B][L][H][R+W][d_k]       content factor U, one contiguous d_k column per slot;
+ *                                    slot j holds column j, so appends never move data
+ *   V      [B][L][H][R+W][d_v]       content factor V, same slots
+ *   scale  GDN, Mamba-2: [B][L][H][R+W] per-column decay scales gamma_j: the true U
+ *                                    column j is gamma_j * U[:, j] (decay applied lazily)
+ *          KDA:          [B][L][H][d_k] per-channel decay products P: the true U is
+ *                                    Diag(P) U (per-row decay applied lazily)
+ *   ncols  [B][L][H] int32            columns held, R <= ncols <= R+W after a conversion
+ *   vbar   [L][H][d_v]                per-head mean value, shared by all requests
+ * The represented dense state of a unit is (1) with the true U; seed_state_to_dense
+ * returns it.  seed_scale_len() gives the per-unit length of `scale`.               */
+typedef struct {
+  float* a;
+  float* U;
+  float* V;
+  float* scale;
+  int32_t* ncols;
+  const float* vbar;
+} seed_state;
+
+/* Per-unit length of seed_state.scale: R+W for GDN and Mamba-2, d_k for KDA. */
+int32_t seed_scale_len(const seed_dims* dims);
+
+/* Bytes of device workspace every call below needs (the device status word).
+ * Zero it once with seed_workspace_init before first use. */
+size_t seed_workspace_bytes(const seed_dims* dims);
+int seed_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* End-of-prefill conversion (SEED figures & tables, Figure 1(a) and Table 1: the
+ * states the prefill leaves are compressed to the shallow form; SEED summary,
+ * Lemma 1: the split along vbar).  For every unit of `layer` (or of all layers
+ * with SEED_ALL_LAYERS):
+ *     a = S vbar / ||vbar||^2,   C = S - a vbar^T,   U V^T = best rank-R approximation of C
+ * with Sigma^{1/2} on each side (one-sided Jacobi SVD of C); scale <- 1; ncols <- R.
+ * Columns of a rank-deficient C are zero.
+ *   S_dense    [B][H][d_k][d_v] row-major for one layer, [B][L][H][d_k][d_v] for all
+ *   sigma_out  optional (may be NULL): the kept singular values, [units in scope][R]
+ * A unit whose vbar is zero is left unchanged and raises SEED_FLAG_ZERO_VBAR.          */
+int seed_state_init_from_dense(const seed_dims* dims, const seed_state* state, int32_t layer,
+                               const float* S_dense, float* sigma_out, void* ws, size_t ws_bytes,
+                               void* stream);
+
+/* One exact decode step of one layer for all B x H units, then the read-out
+ * (SEED summary, "Exact Update (Lemma 2)" and Lemma 1; read-out o = S+^T q with
+ * S+ the updated state).  For Gated DeltaNet, with omega = v^T vbar / ||vbar||^2 and
+ * eps = v - omega vbar:
+ *     a+ = g a + beta (omega - g k^T a) k
+ *     U+ = [g U, k],   V+ = [V, beta (eps - g V U^T k)]
+ *     o  = vbar (a+^T q) + V+ (U+^T q)
+ * KDA applies Diag(alpha) on the key side before the erase; Mamba-2 has no erase
+ * and writes with Delta (V+ = [V, Delta eps]).  The new column pair goes to slot
+ * ncols, which then grows by one.  A unit already at R+W columns is skipped and
+ * SEED_FLAG_FULL is raised: call seed_compress after the step that fills R+W.
+ *   q, k   [B][H][d_k]           v, o [B][H][d_v]
+ *   alpha  GDN: decay g [B][H];  KDA: per-channel decay [B][H][d_k];  Mamba-2: alpha [B][H]
+ *   beta   GDN, KDA: write strength [B][H];  Mamba-2: Delta [B][H]                        */
+int seed_decode_step(const seed_dims* dims, const seed_state* state, int32_t layer,
+                     const float* q, const float* k, const float* v, const float* alpha,
+                     const float* beta, float* o, void* ws, size_t ws_bytes, void* stream);
+
+/* Periodic compression (SEED figures & tables, Figure 1(b): every W steps the
+ * factors are compressed back to rank R; SEED summary, Corollary 4 bounds its
+ * open-loop error).  For every unit of `layer` (or all layers) whose ncols equals
+ * R+W: QR of U and V by Cholesky of the column-equilibrated Gram matrices, the
+ * (R+W) x (R+W) core M = R_u R_v^T, a one-sided Jacobi SVD of M, and
+ *     U' = Q_u X_R Sigma_R^{1/2},   V' = Q_v Y_R Sigma_R^{1/2}
+ * written to slots 0..R-1; scale <- 1; ncols <- R.  The sink a is not touched.
+ * Units with ncols != R+W are left unchanged.
+ *   sigma_out  optional: [units in scope][R] singular values kept (only compressed
+ *              units' rows are written)                                              */
+int seed_compress(const seed_dims* dims, const seed_state* state, int32_t layer,
+                  float* sigma_out, void* ws, size_t ws_bytes, void* stream);
+
+/* Dense state S = a vbar^T + U V^T (true U, scales applied) of units of `layer`
+ * (or all layers).  units: optional list of unit indices within the scope
+ * (b * H + h for one layer, the global unit index for all layers); NULL = every
+ * unit in scope.  S_out [n][d_k][d_v] row-major.                                */
+int seed_state_to_dense(const seed_dims* dims, const seed_state* state, int32_t layer,
+                        const int32_t* units, int32_t n_units, float* S_out, void* ws,
+                        size_t ws_bytes, void* stream);
+
+/* The dense-state step that SEED replaces, kept as the in-run comparison: every
+ * decode step loads and stores whole recurrent states (SEED abstract, readsearch.ai).
+ * One step of `layer` on a dense state S [B][L][H][d_k][d_v] with the form's dense
+ * recurrence, then o = S+^T q.  Arguments as in seed_decode_step.                  */
+int seed_dense_step(const seed_dims* dims, float* S, int32_t layer, const float* q,
+                    const float* k, const float* v, const float* alpha, const float* beta,
+                    float* o, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, returns the accumulated SEED_FLAG_* bits in *flags and
+ * clears them.  Returns SEED_OK or SEED_ERR_CUDA.                                   */
+int seed_get_status(void* ws, void* stream, uint32_t* flags);
+
+/* Static description of a seed_status code. */
+const char* seed_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SEED_H_ */

@@ -28,7 +28,8 @@ def run_units(cfg, b, l, h, n_prefill=None, n_decode=None, keep_shadow=True):
     Keys: o (T, n, d_v); a_t (T, n, d_k); ncols (T,) after each step;
     comp_steps (list of 1-based steps after which a compression ran);
     sigma (n_comp, n, R) kept singular values; gap (n_comp, n) relative gap at R;
-    tail (n_comp + 1, n) discarded tail norm (conversion first);
+    tail (n_comp + 1, n) discarded tail norm (conversion first); S_conv the state
+    right after the conversion;
     a, U, V final factors; S final reconstructed state; S0 the prefill state;
     and, with keep_shadow, S_exact (final open-loop dense state),
     err_open (T, n) ||S~_t - S_t^exact||_F and sink_dev (T, n) max |a_t - sink(S_t^exact)|.
@@ -39,7 +40,7 @@ def run_units(cfg, b, l, h, n_prefill=None, n_decode=None, keep_shadow=True):
     vb = philox.vbar(cfg, l, h).astype(np.float64)
     a, U, V, s0 = convert.convert(S0, vb, cfg.R)
     out = {"S0": S0, "vbar": vb, "conv_sigma": s0[:, :cfg.R].copy(),
-           "conv_gap": compress.rel_gap(s0, cfg.R)}
+           "conv_gap": compress.rel_gap(s0, cfg.R), "S_conv": factored.reconstruct(a, U, V, vb)}
     tails = [compress.tail_norm(s0, cfg.R)]
     S_exact = S0.copy()
     o_all, a_all, ncols_all, sig, gaps, comp_steps = [], [], [], [], [], []

@@ -1,0 +1,41 @@
+// seed_launch.h -- host launchers behind the C ABI (internal to libseed).
+// Arguments are validated by seed_abi.cu before any of these is called.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/seed.h"
+#include "../../include/seed_synth.h"
+
+namespace seed {
+
+bool decode_dims_supported(int dk, int dv);
+
+int launch_decode_step(const seed_dims& d, const seed_state& s, int layer, const float* q,
+                       const float* k, const float* v, const float* alpha, const float* beta,
+                       float* o, uint32_t* status, cudaStream_t st);
+
+int launch_compress(const seed_dims& d, const seed_state& s, int layer, float* sigma_out,
+                    uint32_t* status, cudaStream_t st);
+
+int launch_init_from_dense(const seed_dims& d, const seed_state& s, int layer, const float* S,
+                           float* sigma_out, uint32_t* status, cudaStream_t st);
+
+int launch_to_dense(const seed_dims& d, const seed_state& s, int layer, const int32_t* units,
+                    int n_units, float* S_out, uint32_t* status, cudaStream_t st);
+
+int launch_dense_step(const seed_dims& d, float* S, int layer, const float* q, const float* k,
+                      const float* v, const float* alpha, const float* beta, float* o,
+                      uint32_t* status, cudaStream_t st);
+
+int launch_synth_vbar(const seed_dims& d, const seed_synth_key& key, float* vbar, cudaStream_t st);
+
+int launch_synth_token_inputs(const seed_dims& d, const seed_synth_key& key, int phase, int t,
+                              int layer, const float* vbar, float* q, float* k, float* v,
+                              float* alpha, float* beta, cudaStream_t st);
+
+int launch_synth_dense_prefill(const seed_dims& d, const seed_synth_key& key, int n_tokens,
+                               int layer, const float* vbar, float* S_out, cudaStream_t st);
+
+}  // namespace seed

@@ -1,0 +1,55 @@
+"""Algorithmic byte accounting of the decode step (host logic for measurement).
+
+Per head-step (one unit, one decode step, c columns held before the step), fp32:
+
+  lazy (the layout libseed uses)
+    GDN, Mamba-2  4 [ d_k + (d_k + d_v + 1) c + d_k + d_k + d_v + (c + 1) ]
+                  read a, the c columns of U and V and their c decay scales;
+                  write a, one U column, one V column and c + 1 scales
+    KDA           4 [ d_k + (d_k + d_v) c + d_k + d_k + d_v + 2 d_k ]
+                  the per-channel decay product P (d_k) is read and written
+                  instead of the column scales
+  explicit        4 [ d_k + (d_k + d_v) c + d_k + d_k c + d_k + d_v ]
+                  (U rewritten in full every step)
+  table2          2 * 4 [ d_k + (d_k + d_v) (R + W/2) ]  (every state read and
+                  written in full at the mean column count, the Table 2 traffic
+                  convention of "Shallow Encoding Emits Deep Memories")
+  dense           2 * 4 d_k d_v
+
+The shared v̄ is not counted (Table 17 of the same page), nor are the per-step
+inputs q, k, v, alpha, beta and the output o, nor the 8 bytes of the per-unit
+column counter.
+"""
+
+from __future__ import annotations
+
+FORM_KDA = 1
+
+
+def lazy_bytes(form: int, d_k: int, d_v: int, c: float) -> float:
+    if form == FORM_KDA:
+        return 4.0 * (d_k + (d_k + d_v) * c + d_k + d_k + d_v + 2 * d_k)
+    return 4.0 * (d_k + (d_k + d_v + 1) * c + d_k + d_k + d_v + (c + 1))
+
+
+def explicit_bytes(d_k: int, d_v: int, c: float) -> float:
+    return 4.0 * (d_k + (d_k + d_v) * c + d_k + d_k * c + d_k + d_v)
+
+
+def table2_bytes(d_k: int, d_v: int, R: int, W: int) -> float:
+    return 2 * 4.0 * (d_k + (d_k + d_v) * (R + W / 2))
+
+
+def dense_bytes(d_k: int, d_v: int) -> float:
+    return 2 * 4.0 * d_k * d_v
+
+
+def io_bytes(form: int, d_k: int, d_v: int) -> float:
+    """Per-step inputs and output of one unit: q, k, v, alpha, beta, o."""
+    alpha = d_k if form == FORM_KDA else 1
+    return 4.0 * (2 * d_k + 2 * d_v + alpha + 1)
+
+
+def mean_columns(R: int, W: int) -> float:
+    """Mean column count before a step over one compression window: R + (W - 1) / 2."""
+    return R + (W - 1) / 2.0

@@ -1,0 +1,104 @@
+"""Helpers for the GPU parity tests: run the device path and the oracle on the same
+seeded workload and compare what the method fixes.
+
+The device side goes only through the C ABI (rank_recurrent_state_b200.seed and
+.pipeline); the oracle side only through oracle/ with inputs from workloads/.
+Nothing computed on the device is ever fed to the oracle.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+TOL = 1e-4          # relative Frobenius error, fp32 device vs fp64 oracle
+GAP_TOL = 1e-5      # units with a relative singular gap at R below this are near-ties
+
+
+def rel_fro(x, y) -> float:
+    x = np.asarray(x, dtype=np.float64)
+    y = np.asarray(y, dtype=np.float64)
+    den = np.linalg.norm(y)
+    return float(np.linalg.norm(x - y) / (den if den > 0 else 1.0))
+
+
+def ensure_lib():
+    import torch
+    from rank_recurrent_state_b200 import build
+    build.build()
+    assert torch.cuda.is_available(), "GPU tests need CUDA"
+
+
+def run_device(cfg, sample_units, n_prefill, n_decode, batch=None):
+    """Run prefill, conversion and n_decode steps of every unit of (cfg, batch) on the
+    device; return the trajectories of the sampled global units as numpy arrays."""
+    import torch
+    from rank_recurrent_state_b200 import seed as S
+    from rank_recurrent_state_b200.pipeline import DeviceRun
+
+    run = DeviceRun(cfg, batch=batch, n_prefill=n_prefill)
+    d = run.dims
+    run.prefill_and_convert()
+    su = np.asarray(sample_units, dtype=np.int64)
+    b, rem = np.divmod(su, d.layers * d.heads)
+    l, h = np.divmod(rem, d.heads)
+    buf = S.alloc_step_inputs(d, run.device)
+    outs = [None] * d.layers
+    sig = torch.empty(d.units, d.R, dtype=torch.float32, device=run.device)
+    o_traj, ncols_traj, sig_traj, comp_steps = [], [], [], []
+    conv = run.sigma_conv.reshape(-1, d.R)[torch.as_tensor(su, device=run.device)].cpu().numpy()
+    S0 = run.to_dense(torch.as_tensor(su, dtype=torch.int32, device=run.device)).cpu().numpy()
+    for t in range(n_decode):
+        fired = run.step(buf, outs=outs, sigma=sig)
+        o = np.stack([outs[li][bi, hi].cpu().numpy() for bi, li, hi in zip(b, l, h)])
+        o_traj.append(o)
+        ncols_traj.append(run.state.ncols.reshape(-1)[torch.as_tensor(su, device=run.device)].cpu().numpy())
+        if fired:
+            comp_steps.append(t + 1)
+            sig_traj.append(sig[torch.as_tensor(su, device=run.device)].cpu().numpy())
+    torch.cuda.synchronize()
+    units_t = torch.as_tensor(su, dtype=torch.int32, device=run.device)
+    S_fin = run.to_dense(units_t).cpu().numpy()
+    a_fin = run.state.a.reshape(-1, d.d_k)[units_t.long()].cpu().numpy()
+    flags = run.status()
+    return dict(o=np.array(o_traj), ncols=np.array(ncols_traj), sigma=np.array(sig_traj),
+                comp_steps=comp_steps, S=S_fin, a=a_fin, S_conv=S0, conv_sigma=conv, flags=flags,
+                b=b, l=l, h=h)
+
+
+def run_oracle(cfg, dev, n_prefill, n_decode):
+    from oracle import run as orun
+    return orun.run_units(cfg, dev["b"], dev["l"], dev["h"], n_prefill=n_prefill, n_decode=n_decode,
+                          keep_shadow=False)
+
+
+def compare(cfg, dev, ref, tol=TOL):
+    """Per-unit and pooled relative Frobenius errors; near-tie units are reported and
+    excluded from the per-unit check only.  Returns a dict of the measured errors."""
+    n = dev["o"].shape[1]
+    gaps = [ref["conv_gap"]] + ([ref["gap"][i] for i in range(ref["gap"].shape[0])])
+    min_gap = np.min(np.stack(gaps), axis=0)
+    ties = min_gap < GAP_TOL
+    errs = {"o": [], "S": [], "sigma": [], "a": []}
+    for u in range(n):
+        errs["o"].append(rel_fro(dev["o"][:, u], ref["o"][:, u]))
+        errs["S"].append(rel_fro(dev["S"][u], ref["S"][u]))
+        errs["a"].append(rel_fro(dev["a"][u], ref["a"][u]))
+        if dev["sigma"].size:
+            errs["sigma"].append(rel_fro(dev["sigma"][:, u], ref["sigma"][:, u]))
+    out = {k: np.array(v) for k, v in errs.items()}
+    out["ties"] = int(ties.sum())
+    out["pooled_o"] = rel_fro(dev["o"], ref["o"])
+    out["pooled_S"] = rel_fro(dev["S"], ref["S"])
+    out["pooled_sigma"] = rel_fro(dev["sigma"], ref["sigma"]) if dev["sigma"].size else 0.0
+    out["conv_S"] = np.array([rel_fro(dev["S_conv"][u], ref["S_conv"][u]) for u in range(n)])
+    out["conv_sigma"] = np.array([rel_fro(dev["conv_sigma"][u], ref["conv_sigma"][u]) for u in range(n)])
+    # bookkeeping must be bit-exact
+    assert dev["comp_steps"] == ref["comp_steps"], (dev["comp_steps"], ref["comp_steps"])
+    np.testing.assert_array_equal(dev["ncols"], np.repeat(ref["ncols"][:, None], n, axis=1))
+    for key in ("o", "S", "a", "sigma", "conv_S", "conv_sigma"):
+        if out[key].size:
+            assert np.all(out[key][~ties] <= tol), (key, out[key])
+    for key in ("pooled_o", "pooled_S", "pooled_sigma"):
+        assert out[key] <= tol, (key, out[key])
+    return out
+

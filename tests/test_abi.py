@@ -1,0 +1,127 @@
+"""The C ABI without a GPU: libseed.so loads, exports every function the headers
+declare, and rejects bad arguments on the host before anything is enqueued."""
+
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from rank_recurrent_state_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*[A-Za-z_][\w\s\*]*?\b(seed_\w+)\s*\(", text, flags=re.M):
+            names.add(m.group(1))
+    return names
+
+
+def test_headers_declare_the_entry_points():
+    names = _declared_functions()
+    for n in ("seed_state_init_from_dense", "seed_decode_step", "seed_compress",
+              "seed_state_to_dense", "seed_dense_step", "seed_get_status", "seed_workspace_bytes",
+              "seed_synth_token_inputs", "seed_synth_dense_prefill", "seed_synth_vbar"):
+        assert n in names
+
+
+def test_library_exports_every_declared_function(lib):
+    names = _declared_functions()
+    assert names
+    for n in sorted(names):
+        assert hasattr(lib, n), n
+        assert n in _lib.SIGNATURES, f"binding lacks {n}"
+
+
+def _dims(**kw):
+    base = dict(form=0, batch=2, layers=3, heads=4, d_k=128, d_v=128, R=16, W=16)
+    base.update(kw)
+    return _lib.seed_dims(**base)
+
+
+A = 0x10000          # fake, aligned device addresses: never dereferenced on error paths
+MIS = 0x10004        # misaligned
+
+
+def _state(**kw):
+    base = dict(a=A, U=A, V=A, scale=A, ncols=A, vbar=A)
+    base.update(kw)
+    return _lib.seed_state(**base)
+
+
+def test_status_strings(lib):
+    assert lib.seed_status_string(0) == b"ok"
+    for code in (-1, -2, -3, -4, -5):
+        assert lib.seed_status_string(code) != b"unknown status"
+
+
+def test_scale_len_and_workspace(lib):
+    d = _dims()
+    assert lib.seed_scale_len(ctypes.byref(d)) == 32
+    dk = _dims(form=1)
+    assert lib.seed_scale_len(ctypes.byref(dk)) == 128
+    assert lib.seed_workspace_bytes(ctypes.byref(d)) >= 4
+    bad = _dims(d_k=48)
+    assert lib.seed_scale_len(ctypes.byref(bad)) == -1
+
+
+@pytest.mark.parametrize("dims,code", [
+    (None, -1),
+    (_dims(form=3), -1),
+    (_dims(batch=0), -1),
+    (_dims(R=0), -1),
+    (_dims(d_k=48), -2),
+    (_dims(d_k=256, d_v=256), -2),
+    (_dims(d_k=16, d_v=16, R=8, W=16), -2),     # R + W > d
+    (_dims(R=64, W=64), -2),                    # R + W > SEED_MAX_COLS
+])
+def test_decode_step_rejects_bad_dims(lib, dims, code):
+    d = ctypes.byref(dims) if dims is not None else None
+    s = _state()
+    rc = lib.seed_decode_step(d, ctypes.byref(s), 0, A, A, A, A, A, A, A, 256, None)
+    assert rc == code
+
+
+def test_decode_step_rejects_bad_pointers_and_layer(lib):
+    d, s = _dims(), _state()
+    call = lambda layer=0, st=s, q=A, ws=A, wsb=256: lib.seed_decode_step(  # noqa: E731
+        ctypes.byref(d), ctypes.byref(st), layer, q, A, A, A, A, A, ws, wsb, None)
+    assert call(layer=3) == -1
+    assert call(layer=-1) == -1                  # all layers is not a decode step
+    assert call(q=None) == -1
+    assert call(q=MIS) == -3
+    assert call(st=_state(U=MIS)) == -3
+    assert call(st=_state(ncols=None)) == -1
+    assert call(ws=None) == -5
+    assert call(wsb=8) == -5
+
+
+def test_other_entry_points_validate(lib):
+    d, s = _dims(), _state()
+    assert lib.seed_compress(ctypes.byref(d), ctypes.byref(s), 5, None, A, 256, None) == -1
+    assert lib.seed_compress(ctypes.byref(d), ctypes.byref(s), 0, MIS, A, 256, None) == -3
+    assert lib.seed_state_init_from_dense(ctypes.byref(d), ctypes.byref(s), -1, None, None, A, 256,
+                                          None) == -1
+    assert lib.seed_state_to_dense(ctypes.byref(d), ctypes.byref(s), 0, A, 10**6, A, A, 256, None) == -1
+    assert lib.seed_state_to_dense(ctypes.byref(d), ctypes.byref(s), 0, A, 0, A, A, 256, None) == 0
+    assert lib.seed_dense_step(ctypes.byref(d), MIS, 0, A, A, A, A, A, A, A, 256, None) == -3
+    flags = _lib.c_uint32()
+    assert lib.seed_get_status(None, None, ctypes.byref(flags)) == -5
+    assert lib.seed_get_status(A, None, None) == -1
+    key = _lib.seed_synth_key(0, 0, 0, 0)
+    assert lib.seed_synth_token_inputs(ctypes.byref(d), key, 2, 0, 0, A, A, A, A, A, A, None) == -1
+    assert lib.seed_synth_dense_prefill(ctypes.byref(d), key, -1, 0, A, A, None) == -1
+    bad_key = _lib.seed_synth_key(0, 0, 0, -1)
+    assert lib.seed_synth_dense_prefill(ctypes.byref(d), bad_key, 4, 0, A, A, None) == -1
