@@ -339,6 +339,7 @@ def run_ours(args, world, rank, local):
     barrier(world, dev)
     elapsed_ms = max_over_ranks(start.elapsed_time(end), world, dev)
     flags = S.seed_get_status(run.ws)
+    diag = S.seed_get_diagnostics(run.ws)
 
     units = d.units
     value = args.steps * units * world / (elapsed_ms / 1e3)
@@ -364,7 +365,9 @@ def run_ours(args, world, rank, local):
                         "GBps": dec_gbs},
         "compress": {"launches": len(cmp_ms), "ms_per_launch": (sum(cmp_ms) / len(cmp_ms)) if cmp_ms else None,
                      "ns_per_head_step_amortized": 1e6 * sum(cmp_ms) / (args.steps * units) if cmp_ms else 0.0,
-                     "share_of_step": sum(cmp_ms) / elapsed_ms},
+                     "share_of_step": sum(cmp_ms) / elapsed_ms,
+                     "jacobi_sweeps_mean": (diag["compress_sweeps"] / diag["compress_units"]
+                                            if diag["compress_units"] else None)},
         "gpu_launches": len(dec_ms) + len(cmp_ms),
         "status_flags": flags | flags_warm,
         "setup_s": t_setup,

@@ -173,6 +173,20 @@ int seed_get_status(void* ws, void* stream, uint32_t* flags) {
   return SEED_OK;
 }
 
+int seed_get_diagnostics(void* ws, void* stream, uint32_t* counters) {
+  if (!counters) return SEED_ERR_INVALID_ARG;
+  SEED_TRY(check_ws(ws, kWorkspaceBytes));
+  cudaStream_t st = as_stream(stream);
+  uint32_t host[4] = {0, 0, 0, 0};
+  uint32_t* dev = status_word(ws) + 1;
+  if (cudaMemcpyAsync(host, dev, sizeof(host), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return SEED_ERR_CUDA;
+  if (cudaMemsetAsync(dev, 0, sizeof(host), st) != cudaSuccess) return SEED_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SEED_ERR_CUDA;
+  for (int i = 0; i < 4; ++i) counters[i] = host[i];
+  return SEED_OK;
+}
+
 const char* seed_status_string(int status) {
   switch (status) {
     case SEED_OK: return "ok";

@@ -99,9 +99,15 @@ SEED_DEV void block_uniforms(uint4 w, double u[4]) {
 //
 // n_cols must be even (callers pad with a zero column).  Called by all threads of
 // the block; each pair is handled by a group of G lanes (G a power of two <= 32).
+//
+// Columns whose squared norm is below 1e-10 ||A||_F^2 are treated as zero: their
+// pairs are not rotated.  Such columns are rounding noise (or exact zeros) once
+// n_cols exceeds the rank, and a relative threshold alone would keep rotating
+// them for ever; their contribution is below 1e-5 of ||A||_F.
+// Returns the number of sweeps run (max_sweeps + 1 if it did not converge).
 template <int NT>
-__device__ bool jacobi_svd(float* A, int lda, int n_rows, float* Z, int ldz, int n_cols, float tol,
-                           int max_sweeps, int* s_flag) {
+__device__ int jacobi_svd(float* A, int lda, int n_rows, float* Z, int ldz, int n_cols, float tol,
+                          int max_sweeps, float* s_red) {
   const int tid = threadIdx.x;
   const int npairs = n_cols / 2;
   int G = 32;
@@ -109,10 +115,21 @@ __device__ bool jacobi_svd(float* A, int lda, int n_rows, float* Z, int ldz, int
   const int groups = NT / G;
   const int grp = tid / G, gl = tid % G;
 
+  float f2 = 0.f;
+  for (int j = tid; j < n_cols * n_rows; j += NT) {
+    const float x = A[(j / n_rows) * lda + (j % n_rows)];
+    f2 = fmaf(x, x, f2);
+  }
+  f2 = group_sum<32>(f2);
+  if ((tid & 31) == 0) s_red[tid >> 5] = f2;
   for (int j = tid; j < n_cols * n_cols; j += NT) {
     const int col = j / n_cols, row = j % n_cols;
     Z[col * ldz + row] = (row == col) ? 1.f : 0.f;
   }
+  __syncthreads();
+  float frob2 = 0.f;
+  for (int w = 0; w < NT / 32; ++w) frob2 += s_red[w];
+  const float tiny = 1e-10f * frob2;
   __syncthreads();
 
   for (int sweep = 0; sweep < max_sweeps; ++sweep) {
@@ -147,7 +164,7 @@ __device__ bool jacobi_svd(float* A, int lda, int n_rows, float* Z, int ldz, int
           yy = group_sum_rt(yy, G);
           xy = group_sum_rt(xy, G);
         }
-        if (active && fabsf(xy) > tol * sqrtf(xx) * sqrtf(yy)) {
+        if (active && xx > tiny && yy > tiny && fabsf(xy) > tol * sqrtf(xx) * sqrtf(yy)) {
           rotated = 1;
           const float zeta = (yy - xx) / (2.f * xy);
           float t;
@@ -174,10 +191,9 @@ __device__ bool jacobi_svd(float* A, int lda, int n_rows, float* Z, int ldz, int
       }
       __syncthreads();
     }
-    if (!__syncthreads_or(rotated)) return true;
+    if (!__syncthreads_or(rotated)) return sweep + 1;
   }
-  (void)s_flag;
-  return false;
+  return max_sweeps + 1;
 }
 
 }  // namespace seed

@@ -250,7 +250,12 @@ __global__ void __launch_bounds__(NT) compress_kernel(const CompressParams p) {
   }
   __syncthreads();
   const float tol = 8.f * sqrtf((float)m) * 5.9604645e-8f;
-  const bool conv = jacobi_svd<NT>(sM, ldm, m, sZ, ldz, mp, tol, 40, nullptr);
+  const int sweeps = jacobi_svd<NT>(sM, ldm, m, sZ, ldz, mp, tol, 40, s_red);
+  const bool conv = sweeps <= 40;
+  if (tid == 0) {
+    atomicAdd(p.status + 1, (uint32_t)sweeps);
+    atomicAdd(p.status + 2, 1u);
+  }
   for (int j = tid; j < mp; j += NT) {
     float s2 = 0.f;
     for (int i = 0; i < m; ++i) s2 = fmaf(sM[j * ldm + i], sM[j * ldm + i], s2);
@@ -435,7 +440,12 @@ __global__ void __launch_bounds__(NT) init_kernel(const InitParams p) {
   }
   __syncthreads();
   const float tol = 8.f * sqrtf((float)DV) * 5.9604645e-8f;
-  const bool conv = jacobi_svd<NT>(sC, LDC, DV, sZ, LDZ, DK, tol, 60, nullptr);
+  const int sweeps = jacobi_svd<NT>(sC, LDC, DV, sZ, LDZ, DK, tol, 60, s_red);
+  const bool conv = sweeps <= 60;
+  if (tid == 0) {
+    atomicAdd(p.status + 3, (uint32_t)sweeps);
+    atomicAdd(p.status + 4, 1u);
+  }
   for (int j = tid; j < DK; j += NT) {
     float s2 = 0.f;
     for (int i = 0; i < DV; ++i) s2 = fmaf(sC[j * LDC + i], sC[j * LDC + i], s2);

@@ -194,6 +194,13 @@ def seed_get_status(ws: Workspace, stream=None) -> int:
     return int(flags.value)
 
 
+def seed_get_diagnostics(ws: Workspace, stream=None) -> dict:
+    c = (_lib.c_uint32 * 4)()
+    _check("seed_get_diagnostics", _lib.load().seed_get_diagnostics(ws.ptr, _stream(stream), c))
+    return {"compress_sweeps": c[0], "compress_units": c[1], "convert_sweeps": c[2],
+            "convert_units": c[3]}
+
+
 # ------------------------------------------------------------------ synthetic workloads
 
 def synth_key(cfg, b0: int = 0) -> _lib.seed_synth_key:
