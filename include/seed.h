@@ -94,8 +94,9 @@ typedef struct {
  *   U      [B][L][H][R+W][d_k]       content factor U, one contiguous d_k column per slot;
  *                                    slot j holds column j, so appends never move data
  *   V      [B][L][H][R+W][d_v]       content factor V, same slots
- *   scale  GDN, Mamba-2: [B][L][H][R+W] per-column decay scales gamma_j: the true U
- *                                    column j is gamma_j * U[:, j] (decay applied lazily)
+ *   scale  GDN, Mamba-2: [B][L][H][ceil4(R+W)] per-column decay scales gamma_j: the true
+ *                                    U column j is gamma_j * U[:, j] (decay applied lazily);
+ *                                    the per-unit stride is R+W rounded up to a multiple of 4
  *          KDA:          [B][L][H][d_k] per-channel decay products P: the true U is
  *                                    Diag(P) U (per-row decay applied lazily)
  *   ncols  [B][L][H] int32            columns held, R <= ncols <= R+W after a conversion
@@ -111,7 +112,8 @@ typedef struct {
   const float* vbar;
 } seed_state;
 
-/* Per-unit length of seed_state.scale: R+W for GDN and Mamba-2, d_k for KDA. */
+/* Per-unit length of seed_state.scale: R+W rounded up to a multiple of 4 for GDN and
+ * Mamba-2, d_k for KDA.  Returns -1 for unsupported dims. */
 int32_t seed_scale_len(const seed_dims* dims);
 
 /* Bytes of device workspace every call below needs (the device status word).

@@ -69,7 +69,7 @@ extern "C" {
 
 int32_t seed_scale_len(const seed_dims* dims) {
   if (check_dims(dims)) return -1;
-  return dims->form == SEED_KDA ? dims->d_k : dims->R + dims->W;
+  return seed::scale_len(*dims);
 }
 
 size_t seed_workspace_bytes(const seed_dims* dims) {

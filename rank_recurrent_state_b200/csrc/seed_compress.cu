@@ -19,60 +19,9 @@
 // columns are the rows of C), U = X_R Sigma^{1/2}, V = Y_R Sigma^{1/2}.
 #include "seed_common.cuh"
 #include "seed_launch.h"
+#include "seed_tma.cuh"
 
 namespace seed {
-
-// ------------------------------------------------------------------ TMA bulk copy
-SEED_DEV uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-SEED_DEV void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count));
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-SEED_DEV void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
-               "r"(bytes)
-               : "memory");
-}
-
-// global -> shared bulk copy completing on `bar` (no multicast); 16-byte aligned, bytes % 16 == 0
-SEED_DEV void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_addr(dst)),
-      "l"(src), "r"(bytes), "r"(smem_addr(bar))
-      : "memory");
-}
-
-SEED_DEV bool mbar_test_wait(uint64_t* bar, uint32_t phase) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
-      : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(phase)
-      : "memory");
-  return ok != 0;
-}
-
-SEED_DEV uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-  return t;
-}
-
-// Bounded wait: polls without blocking (with a short sleep between polls) and
-// gives up after `limit_ns` nanoseconds of wall time, returning false.
-SEED_DEV bool mbar_wait_bounded(uint64_t* bar, uint32_t phase, uint64_t limit_ns) {
-  const uint64_t t0 = global_ns();
-  while (!mbar_test_wait(bar, phase)) {
-    if (global_ns() - t0 > limit_ns) return false;
-    __nanosleep(64);
-  }
-  return true;
-}
-
-constexpr uint64_t kWaitLimit = 1000000000ull;   // 1 s
 
 // ------------------------------------------------------------------ Householder QR
 // In-place QR of an n x m panel A (column-major, lda = n, m <= n) by m Householder
@@ -162,7 +111,7 @@ struct CompressParams {
   int32_t* ncols;
   float* sigma_out;
   uint32_t* status;
-  int B, L, H, layer, R, W;  // layer < 0: all layers
+  int B, L, H, layer, R, W, slen;  // layer < 0: all layers
 };
 
 template <int NT>
@@ -198,7 +147,7 @@ __global__ void __launch_bounds__(NT) compress_kernel(const CompressParams p) {
   float* sig = tau_v + m;                                    // mp
   float* s_red = sig + mp;                                   // NW
   float* s_scale = s_red + NW;                               // KDA ? DK : m
-  int* sel = reinterpret_cast<int*>(s_scale + (KDA ? DK : m));  // R
+  int* sel = reinterpret_cast<int*>(s_scale + (KDA ? DK : ((m + 3) & ~3)));  // R
   __shared__ __align__(8) uint64_t bar;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -216,16 +165,17 @@ __global__ void __launch_bounds__(NT) compress_kernel(const CompressParams p) {
   // 1. panels -> shared memory (TMA bulk copies, no multicast)
   if (tid == 0) {
     mbar_init(&bar, 1);
-    mbar_expect_tx(&bar, (uint32_t)(m * (DK + DV) * sizeof(float)));
+    fence_mbar_init();
+    mbar_arrive_expect_tx(&bar, (uint32_t)(m * (DK + DV) * sizeof(float)));
     bulk_g2s(sU, p.U + unit * (long long)m * DK, (uint32_t)(m * DK * sizeof(float)), &bar);
     bulk_g2s(sV, p.V + unit * (long long)m * DV, (uint32_t)(m * DV * sizeof(float)), &bar);
   }
-  const int slen = KDA ? DK : m;
+  const int slen = p.slen;
   for (int i = tid; i < slen; i += NT) s_scale[i] = p.scale[unit * slen + i];
   __syncthreads();   // barrier initialised before anyone polls it
-  if (!mbar_wait_bounded(&bar, 0, kWaitLimit)) {
+  if (!mbar_wait_bounded(&bar, 0, kWaitLimitNs)) {
     if (tid == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
-    mbar_wait_bounded(&bar, 0, kWaitLimit);
+    mbar_wait_bounded(&bar, 0, kWaitLimitNs);
     return;
   }
   // fold the lazy decay into U
@@ -328,7 +278,7 @@ __global__ void __launch_bounds__(NT) compress_kernel(const CompressParams p) {
 static size_t compress_smem_bytes(int form, int dk, int dv, int R, int W, int nt) {
   const int m = R + W, mp = m + (m & 1);
   size_t f = (size_t)m * dk + (size_t)m * dv + (size_t)mp * (m + 1) + (size_t)mp * (mp + 1) +
-             2 * m + mp + nt / 32 + (form == SEED_KDA ? dk : m) + R;
+             2 * m + mp + nt / 32 + (form == SEED_KDA ? dk : ((m + 3) & ~3)) + R;
   return f * sizeof(float) + 16;
 }
 
@@ -360,7 +310,7 @@ static int launch_compress_t(const CompressParams& p, int blocks, cudaStream_t s
 int launch_compress(const seed_dims& d, const seed_state& s, int layer, float* sigma_out,
                     uint32_t* status, cudaStream_t st) {
   CompressParams p{s.U, s.V, s.scale, s.ncols, sigma_out, status,
-                   d.batch, d.layers, d.heads, layer, d.R, d.W};
+                   d.batch, d.layers, d.heads, layer, d.R, d.W, scale_len(d)};
   const int blocks = d.batch * d.heads * (layer < 0 ? d.layers : 1);
   switch (d.form) {
     case SEED_GDN: SEED_DISPATCH_DIMS(launch_compress_t, SEED_GDN, p, blocks, st);
@@ -381,7 +331,7 @@ struct InitParams {
   const float* vbar;
   float* sigma_out;
   uint32_t* status;
-  int B, L, H, layer, R, W, form;
+  int B, L, H, layer, R, W, form, slen;
 };
 
 template <int DK, int DV, int NT>
@@ -484,8 +434,7 @@ __global__ void __launch_bounds__(NT) init_kernel(const InitParams p) {
     bad |= !isfinite(s_a[i]);
     p.a[unit * DK + i] = s_a[i];
   }
-  const int slen = p.form == SEED_KDA ? DK : m;
-  for (int i = tid; i < slen; i += NT) p.scale[unit * slen + i] = 1.f;
+  for (int i = tid; i < p.slen; i += NT) p.scale[unit * p.slen + i] = 1.f;
   if (tid == 0) p.ncols[unit] = p.R;
   if (!conv && tid == 0) raise_flag(p.status, SEED_FLAG_NOCONVERGE);
   if (bad && conv) raise_flag(p.status, SEED_FLAG_NONFINITE);
@@ -507,7 +456,7 @@ static int launch_init_t(const InitParams& p, int blocks, cudaStream_t st) {
 int launch_init_from_dense(const seed_dims& d, const seed_state& s, int layer, const float* S,
                            float* sigma_out, uint32_t* status, cudaStream_t st) {
   InitParams p{S, s.a, s.U, s.V, s.scale, s.ncols, s.vbar, sigma_out, status,
-               d.batch, d.layers, d.heads, layer, d.R, d.W, d.form};
+               d.batch, d.layers, d.heads, layer, d.R, d.W, d.form, scale_len(d)};
   const int blocks = d.batch * d.heads * (layer < 0 ? d.layers : 1);
   SEED_DISPATCH_DIMS(launch_init_t, 0, p, blocks, st);
 }
@@ -523,7 +472,7 @@ struct ToDenseParams {
   const int32_t* units;
   float* S;
   uint32_t* status;
-  int B, L, H, layer, R, W, form;
+  int B, L, H, layer, R, W, form, slen;
 };
 
 template <int DK, int DV, int NT>
@@ -552,7 +501,7 @@ __global__ void __launch_bounds__(NT) to_dense_kernel(const ToDenseParams p) {
   }
   for (int idx = threadIdx.x; idx < c * DK; idx += NT) {
     const int j = idx / DK, i = idx - j * DK;
-    const float sc = kda ? p.scale[unit * DK + i] : p.scale[unit * m + j];
+    const float sc = kda ? p.scale[unit * DK + i] : p.scale[unit * p.slen + j];
     sU[idx] = sc * p.U[unit * (long long)m * DK + idx];
   }
   for (int idx = threadIdx.x; idx < c * DV; idx += NT) sV[idx] = p.V[unit * (long long)m * DV + idx];
@@ -583,7 +532,7 @@ static int launch_to_dense_t(const ToDenseParams& p, int blocks, cudaStream_t st
 int launch_to_dense(const seed_dims& d, const seed_state& s, int layer, const int32_t* units,
                     int n_units, float* S_out, uint32_t* status, cudaStream_t st) {
   ToDenseParams p{s.a, s.U, s.V, s.scale, s.ncols, s.vbar, units, S_out, status,
-                  d.batch, d.layers, d.heads, layer, d.R, d.W, d.form};
+                  d.batch, d.layers, d.heads, layer, d.R, d.W, d.form, scale_len(d)};
   SEED_DISPATCH_DIMS(launch_to_dense_t, 0, p, n_units, st);
 }
 

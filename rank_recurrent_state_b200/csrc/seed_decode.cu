@@ -2,10 +2,15 @@
 //
 // "Shallow Encoding Emits Deep Memories", SEED summary (picx.dev), "Exact Update
 // (Lemma 2)" with the sink recurrence of Lemma 1, and the read-out o = S+^T q.
-// One CTA per (request, head) unit of the layer.  The step is HBM-bound: the unit's
-// c stored columns of U and V are read once (coalesced float4, one warp-row per
-// column), and only the touched bytes are written: the sink a, one new column of
-// U and of V, the decay scales and the column count.
+//
+// The step is HBM-bound: each (request, head) unit reads its c stored columns of
+// U and V once and writes back only the touched bytes (the sink a, one new column
+// of U and of V, the decay scales, the column count).  The kernel is persistent
+// and warp-specialised: in each CTA one producer warp streams units through a
+// ring of shared-memory stages with TMA bulk copies (cp.async.bulk, completion on
+// an mbarrier, no multicast), and four consumer warps compute each unit from
+// shared memory and hand the stage back through a second mbarrier.  The producer
+// runs NS units ahead, so every SM keeps several units' panels in flight.
 //
 // Lazy decay.  Gated DeltaNet and Mamba-2 scale every old U column by the same
 // scalar per step; instead of rewriting U the kernel keeps per-column scales
@@ -15,6 +20,7 @@
 // true value is k.  Both are folded back into U by the compression.
 #include "seed_common.cuh"
 #include "seed_launch.h"
+#include "seed_tma.cuh"
 
 namespace seed {
 
@@ -32,17 +38,73 @@ struct DecodeParams {
   int32_t* ncols;
   const float* vbar;
   uint32_t* status;
-  int B, L, H, layer, R, W;
+  int B, L, H, layer, R, W, slen;
 };
 
-// FORM: seed_form; DK, DV: head dims; NW: warps per CTA; MAXC: bound on the
-// column count c a unit may hold before the step (c <= R + W - 1 <= MAXC).
-template <int FORM, int DK, int DV, int NW, int MAXC>
-__global__ void __launch_bounds__(NW * 32) decode_step_kernel(const DecodeParams p) {
+// One pipeline stage: everything a unit's step reads.
+template <int FORM, int DK, int DV, int MAXC>
+struct DecodeStage {
+  static constexpr bool KDA = FORM == SEED_KDA;
+  static constexpr int GPAD = (MAXC + 3) & ~3;
+  float U[MAXC * DK];
+  float V[MAXC * DV];
+  float a[DK];
+  float k[DK];
+  float q[DK];
+  float v[DV];
+  float vb[DV];
+  float al[KDA ? DK : 4];
+  float P[KDA ? DK : 4];
+  float gam[GPAD];
+  float g;
+  float beta;
+  int c;
+  int pad;
+};
+
+// Sum of NV per-lane values over the 32 lanes of a warp by recursive halving:
+// 2 NV - 2 shuffles for NV <= 32 instead of 5 NV.  Lane l ends up holding the
+// total of value (l >> (5 - log2 NV)) & (NV - 1).
+template <int NV>
+SEED_DEV float warp_xreduce(float (&v)[NV]) {
+  const int lane = threadIdx.x & 31;
+  int n = NV;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    if (n > 1) {
+      const bool hi = (lane & off) != 0;
+#pragma unroll
+      for (int i = 0; i < NV / 2; ++i) {
+        if (i < n / 2) {
+          const float send = hi ? v[i] : v[i + n / 2];
+          const float keep = hi ? v[i + n / 2] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+      }
+      n >>= 1;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
+    }
+  }
+  return v[0];
+}
+
+template <int NV>
+SEED_DEV constexpr int log2c() { return NV <= 1 ? 0 : 1 + log2c<NV / 2>(); }
+
+constexpr int kConsumerWarps = 4;
+constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
+
+SEED_DEV void consumer_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+template <int FORM, int DK, int DV, int MAXC, int NS>
+__global__ void __launch_bounds__(kDecodeThreads) decode_step_kernel(const DecodeParams p) {
+  using Stage = DecodeStage<FORM, DK, DV, MAXC>;
+  constexpr int NW = kConsumerWarps;
   constexpr int NT = NW * 32;
   constexpr int LK = DK / 4;            // lanes per U column (float4 each)
   constexpr int CPK = 32 / LK;          // U columns per warp pass
-  constexpr int GK = NW * CPK;          // U column groups in the CTA
+  constexpr int GK = NW * CPK;          // U column groups
   constexpr int CU = (MAXC + GK - 1) / GK;
   constexpr int LV = DV / 4;
   constexpr int CPV = 32 / LV;
@@ -50,237 +112,323 @@ __global__ void __launch_bounds__(NW * 32) decode_step_kernel(const DecodeParams
   constexpr int CV = (MAXC + GV - 1) / GV;
   constexpr bool KDA = FORM == SEED_KDA;
   constexpr bool M2 = FORM == SEED_MAMBA2;
+  constexpr int NDOT = M2 ? 1 : 2;      // dots per U column: with q, and with k for the erase
 
-  __shared__ __align__(16) float s_a[DK];
-  __shared__ __align__(16) float s_k[DK];
-  __shared__ __align__(16) float s_q[DK];
-  __shared__ __align__(16) float s_v[DV];
-  __shared__ __align__(16) float s_vb[DV];
-  __shared__ __align__(16) float s_al[KDA ? DK : 4];
-  __shared__ __align__(16) float s_P[KDA ? DK : 4];
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  Stage* stages = reinterpret_cast<Stage*>(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + NS * sizeof(Stage));
+  uint64_t* empty = full + NS;
   __shared__ float s_dk[MAXC];
   __shared__ float s_dq[MAXC];
-  __shared__ float s_gam[MAXC + 1];
   __shared__ __align__(16) float s_yk[NW][DV];
   __shared__ __align__(16) float s_yq[NW][DV];
-  __shared__ float s_red[NW][5];
+  __shared__ float s_red[NW][8];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int bh = blockIdx.x;
-  const int b = bh / p.H, h = bh - b * p.H;
-  const long long unit = ((long long)b * p.L + p.layer) * p.H + h;
+  const int n_units = p.B * p.H;
   const int m = p.R + p.W;
-  const int c = p.ncols[unit];
-  if (c < 0 || c >= m) {
-    if (tid == 0) raise_flag(p.status, c == m ? SEED_FLAG_FULL : SEED_FLAG_BADCOLS);
-    return;
-  }
-
-  // 1. issue the factor loads first: they are the bytes that bound the step
-  const float* Uu = p.U + unit * (long long)m * DK;
-  const float* Vu = p.V + unit * (long long)m * DV;
-  const int gk = warp * CPK + lane / LK, lk = lane % LK;
-  const int gv = warp * CPV + lane / LV, lv = lane % LV;
-  float4 ur[CU], vr[CV];
-#pragma unroll
-  for (int i = 0; i < CU; ++i) {
-    const int j = gk + GK * i;
-    ur[i] = j < c ? ld_stream4(Uu + (long long)j * DK + 4 * lk) : zero4();
-  }
-#pragma unroll
-  for (int i = 0; i < CV; ++i) {
-    const int j = gv + GV * i;
-    vr[i] = j < c ? ld_stream4(Vu + (long long)j * DV + 4 * lv) : zero4();
-  }
-
-  // 2. the unit's vectors and scalars
-  for (int i = tid; i < DK / 4; i += NT) {
-    st4(s_a + 4 * i, ld4(p.a + unit * DK + 4 * i));
-    st4(s_k + 4 * i, ld4(p.k + (long long)bh * DK + 4 * i));
-    st4(s_q + 4 * i, ld4(p.q + (long long)bh * DK + 4 * i));
-    if constexpr (KDA) {
-      st4(s_al + 4 * i, ld4(p.alpha + (long long)bh * DK + 4 * i));
-      st4(s_P + 4 * i, ld4(p.scale + unit * DK + 4 * i));
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], NW);
     }
+    fence_mbar_init();
   }
-  for (int i = tid; i < DV / 4; i += NT) {
-    st4(s_v + 4 * i, ld4(p.v + (long long)bh * DV + 4 * i));
-    st4(s_vb + 4 * i, ld4(p.vbar + ((long long)p.layer * p.H + h) * DV + 4 * i));
-  }
-  if constexpr (!KDA) {
-    for (int j = tid; j < c; j += NT) s_gam[j] = p.scale[unit * m + j];
-  }
-  const float g = KDA ? 1.f : p.alpha[bh];   // GDN decay g / Mamba-2 alpha
-  const float be = p.beta[bh];               // GDN/KDA beta / Mamba-2 Delta
   __syncthreads();
 
-  // 3. dots of the stored U columns with k and q (KDA: with P+ (.) k, P+ (.) q,
-  //    P+ = P (.) alpha, so that they are the dots of the decayed true columns)
-  float4 kk = ld4(s_k + 4 * lk), qq = ld4(s_q + 4 * lk);
-  if constexpr (KDA) {
-    const float4 pp = mul4(ld4(s_P + 4 * lk), ld4(s_al + 4 * lk));
-    kk = mul4(kk, pp);
-    qq = mul4(qq, pp);
-  }
-  float dk[CU], dq[CU];
-#pragma unroll
-  for (int i = 0; i < CU; ++i) {
-    dk[i] = dot4(ur[i], kk);
-    dq[i] = dot4(ur[i], qq);
-  }
-#pragma unroll
-  for (int i = 0; i < CU; ++i) {
-    if constexpr (!M2) dk[i] = group_sum<LK>(dk[i]);
-    dq[i] = group_sum<LK>(dq[i]);
-  }
-  if (lk == 0) {
-#pragma unroll
-    for (int i = 0; i < CU; ++i) {
-      const int j = gk + GK * i;
-      if (j < c) {
-        s_dk[j] = dk[i];
-        s_dq[j] = dq[i];
+  // ------------------------------------------------------------------ producer warp
+  if (warp == NW) {
+    if (lane != 0) return;
+    int u = blockIdx.x;
+    int c_next = 0;
+    float g_next = 0.f, b_next = 0.f;
+    if (u < n_units) {
+      const long long un = ((long long)(u / p.H) * p.L + p.layer) * p.H + (u % p.H);
+      c_next = p.ncols[un];
+      g_next = KDA ? 1.f : p.alpha[u];
+      b_next = p.beta[u];
+    }
+    for (int i = 0; u < n_units; u += gridDim.x, ++i) {
+      const int s = i % NS;
+      const uint32_t ph = (uint32_t)(i / NS) & 1u;
+      const int b = u / p.H, h = u - (u / p.H) * p.H;
+      const long long unit = ((long long)b * p.L + p.layer) * p.H + h;
+      const int c = c_next;
+      const float g = g_next, be = b_next;
+      const int u2 = u + gridDim.x;
+      if (u2 < n_units) {   // prefetch the next unit's scalars while this one is issued
+        const long long un = ((long long)(u2 / p.H) * p.L + p.layer) * p.H + (u2 % p.H);
+        c_next = p.ncols[un];
+        g_next = KDA ? 1.f : p.alpha[u2];
+        b_next = p.beta[u2];
+      }
+      if (i >= NS && !mbar_wait_bounded(&empty[s], ph ^ 1u, kWaitLimitNs)) {
+        raise_flag(p.status, SEED_FLAG_TIMEOUT);
+        return;
+      }
+      Stage& S = stages[s];
+      S.c = c;
+      S.g = g;
+      S.beta = be;
+      const bool valid = c >= 0 && c < m;
+      uint32_t bytes = 0;
+      if (valid) {
+        bytes = (uint32_t)(c * (DK + DV) + 3 * DK + 2 * DV) * 4u;
+        bytes += KDA ? 2u * DK * 4u : (uint32_t)((c + 3) & ~3) * 4u;
+      }
+      mbar_arrive_expect_tx(&full[s], bytes);
+      if (valid) {
+        if (c > 0) {
+          bulk_g2s(S.U, p.U + unit * (long long)m * DK, (uint32_t)(c * DK * 4), &full[s]);
+          bulk_g2s(S.V, p.V + unit * (long long)m * DV, (uint32_t)(c * DV * 4), &full[s]);
+        }
+        bulk_g2s(S.a, p.a + unit * DK, DK * 4, &full[s]);
+        bulk_g2s(S.k, p.k + (long long)u * DK, DK * 4, &full[s]);
+        bulk_g2s(S.q, p.q + (long long)u * DK, DK * 4, &full[s]);
+        bulk_g2s(S.v, p.v + (long long)u * DV, DV * 4, &full[s]);
+        bulk_g2s(S.vb, p.vbar + ((long long)p.layer * p.H + h) * DV, DV * 4, &full[s]);
+        if constexpr (KDA) {
+          bulk_g2s(S.al, p.alpha + (long long)u * DK, DK * 4, &full[s]);
+          bulk_g2s(S.P, p.scale + unit * DK, DK * 4, &full[s]);
+        } else if (c > 0) {
+          bulk_g2s(S.gam, p.scale + unit * p.slen, (uint32_t)((c + 3) & ~3) * 4u, &full[s]);
+        }
       }
     }
-  }
-
-  // scalars: k^T a', a'^T q, k^T q (a' = alpha (.) a for KDA), v^T vbar, vbar^T vbar
-  float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f, r4 = 0.f;
-  for (int i = tid; i < DK; i += NT) {
-    const float ai = KDA ? s_al[i] * s_a[i] : s_a[i];
-    r0 = fmaf(s_k[i], ai, r0);
-    r1 = fmaf(ai, s_q[i], r1);
-    r2 = fmaf(s_k[i], s_q[i], r2);
-  }
-  for (int i = tid; i < DV; i += NT) {
-    r3 = fmaf(s_v[i], s_vb[i], r3);
-    r4 = fmaf(s_vb[i], s_vb[i], r4);
-  }
-  r0 = group_sum<32>(r0);
-  r1 = group_sum<32>(r1);
-  r2 = group_sum<32>(r2);
-  r3 = group_sum<32>(r3);
-  r4 = group_sum<32>(r4);
-  if (lane == 0) {
-    s_red[warp][0] = r0;
-    s_red[warp][1] = r1;
-    s_red[warp][2] = r2;
-    s_red[warp][3] = r3;
-    s_red[warp][4] = r4;
-  }
-  __syncthreads();
-  float ka = 0.f, aq = 0.f, kq = 0.f, vvb = 0.f, vbvb = 0.f;
-#pragma unroll
-  for (int w = 0; w < NW; ++w) {
-    ka += s_red[w][0];
-    aq += s_red[w][1];
-    kq += s_red[w][2];
-    vvb += s_red[w][3];
-    vbvb += s_red[w][4];
-  }
-  if (!(vbvb > 0.f)) {
-    if (tid == 0) raise_flag(p.status, SEED_FLAG_ZERO_VBAR);
     return;
   }
-  const float omega = vvb / vbvb;
 
-  // 4. V times the column coefficients: y_k = V (g gamma (.) U^T k) for the erase
-  //    term, y_q = V (g gamma (.) U^T q) for the read-out (decayed true columns)
-  float4 yk = zero4(), yq = zero4();
-#pragma unroll
-  for (int i = 0; i < CV; ++i) {
-    const int j = gv + GV * i;
-    if (j < c) {
-      const float sc = KDA ? 1.f : g * s_gam[j];
-      if constexpr (!M2) yk = fma4(sc * s_dk[j], vr[i], yk);
-      yq = fma4(sc * s_dq[j], vr[i], yq);
+  // ------------------------------------------------------------------ consumer warps
+  const int gk = warp * CPK + lane / LK, lk = lane % LK;
+  const int gv = warp * CPV + lane / LV, lv = lane % LV;
+  for (int i = 0, u = blockIdx.x; u < n_units; u += gridDim.x, ++i) {
+    const int s = i % NS;
+    const uint32_t ph = (uint32_t)(i / NS) & 1u;
+    if (!mbar_wait_bounded(&full[s], ph, kWaitLimitNs)) {
+      if (tid == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
+      mbar_wait_bounded(&full[s], ph, kWaitLimitNs);   // let copies in flight land
+      return;
     }
-  }
+    const Stage& S = stages[s];
+    const int b = u / p.H, h = u - (u / p.H) * p.H;
+    const long long unit = ((long long)b * p.L + p.layer) * p.H + h;
+    const int c = S.c;
+    const float g = S.g, be = S.beta;
+    bool skip = false;
+    if (c < 0 || c >= m) {
+      if (tid == 0) raise_flag(p.status, c == m ? SEED_FLAG_FULL : SEED_FLAG_BADCOLS);
+      skip = true;
+    }
+    if (!skip) {
+      // 1. dots of the stored U columns with k and q (KDA: with P+ (.) k, P+ (.) q,
+      //    P+ = P (.) alpha, the dots of the decayed true columns)
+      float4 kk = ld4(S.k + 4 * lk), qq = ld4(S.q + 4 * lk);
+      if constexpr (KDA) {
+        const float4 pp = mul4(ld4(S.P + 4 * lk), ld4(S.al + 4 * lk));
+        kk = mul4(kk, pp);
+        qq = mul4(qq, pp);
+      }
+      float dv[NDOT * CU];
 #pragma unroll
-  for (int off = LV; off < 32; off <<= 1) {
-    yk.x += __shfl_xor_sync(0xffffffffu, yk.x, off);
-    yk.y += __shfl_xor_sync(0xffffffffu, yk.y, off);
-    yk.z += __shfl_xor_sync(0xffffffffu, yk.z, off);
-    yk.w += __shfl_xor_sync(0xffffffffu, yk.w, off);
-    yq.x += __shfl_xor_sync(0xffffffffu, yq.x, off);
-    yq.y += __shfl_xor_sync(0xffffffffu, yq.y, off);
-    yq.z += __shfl_xor_sync(0xffffffffu, yq.z, off);
-    yq.w += __shfl_xor_sync(0xffffffffu, yq.w, off);
-  }
-  if (lane < LV) {
-    st4(&s_yk[warp][4 * lane], yk);
-    st4(&s_yq[warp][4 * lane], yq);
-  }
-  __syncthreads();
+      for (int r = 0; r < CU; ++r) {
+        const int j = gk + GK * r;
+        const float4 uc = j < c ? ld4(S.U + j * DK + 4 * lk) : zero4();
+        dv[r] = dot4(uc, qq);
+        if constexpr (!M2) dv[CU + r] = dot4(uc, kk);
+      }
+      if constexpr (LK == 32 && ((NDOT * CU) & (NDOT * CU - 1)) == 0) {
+        constexpr int NV = NDOT * CU;
+        const float tot = warp_xreduce<NV>(dv);
+        constexpr int SH = 5 - log2c<NV>();
+        if ((lane & ((1 << SH) - 1)) == 0) {
+          const int idx = (lane >> SH) & (NV - 1);
+          const int r = idx % CU;
+          const int j = gk + GK * r;
+          if (j < c) {
+            if (idx < CU) s_dq[j] = tot;
+            else s_dk[j] = tot;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int r = 0; r < NDOT * CU; ++r) dv[r] = group_sum<LK>(dv[r]);
+        if (lk == 0) {
+#pragma unroll
+          for (int r = 0; r < CU; ++r) {
+            const int j = gk + GK * r;
+            if (j < c) {
+              s_dq[j] = dv[r];
+              if constexpr (!M2) s_dk[j] = dv[CU + r];
+            }
+          }
+        }
+      }
+      // scalars: k^T a', a'^T q, k^T q (a' = alpha (.) a for KDA), v^T vbar, vbar^T vbar
+      float sc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int e = tid; e < DK; e += NT) {
+        const float ae = KDA ? S.al[e] * S.a[e] : S.a[e];
+        sc[0] = fmaf(S.k[e], ae, sc[0]);
+        sc[1] = fmaf(ae, S.q[e], sc[1]);
+        sc[2] = fmaf(S.k[e], S.q[e], sc[2]);
+      }
+      for (int e = tid; e < DV; e += NT) {
+        sc[3] = fmaf(S.v[e], S.vb[e], sc[3]);
+        sc[4] = fmaf(S.vb[e], S.vb[e], sc[4]);
+      }
+      {
+        const float tot = warp_xreduce<8>(sc);
+        if ((lane & 3) == 0) s_red[warp][(lane >> 2) & 7] = tot;
+      }
+      consumer_sync();
+      float ka = 0.f, aq = 0.f, kq = 0.f, vvb = 0.f, vbvb = 0.f;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        ka += s_red[w][0];
+        aq += s_red[w][1];
+        kq += s_red[w][2];
+        vvb += s_red[w][3];
+        vbvb += s_red[w][4];
+      }
+      if (!(vbvb > 0.f)) {
+        if (tid == 0) raise_flag(p.status, SEED_FLAG_ZERO_VBAR);
+        skip = true;
+      }
+      if (!skip) {
+        const float omega = vvb / vbvb;
+        // 2. V times the column coefficients: y_k = V (g gamma (.) U^T k) for the
+        //    erase, y_q = V (g gamma (.) U^T q) for the read-out (decayed true columns)
+        float4 yk = zero4(), yq = zero4();
+#pragma unroll
+        for (int r = 0; r < CV; ++r) {
+          const int j = gv + GV * r;
+          if (j < c) {
+            const float4 vc = ld4(S.V + j * DV + 4 * lv);
+            const float f = KDA ? 1.f : g * S.gam[j];
+            if constexpr (!M2) yk = fma4(f * s_dk[j], vc, yk);
+            yq = fma4(f * s_dq[j], vc, yq);
+          }
+        }
+#pragma unroll
+        for (int off = LV; off < 32; off <<= 1) {
+          if constexpr (!M2) {
+            yk.x += __shfl_xor_sync(0xffffffffu, yk.x, off);
+            yk.y += __shfl_xor_sync(0xffffffffu, yk.y, off);
+            yk.z += __shfl_xor_sync(0xffffffffu, yk.z, off);
+            yk.w += __shfl_xor_sync(0xffffffffu, yk.w, off);
+          }
+          yq.x += __shfl_xor_sync(0xffffffffu, yq.x, off);
+          yq.y += __shfl_xor_sync(0xffffffffu, yq.y, off);
+          yq.z += __shfl_xor_sync(0xffffffffu, yq.z, off);
+          yq.w += __shfl_xor_sync(0xffffffffu, yq.w, off);
+        }
+        if (lane < LV) {
+          if constexpr (!M2) st4(&s_yk[warp][4 * lane], yk);
+          st4(&s_yq[warp][4 * lane], yq);
+        }
+        consumer_sync();
 
-  // 5. sink update, new column pair, read-out
-  float coef;   // a+ = a' + coef * k   (a' = g a, alpha (.) a, alpha a)
-  if constexpr (FORM == SEED_GDN) coef = be * (omega - g * ka);
-  else if constexpr (KDA) coef = be * (omega - ka);
-  else coef = be * omega;
-  const float apq = (KDA ? aq : g * aq) + coef * kq;   // a+^T q
-  bool bad = false;
-  float* Vnew = p.V + unit * (long long)m * DV + (long long)c * DV;
-  float* Unew = p.U + unit * (long long)m * DK + (long long)c * DK;
-  for (int i = tid; i < DV; i += NT) {
-    float yki = 0.f, yqi = 0.f;
+        // 3. sink update, new column pair, read-out
+        float coef;   // a+ = a' + coef * k   (a' = g a, alpha (.) a, alpha a)
+        if constexpr (FORM == SEED_GDN) coef = be * (omega - g * ka);
+        else if constexpr (KDA) coef = be * (omega - ka);
+        else coef = be * omega;
+        const float apq = (KDA ? aq : g * aq) + coef * kq;   // a+^T q
+        bool bad = false;
+        float* Vnew = p.V + unit * (long long)m * DV + (long long)c * DV;
+        float* Unew = p.U + unit * (long long)m * DK + (long long)c * DK;
+        for (int e = tid; e < DV; e += NT) {
+          float yke = 0.f, yqe = 0.f;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      yki += s_yk[w][i];
-      yqi += s_yq[w][i];
+          for (int w = 0; w < NW; ++w) {
+            if constexpr (!M2) yke += s_yk[w][e];
+            yqe += s_yq[w][e];
+          }
+          const float eps = S.v[e] - omega * S.vb[e];
+          const float ncol = M2 ? be * eps : be * (eps - yke);
+          const float oe = fmaf(S.vb[e], apq, yqe) + ncol * kq;
+          bad |= !(isfinite(ncol) && isfinite(oe));
+          Vnew[e] = ncol;
+          p.o[(long long)u * DV + e] = oe;
+        }
+        for (int e = tid; e < DK; e += NT) {
+          const float ae = S.a[e];
+          const float ke = S.k[e];
+          float anew;
+          if constexpr (KDA) {
+            const float pn = S.P[e] * S.al[e];
+            anew = fmaf(S.al[e], ae, coef * ke);
+            const float us = ke / pn;
+            bad |= !isfinite(us);
+            Unew[e] = us;
+            p.scale[unit * DK + e] = pn;
+          } else {
+            anew = fmaf(g, ae, coef * ke);
+            Unew[e] = ke;
+          }
+          bad |= !isfinite(anew);
+          p.a[unit * DK + e] = anew;
+        }
+        if constexpr (!KDA) {
+          for (int j = tid; j <= c; j += NT) p.scale[unit * p.slen + j] = j < c ? g * S.gam[j] : 1.f;
+        }
+        if (tid == 0) p.ncols[unit] = c + 1;
+        if (bad) raise_flag(p.status, SEED_FLAG_NONFINITE);
+      }
     }
-    const float eps = s_v[i] - omega * s_vb[i];
-    const float ncol = M2 ? be * eps : be * (eps - yki);
-    const float oi = fmaf(s_vb[i], apq, yqi) + ncol * kq;
-    bad |= !(isfinite(ncol) && isfinite(oi));
-    Vnew[i] = ncol;
-    p.o[(long long)bh * DV + i] = oi;
+    // hand the stage back to the producer (every consumer read of S is above)
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
   }
-  for (int i = tid; i < DK; i += NT) {
-    const float ai = s_a[i];
-    const float ki = s_k[i];
-    float anew;
-    if constexpr (KDA) {
-      const float pn = s_P[i] * s_al[i];
-      anew = fmaf(s_al[i], ai, coef * ki);
-      const float us = ki / pn;
-      bad |= !isfinite(us);
-      Unew[i] = us;
-      p.scale[unit * DK + i] = pn;
-    } else {
-      anew = fmaf(g, ai, coef * ki);
-      Unew[i] = ki;
-    }
-    bad |= !isfinite(anew);
-    p.a[unit * DK + i] = anew;
-  }
-  if constexpr (!KDA) {
-    for (int j = tid; j <= c; j += NT) p.scale[unit * m + j] = j < c ? g * s_gam[j] : 1.f;
-  }
-  if (tid == 0) p.ncols[unit] = c + 1;
-  if (bad) raise_flag(p.status, SEED_FLAG_NONFINITE);
 }
 
-template <int FORM, int DK, int DV, int NW, int MAXC>
-static int launch_one(const DecodeParams& p, int blocks, cudaStream_t st) {
-  decode_step_kernel<FORM, DK, DV, NW, MAXC><<<blocks, NW * 32, 0, st>>>(p);
+template <int FORM, int DK, int DV, int MAXC>
+static int launch_one(const DecodeParams& p, cudaStream_t st) {
+  using Stage = DecodeStage<FORM, DK, DV, MAXC>;
+  // stages: as many as fit in ~108 KB so that two CTAs share an SM, at least two
+  constexpr int NS0 = (int)((108 * 1024) / sizeof(Stage));
+  constexpr int NS = NS0 < 2 ? 2 : (NS0 > 6 ? 6 : NS0);
+  const size_t smem = NS * sizeof(Stage) + 2 * NS * sizeof(uint64_t);
+  auto kern = decode_step_kernel<FORM, DK, DV, MAXC, NS>;
+  // per device: the shared-memory opt-in and the resident CTAs per SM
+  constexpr int kMaxDev = 64;
+  static int grid_per_sm[kMaxDev] = {0};
+  static int sm_count[kMaxDev] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return SEED_ERR_CUDA;
+  if (grid_per_sm[dev] == 0) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return SEED_ERR_CUDA;
+    int n = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return SEED_ERR_CUDA;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kDecodeThreads, smem) !=
+        cudaSuccess)
+      return SEED_ERR_CUDA;
+    sm_count[dev] = sms;
+    grid_per_sm[dev] = n > 0 ? n : 1;
+  }
+  const int units = p.B * p.H;
+  int grid = grid_per_sm[dev] * sm_count[dev];
+  if (grid > units) grid = units;
+  kern<<<grid, kDecodeThreads, smem, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? SEED_OK : SEED_ERR_CUDA;
 }
 
 template <int FORM, int DK, int DV>
-static int launch_cols(const DecodeParams& p, int blocks, cudaStream_t st) {
+static int launch_cols(const DecodeParams& p, cudaStream_t st) {
   const int maxc = p.R + p.W - 1;
-  if (maxc <= 8) return launch_one<FORM, DK, DV, 4, 8>(p, blocks, st);
-  if (maxc <= 16) return launch_one<FORM, DK, DV, 4, 16>(p, blocks, st);
-  if (maxc <= 32) return launch_one<FORM, DK, DV, 4, 32>(p, blocks, st);
-  if (maxc <= 64) return launch_one<FORM, DK, DV, 8, 64>(p, blocks, st);
-  return launch_one<FORM, DK, DV, 12, 96>(p, blocks, st);
+  if (maxc <= 8) return launch_one<FORM, DK, DV, 8>(p, st);
+  if (maxc <= 16) return launch_one<FORM, DK, DV, 16>(p, st);
+  if (maxc <= 32) return launch_one<FORM, DK, DV, 32>(p, st);
+  if (maxc <= 64) return launch_one<FORM, DK, DV, 64>(p, st);
+  return launch_one<FORM, DK, DV, 96>(p, st);
 }
 
 template <int FORM>
-static int launch_dims(const DecodeParams& p, int dk, int dv, int blocks, cudaStream_t st) {
+static int launch_dims(const DecodeParams& p, int dk, int dv, cudaStream_t st) {
 #define SEED_DIMS_CASE(K, V) \
-  if (dk == K && dv == V) return launch_cols<FORM, K, V>(p, blocks, st);
+  if (dk == K && dv == V) return launch_cols<FORM, K, V>(p, st);
   SEED_DIMS_CASE(16, 16)
   SEED_DIMS_CASE(32, 32)
   SEED_DIMS_CASE(64, 64)
@@ -295,12 +443,11 @@ int launch_decode_step(const seed_dims& d, const seed_state& s, int layer, const
                        const float* k, const float* v, const float* alpha, const float* beta,
                        float* o, uint32_t* status, cudaStream_t st) {
   DecodeParams p{q, k, v, alpha, beta, o, s.a, s.U, s.V, s.scale, s.ncols, s.vbar, status,
-                 d.batch, d.layers, d.heads, layer, d.R, d.W};
-  const int blocks = d.batch * d.heads;
+                 d.batch, d.layers, d.heads, layer, d.R, d.W, scale_len(d)};
   switch (d.form) {
-    case SEED_GDN: return launch_dims<SEED_GDN>(p, d.d_k, d.d_v, blocks, st);
-    case SEED_KDA: return launch_dims<SEED_KDA>(p, d.d_k, d.d_v, blocks, st);
-    case SEED_MAMBA2: return launch_dims<SEED_MAMBA2>(p, d.d_k, d.d_v, blocks, st);
+    case SEED_GDN: return launch_dims<SEED_GDN>(p, d.d_k, d.d_v, st);
+    case SEED_KDA: return launch_dims<SEED_KDA>(p, d.d_k, d.d_v, st);
+    case SEED_MAMBA2: return launch_dims<SEED_MAMBA2>(p, d.d_k, d.d_v, st);
   }
   return SEED_ERR_INVALID_ARG;
 }

@@ -10,6 +10,12 @@
 
 namespace seed {
 
+// Per-unit length of seed_state.scale: d_k for KDA (the decay product P), else
+// R + W rounded up to a multiple of 4 (column scales, 16-byte aligned per unit).
+inline int scale_len(const seed_dims& d) {
+  return d.form == SEED_KDA ? d.d_k : ((d.R + d.W + 3) & ~3);
+}
+
 bool decode_dims_supported(int dk, int dv);
 
 int launch_decode_step(const seed_dims& d, const seed_state& s, int layer, const float* q,

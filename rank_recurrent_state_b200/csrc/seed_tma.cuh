@@ -1,0 +1,70 @@
+// seed_tma.cuh -- TMA bulk copies and mbarriers (inline PTX, sm_90+ / sm_100a).
+// Only non-multicast global -> shared bulk copies are used.
+#pragma once
+
+#include <stdint.h>
+
+#include "seed_common.cuh"
+
+namespace seed {
+
+SEED_DEV uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+SEED_DEV void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count));
+}
+
+// Make barrier initialisation visible to the async proxy before any bulk copy uses it.
+SEED_DEV void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+
+SEED_DEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+SEED_DEV void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+// global -> shared bulk copy completing on `bar` (no multicast); both addresses
+// 16-byte aligned, bytes a multiple of 16.
+SEED_DEV void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+SEED_DEV bool mbar_test_wait(uint64_t* bar, uint32_t phase) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(phase)
+      : "memory");
+  return ok != 0;
+}
+
+SEED_DEV uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s
+
+// Bounded wait for the phase with the given parity: polls without blocking, with
+// a short sleep between polls, and gives up after `limit_ns` of wall time.
+SEED_DEV bool mbar_wait_bounded(uint64_t* bar, uint32_t phase, uint64_t limit_ns) {
+  if (mbar_test_wait(bar, phase)) return true;
+  const uint64_t t0 = global_ns();
+  while (!mbar_test_wait(bar, phase)) {
+    if (global_ns() - t0 > limit_ns) return false;
+    __nanosleep(32);
+  }
+  return true;
+}
+
+}  // namespace seed

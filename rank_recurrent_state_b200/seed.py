@@ -96,7 +96,7 @@ class State:
     a: torch.Tensor          # [B][L][H][d_k]
     U: torch.Tensor          # [B][L][H][R+W][d_k]
     V: torch.Tensor          # [B][L][H][R+W][d_v]
-    scale: torch.Tensor      # [B][L][H][R+W] (GDN, Mamba-2) or [B][L][H][d_k] (KDA)
+    scale: torch.Tensor      # [B][L][H][ceil4(R+W)] (GDN, Mamba-2) or [B][L][H][d_k] (KDA)
     ncols: torch.Tensor      # [B][L][H] int32
     vbar: torch.Tensor       # [L][H][d_v]
 
@@ -108,7 +108,7 @@ class State:
     def allocate(dims: Dims, vbar: torch.Tensor, device=None) -> "State":
         dev = vbar.device if device is None else device
         B, L, H = dims.batch, dims.layers, dims.heads
-        slen = dims.d_k if dims.form == SEED_KDA else dims.m
+        slen = dims.d_k if dims.form == SEED_KDA else (dims.m + 3) // 4 * 4
         f32 = dict(dtype=torch.float32, device=dev)
         return State(a=torch.zeros(B, L, H, dims.d_k, **f32),
                      U=torch.zeros(B, L, H, dims.m, dims.d_k, **f32),

@@ -68,16 +68,35 @@ def run_device(cfg, sample_units, n_prefill, n_decode, batch=None):
 def run_oracle(cfg, dev, n_prefill, n_decode):
     from oracle import run as orun
     return orun.run_units(cfg, dev["b"], dev["l"], dev["h"], n_prefill=n_prefill, n_decode=n_decode,
-                          keep_shadow=False)
+                          keep_shadow=True)
 
 
-def compare(cfg, dev, ref, tol=TOL):
-    """Per-unit and pooled relative Frobenius errors; near-tie units are reported and
-    excluded from the per-unit check only.  Returns a dict of the measured errors."""
+def max_decay(cfg, dev, n_decode) -> np.ndarray:
+    """Largest per-step contraction factor over the decode run, per sampled unit
+    (g for GDN, alpha for Mamba-2, max_i alpha_i for KDA), from the host generator."""
+    from workloads import philox
+    inp = philox.token_inputs(cfg, dev["b"][:, None], dev["l"][:, None], dev["h"][:, None],
+                              np.arange(n_decode)[None, :], philox.PHASE_DECODE, need_q=False)
+    al = np.asarray(inp["alpha"], dtype=np.float64)
+    return al.max(axis=(1, 2)) if al.ndim == 3 else al.max(axis=1)
+
+
+def compare(cfg, dev, ref, tol=TOL, max_tie_frac=0.25):
+    """Device against oracle.
+
+    Units whose smallest relative singular gap at R (conversion and every
+    compression) is below GAP_TOL are near-ties: several truncations are correct
+    there, so for them only what is unique is compared (the kept singular values
+    and the sink coefficient a, which no truncation touches) and the state is
+    checked for validity against the open-loop bound of Corollary 4 (distance to
+    the never-compressed dense state at most eps_bar / (1 - g_bar^W)).  Every
+    other unit is compared in full, per unit and pooled.  Bookkeeping is bit-exact.
+    """
     n = dev["o"].shape[1]
     gaps = [ref["conv_gap"]] + ([ref["gap"][i] for i in range(ref["gap"].shape[0])])
     min_gap = np.min(np.stack(gaps), axis=0)
     ties = min_gap < GAP_TOL
+    ok = ~ties
     errs = {"o": [], "S": [], "sigma": [], "a": []}
     for u in range(n):
         errs["o"].append(rel_fro(dev["o"][:, u], ref["o"][:, u]))
@@ -87,18 +106,31 @@ def compare(cfg, dev, ref, tol=TOL):
             errs["sigma"].append(rel_fro(dev["sigma"][:, u], ref["sigma"][:, u]))
     out = {k: np.array(v) for k, v in errs.items()}
     out["ties"] = int(ties.sum())
-    out["pooled_o"] = rel_fro(dev["o"], ref["o"])
-    out["pooled_S"] = rel_fro(dev["S"], ref["S"])
-    out["pooled_sigma"] = rel_fro(dev["sigma"], ref["sigma"]) if dev["sigma"].size else 0.0
     out["conv_S"] = np.array([rel_fro(dev["S_conv"][u], ref["S_conv"][u]) for u in range(n)])
     out["conv_sigma"] = np.array([rel_fro(dev["conv_sigma"][u], ref["conv_sigma"][u]) for u in range(n)])
     # bookkeeping must be bit-exact
     assert dev["comp_steps"] == ref["comp_steps"], (dev["comp_steps"], ref["comp_steps"])
     np.testing.assert_array_equal(dev["ncols"], np.repeat(ref["ncols"][:, None], n, axis=1))
+    assert out["ties"] <= max_tie_frac * n, ("too many near-ties", out["ties"], n)
+    # full comparison on units with a unique truncation
     for key in ("o", "S", "a", "sigma", "conv_S", "conv_sigma"):
         if out[key].size:
-            assert np.all(out[key][~ties] <= tol), (key, out[key])
-    for key in ("pooled_o", "pooled_S", "pooled_sigma"):
-        assert out[key] <= tol, (key, out[key])
+            assert np.all(out[key][ok] <= tol), (key, out[key])
+    if ok.any():
+        out["pooled_o"] = rel_fro(dev["o"][:, ok], ref["o"][:, ok])
+        out["pooled_S"] = rel_fro(dev["S"][ok], ref["S"][ok])
+        out["pooled_sigma"] = rel_fro(dev["sigma"][:, ok], ref["sigma"][:, ok]) if dev["sigma"].size else 0.0
+        for key in ("pooled_o", "pooled_S", "pooled_sigma"):
+            assert out[key] <= tol, (key, out[key])
+    # near-ties: unique quantities, and validity of the state
+    if ties.any():
+        for key in ("a", "sigma", "conv_sigma"):
+            if out[key].size:
+                assert np.all(out[key][ties] <= tol), (key + " (near-tie units)", out[key][ties])
+        g_bar = max_decay(cfg, dev, dev["o"].shape[0])
+        eps_bar = np.max(ref["tail"], axis=0)
+        bound = eps_bar / (1.0 - g_bar ** cfg.W)
+        dist = np.array([np.linalg.norm(dev["S"][u] - ref["S_exact"][u]) for u in range(n)])
+        assert np.all(dist[ties] <= bound[ties] * (1 + 1e-3) + 1e-4 * np.linalg.norm(ref["S_exact"][ties])), \
+            ("near-tie state outside the Corollary 4 bound", dist[ties], bound[ties])
     return out
-
