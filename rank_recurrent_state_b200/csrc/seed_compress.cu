@@ -129,11 +129,13 @@ SEED_DEV int select_top(const float* sig, int n, int R, int* sel) {
   return 0;
 }
 
+// One unit whose column count is R + W (checked by the caller), whole CTA.
+// `phase` is the parity of this unit's use of the CTA's mbarrier.
 template <int FORM, int DK, int DV, int NT>
-__global__ void __launch_bounds__(NT) compress_kernel(const CompressParams p) {
+__device__ void compress_unit(const CompressParams& p, long long unit, long long srow,
+                              unsigned char* smem_raw, uint64_t& bar, uint32_t phase) {
   constexpr int NW = NT / 32;
   constexpr bool KDA = FORM == SEED_KDA;
-  extern __shared__ __align__(128) unsigned char smem_raw[];
   const int m = p.R + p.W;
   const int mp = m + (m & 1);          // Jacobi needs an even column count
   const int ldm = m + 1;
@@ -148,34 +150,22 @@ __global__ void __launch_bounds__(NT) compress_kernel(const CompressParams p) {
   float* s_red = sig + mp;                                   // NW
   float* s_scale = s_red + NW;                               // KDA ? DK : m
   int* sel = reinterpret_cast<int*>(s_scale + (KDA ? DK : ((m + 3) & ~3)));  // R
-  __shared__ __align__(8) uint64_t bar;
-
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int units_in_scope = p.layer < 0 ? p.L * p.H : p.H;
-  const int b = blockIdx.x / units_in_scope;
-  const int rest = blockIdx.x - b * units_in_scope;
-  const long long unit = p.layer < 0 ? (long long)blockIdx.x
-                                     : ((long long)b * p.L + p.layer) * p.H + rest;
-  const int c = p.ncols[unit];
-  if (c != m) {
-    if ((c < 0 || c > m) && tid == 0) raise_flag(p.status, SEED_FLAG_BADCOLS);
-    return;
-  }
 
   // 1. panels -> shared memory (TMA bulk copies, no multicast)
   if (tid == 0) {
-    mbar_init(&bar, 1);
-    fence_mbar_init();
     mbar_arrive_expect_tx(&bar, (uint32_t)(m * (DK + DV) * sizeof(float)));
     bulk_g2s(sU, p.U + unit * (long long)m * DK, (uint32_t)(m * DK * sizeof(float)), &bar);
     bulk_g2s(sV, p.V + unit * (long long)m * DV, (uint32_t)(m * DV * sizeof(float)), &bar);
   }
   const int slen = p.slen;
   for (int i = tid; i < slen; i += NT) s_scale[i] = p.scale[unit * slen + i];
-  __syncthreads();   // barrier initialised before anyone polls it
-  if (!mbar_wait_bounded(&bar, 0, kWaitLimitNs)) {
+  __syncthreads();
+  // every thread polls, and the outcome is made uniform so no barrier below diverges
+  if (!__syncthreads_and(mbar_wait_bounded(&bar, phase, kWaitLimitNs))) {
     if (tid == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
-    mbar_wait_bounded(&bar, 0, kWaitLimitNs);
+    mbar_wait_bounded(&bar, phase, kWaitLimitNs);
+    __syncthreads();
     return;
   }
   // fold the lazy decay into U
@@ -266,13 +256,55 @@ __global__ void __launch_bounds__(NT) compress_kernel(const CompressParams p) {
     }
   }
   if (p.sigma_out) {
-    const long long srow = p.layer < 0 ? unit : (long long)blockIdx.x;
     for (int r = tid; r < p.R; r += NT) p.sigma_out[srow * p.R + r] = sig[sel[r]];
   }
   for (int i = tid; i < slen; i += NT) p.scale[unit * slen + i] = 1.f;
   if (tid == 0) p.ncols[unit] = p.R;
   if (!conv && tid == 0) raise_flag(p.status, SEED_FLAG_NOCONVERGE);
   if (bad && conv) raise_flag(p.status, SEED_FLAG_NONFINITE);
+  __syncthreads();
+}
+
+// Scans the scope in chunks of NT units, collects those holding R + W columns and
+// compresses them one after the other with the whole CTA.  A modest grid suffices:
+// after the fast kernel this pass normally finds nothing left to do.
+template <int FORM, int DK, int DV, int NT>
+__global__ void __launch_bounds__(NT) compress_kernel(const CompressParams p) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int s_list[NT];
+  __shared__ int s_cnt;
+  const int tid = threadIdx.x;
+  const int m = p.R + p.W;
+  const int per = p.layer < 0 ? p.L * p.H : p.H;
+  const long long total = (long long)p.B * per;
+  if (tid == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  uint32_t phase = 0;
+  for (long long base = (long long)blockIdx.x * NT; base < total; base += (long long)gridDim.x * NT) {
+    if (tid == 0) s_cnt = 0;
+    __syncthreads();
+    const long long idx = base + tid;
+    if (idx < total) {
+      const long long b = idx / per, rest = idx - b * per;
+      const long long unit = p.layer < 0 ? idx : (b * p.L + p.layer) * p.H + rest;
+      const int c = p.ncols[unit];
+      if (c == m) s_list[atomicAdd(&s_cnt, 1)] = (int)(idx - base);
+      else if (c < 0 || c > m) raise_flag(p.status, SEED_FLAG_BADCOLS);
+    }
+    __syncthreads();
+    const int n = s_cnt;
+    for (int k = 0; k < n; ++k) {
+      const long long i2 = base + s_list[k];
+      const long long b = i2 / per, rest = i2 - b * per;
+      const long long unit = p.layer < 0 ? i2 : (b * p.L + p.layer) * p.H + rest;
+      compress_unit<FORM, DK, DV, NT>(p, unit, i2, smem_raw, bar, phase);
+      phase ^= 1u;
+    }
+    __syncthreads();
+  }
 }
 
 static size_t compress_smem_bytes(int form, int dk, int dv, int R, int W, int nt) {
@@ -292,7 +324,8 @@ static int launch_compress_t(const CompressParams& p, int blocks, cudaStream_t s
         cudaSuccess)
       return SEED_ERR_CUDA;
   }
-  kern<<<blocks, NT, smem, st>>>(p);
+  const int grid = (blocks + NT - 1) / NT < 1184 ? (blocks + NT - 1) / NT : 1184;
+  kern<<<grid, NT, smem, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? SEED_OK : SEED_ERR_CUDA;
 }
 
@@ -309,6 +342,10 @@ static int launch_compress_t(const CompressParams& p, int blocks, cudaStream_t s
 
 int launch_compress(const seed_dims& d, const seed_state& s, int layer, float* sigma_out,
                     uint32_t* status, cudaStream_t st) {
+  if (compress_fast_supported(d)) {
+    const int rc = launch_compress_fast(d, s, layer, sigma_out, status, st);
+    if (rc != SEED_OK) return rc;
+  }
   CompressParams p{s.U, s.V, s.scale, s.ncols, sigma_out, status,
                    d.batch, d.layers, d.heads, layer, d.R, d.W, scale_len(d)};
   const int blocks = d.batch * d.heads * (layer < 0 ? d.layers : 1);

@@ -97,6 +97,18 @@ constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
 
 SEED_DEV void consumer_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
+// Barrier over the consumer warps that also ANDs a predicate across them.
+SEED_DEV bool consumer_and(bool v) {
+  uint32_t out;
+  asm volatile(
+      "{\n .reg .pred pi, po;\n setp.ne.u32 pi, %1, 0;\n bar.red.and.pred po, 1, 128, pi;\n"
+      " selp.u32 %0, 1, 0, po;\n}"
+      : "=r"(out)
+      : "r"((uint32_t)v)
+      : "memory");
+  return out != 0;
+}
+
 template <int FORM, int DK, int DV, int MAXC, int NS>
 __global__ void __launch_bounds__(kDecodeThreads) decode_step_kernel(const DecodeParams p) {
   using Stage = DecodeStage<FORM, DK, DV, MAXC>;
@@ -204,7 +216,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_step_kernel(const Decod
   for (int i = 0, u = blockIdx.x; u < n_units; u += gridDim.x, ++i) {
     const int s = i % NS;
     const uint32_t ph = (uint32_t)(i / NS) & 1u;
-    if (!mbar_wait_bounded(&full[s], ph, kWaitLimitNs)) {
+    if (!consumer_and(mbar_wait_bounded(&full[s], ph, kWaitLimitNs))) {
       if (tid == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
       mbar_wait_bounded(&full[s], ph, kWaitLimitNs);   // let copies in flight land
       return;

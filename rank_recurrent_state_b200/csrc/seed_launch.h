@@ -22,6 +22,10 @@ int launch_decode_step(const seed_dims& d, const seed_state& s, int layer, const
                        const float* k, const float* v, const float* alpha, const float* beta,
                        float* o, uint32_t* status, cudaStream_t st);
 
+bool compress_fast_supported(const seed_dims& d);
+int launch_compress_fast(const seed_dims& d, const seed_state& s, int layer, float* sigma_out,
+                         uint32_t* status, cudaStream_t st);
+
 int launch_compress(const seed_dims& d, const seed_state& s, int layer, float* sigma_out,
                     uint32_t* status, cudaStream_t st);
 

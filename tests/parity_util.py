@@ -84,18 +84,24 @@ def max_decay(cfg, dev, n_decode) -> np.ndarray:
 def compare(cfg, dev, ref, tol=TOL, max_tie_frac=0.25):
     """Device against oracle.
 
-    Units whose smallest relative singular gap at R (conversion and every
-    compression) is below GAP_TOL are near-ties: several truncations are correct
-    there, so for them only what is unique is compared (the kept singular values
+    Units whose relative singular gap (sigma_R - sigma_{R+1}) / sigma_1 falls below
+    GAP_TOL at the conversion or at a compression where sigma_R / sigma_1 exceeds
+    the tolerance are near-ties: several truncations are correct there, so for them only what is unique is compared (the kept singular values
     and the sink coefficient a, which no truncation touches) and the state is
     checked for validity against the open-loop bound of Corollary 4 (distance to
     the never-compressed dense state at most eps_bar / (1 - g_bar^W)).  Every
     other unit is compared in full, per unit and pooled.  Bookkeeping is bit-exact.
     """
     n = dev["o"].shape[1]
-    gaps = [ref["conv_gap"]] + ([ref["gap"][i] for i in range(ref["gap"].shape[0])])
-    min_gap = np.min(np.stack(gaps), axis=0)
-    ties = min_gap < GAP_TOL
+    # a truncation is ambiguous where sigma_R and sigma_{R+1} nearly coincide AND the
+    # discarded/kept direction carries energy above the tolerance; below it any choice
+    # changes the state by less than the tolerance and the unit is compared in full
+    gaps = [ref["conv_gap"]] + [ref["gap"][i] for i in range(ref["gap"].shape[0])]
+    sigs = [ref["conv_sigma"]] + [ref["sigma"][i] for i in range(ref["sigma"].shape[0])]
+    ties = np.zeros(n, dtype=bool)
+    for g, sg in zip(gaps, sigs):
+        top = np.where(sg[:, 0] > 0, sg[:, 0], 1.0)
+        ties |= (g < GAP_TOL) & (sg[:, -1] > tol * top)
     ok = ~ties
     errs = {"o": [], "S": [], "sigma": [], "a": []}
     for u in range(n):
