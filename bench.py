@@ -47,7 +47,9 @@ def parse_args(argv=None):
     ap.add_argument("--config", type=int, default=2, help="workload id (2: the full GDN stack)")
     ap.add_argument("--batch", type=int, default=None, help="requests per GPU (default: the workload's)")
     ap.add_argument("--prefill", type=int, default=None, help="prefill tokens (default: the workload's)")
-    ap.add_argument("--input-steps", type=int, default=16, help="distinct pre-generated input steps")
+    ap.add_argument("--input-steps", type=int, default=48,
+                    help="distinct pre-generated input steps, cycled (>= 3 W so that a key comes "
+                         "back only after its old copy has decayed)")
     ap.add_argument("--dense-steps", type=int, default=8)
     ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -367,7 +369,8 @@ def run_ours(args, world, rank, local):
                      "ns_per_head_step_amortized": 1e6 * sum(cmp_ms) / (args.steps * units) if cmp_ms else 0.0,
                      "share_of_step": sum(cmp_ms) / elapsed_ms,
                      "jacobi_sweeps_mean": (diag["compress_sweeps"] / diag["compress_units"]
-                                            if diag["compress_units"] else None)},
+                                            if diag["compress_units"] else None),
+                     "cholqr_units": diag["cholqr_units"], "householder_units": diag["householder_units"]},
         "gpu_launches": len(dec_ms) + len(cmp_ms),
         "status_flags": flags | flags_warm,
         "setup_s": t_setup,

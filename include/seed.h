@@ -186,10 +186,12 @@ int seed_dense_step(const seed_dims* dims, float* S, int32_t layer, const float*
  * clears them.  Returns SEED_OK or SEED_ERR_CUDA.                                   */
 int seed_get_status(void* ws, void* stream, uint32_t* flags);
 
-/* Synchronises `stream`, copies four diagnostic counters kept next to the status
- * word and clears them: [0] Jacobi sweeps run by seed_compress, [1] units it
- * compressed, [2] Jacobi sweeps run by seed_state_init_from_dense, [3] units it
- * converted.  Returns SEED_OK or SEED_ERR_CUDA.                                     */
+/* Synchronises `stream`, copies six diagnostic counters kept next to the status
+ * word into counters[0..5] and clears them: [0] Jacobi sweeps run by seed_compress,
+ * [1] units compressed by its Householder path, [2] Jacobi sweeps run by
+ * seed_state_init_from_dense, [3] units it converted, [4] units compressed by the
+ * Cholesky-QR path, [5] units the Cholesky-QR path left to the Householder path.
+ * Returns SEED_OK or SEED_ERR_CUDA.                                                 */
 int seed_get_diagnostics(void* ws, void* stream, uint32_t* counters);
 
 /* Static description of a seed_status code. */

@@ -10,7 +10,8 @@
 
 namespace {
 
-constexpr size_t kWorkspaceBytes = 256;   // the device status word, padded
+constexpr size_t kWorkspaceBytes = 256;   // the device status word and counters, padded
+constexpr int kDiagCounters = 6;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -177,13 +178,13 @@ int seed_get_diagnostics(void* ws, void* stream, uint32_t* counters) {
   if (!counters) return SEED_ERR_INVALID_ARG;
   SEED_TRY(check_ws(ws, kWorkspaceBytes));
   cudaStream_t st = as_stream(stream);
-  uint32_t host[4] = {0, 0, 0, 0};
+  uint32_t host[kDiagCounters] = {0};
   uint32_t* dev = status_word(ws) + 1;
   if (cudaMemcpyAsync(host, dev, sizeof(host), cudaMemcpyDeviceToHost, st) != cudaSuccess)
     return SEED_ERR_CUDA;
   if (cudaMemsetAsync(dev, 0, sizeof(host), st) != cudaSuccess) return SEED_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return SEED_ERR_CUDA;
-  for (int i = 0; i < 4; ++i) counters[i] = host[i];
+  for (int i = 0; i < kDiagCounters; ++i) counters[i] = host[i];
   return SEED_OK;
 }
 

@@ -100,14 +100,14 @@ SEED_DEV void block_uniforms(uint4 w, double u[4]) {
 // n_cols must be even (callers pad with a zero column).  Called by all threads of
 // the block; each pair is handled by a group of G lanes (G a power of two <= 32).
 //
-// Columns whose squared norm is below 1e-10 ||A||_F^2 are treated as zero: their
-// pairs are not rotated.  Such columns are rounding noise (or exact zeros) once
-// n_cols exceeds the rank, and a relative threshold alone would keep rotating
-// them for ever; their contribution is below 1e-5 of ||A||_F.
+// Columns whose squared norm is below tiny_rel ||A||_F^2 are treated as zero:
+// their pairs are not rotated.  Such columns are rounding noise (or exact zeros)
+// where n_cols exceeds the rank, and a relative threshold alone would keep
+// rotating them for ever; their contribution is below sqrt(tiny_rel) ||A||_F.
 // Returns the number of sweeps run (max_sweeps + 1 if it did not converge).
 template <int NT>
 __device__ int jacobi_svd(float* A, int lda, int n_rows, float* Z, int ldz, int n_cols, float tol,
-                          int max_sweeps, float* s_red) {
+                          int max_sweeps, float* s_red, float tiny_rel) {
   const int tid = threadIdx.x;
   const int npairs = n_cols / 2;
   int G = 32;
@@ -129,7 +129,7 @@ __device__ int jacobi_svd(float* A, int lda, int n_rows, float* Z, int ldz, int 
   __syncthreads();
   float frob2 = 0.f;
   for (int w = 0; w < NT / 32; ++w) frob2 += s_red[w];
-  const float tiny = 1e-10f * frob2;
+  const float tiny = tiny_rel * frob2;
   __syncthreads();
 
   for (int sweep = 0; sweep < max_sweeps; ++sweep) {

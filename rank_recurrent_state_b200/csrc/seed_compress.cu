@@ -149,7 +149,9 @@ __device__ void compress_unit(const CompressParams& p, long long unit, long long
   float* sig = tau_v + m;                                    // mp
   float* s_red = sig + mp;                                   // NW
   float* s_scale = s_red + NW;                               // KDA ? DK : m
-  int* sel = reinterpret_cast<int*>(s_scale + (KDA ? DK : ((m + 3) & ~3)));  // R
+  float* cs_u = s_scale + (KDA ? DK : ((m + 3) & ~3));      // m: column scales of U
+  float* cs_v = cs_u + m;                                    // m: column scales of V
+  int* sel = reinterpret_cast<int*>(cs_v + m);               // R
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   // 1. panels -> shared memory (TMA bulk copies, no multicast)
@@ -168,29 +170,54 @@ __device__ void compress_unit(const CompressParams& p, long long unit, long long
     __syncthreads();
     return;
   }
-  // fold the lazy decay into U
-  for (int idx = tid; idx < m * DK; idx += NT) {
-    const int j = idx / DK, i = idx - j * DK;
-    sU[idx] *= KDA ? s_scale[i] : s_scale[j];
+  // KDA's per-row decay is folded into the panel (P >= 0.85^W stays far from
+  // underflow); the per-column decay of GDN / Mamba-2 stays a column factor
+  if constexpr (KDA) {
+    for (int idx = tid; idx < m * DK; idx += NT) {
+      const int i = idx % DK;
+      sU[idx] *= s_scale[i];
+    }
+    __syncthreads();
+  }
+  // column equilibration by the largest magnitude: the QR then never squares
+  // values near the float32 underflow (a long-decayed column may hold 1e-30), where
+  // reflectors built from denormals lose their orthogonality
+  for (int j = warp; j < 2 * m; j += NW) {
+    const bool isU = j < m;
+    const int col = isU ? j : j - m;
+    float* x = isU ? sU + col * DK : sV + col * DV;
+    const int n = isU ? DK : DV;
+    float mx = 0.f;
+    for (int i = lane; i < n; i += 32) mx = fmaxf(mx, fabsf(x[i]));
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    const float inv = mx > 0.f ? 1.f / mx : 0.f;
+    for (int i = lane; i < n; i += 32) x[i] *= inv;
+    if (lane == 0) {
+      if (isU) cs_u[col] = mx * (KDA ? 1.f : s_scale[col]);
+      else cs_v[col] = mx;
+    }
   }
   __syncthreads();
 
-  // 2. QR of both panels
+  // 2. QR of both equilibrated panels
   householder_qr<NT>(sU, DK, m, tau_u, s_red);
   householder_qr<NT>(sV, DV, m, tau_v, s_red);
 
-  // 3. core M = R_u R_v^T, column-major with ld m+1 (plus a zero column if m is odd)
+  // 3. core M = R_u R_v^T = Rhat_u diag(cs_u cs_v) Rhat_v^T, column-major with ld
+  //    m+1 (plus a zero column if m is odd)
   for (int idx = tid; idx < mp * m; idx += NT) {
     const int j = idx / m, i = idx - j * m;   // M[i][j]
     float acc = 0.f;
     if (j < m) {
-      for (int k = max(i, j); k < m; ++k) acc = fmaf(sU[k * DK + i], sV[k * DV + j], acc);
+      for (int k = max(i, j); k < m; ++k)
+        acc = fmaf(sU[k * DK + i] * (cs_u[k] * cs_v[k]), sV[k * DV + j], acc);
     }
     sM[j * ldm + i] = acc;
   }
   __syncthreads();
   const float tol = 8.f * sqrtf((float)m) * 5.9604645e-8f;
-  const int sweeps = jacobi_svd<NT>(sM, ldm, m, sZ, ldz, mp, tol, 40, s_red);
+  const int sweeps = jacobi_svd<NT>(sM, ldm, m, sZ, ldz, mp, tol, 40, s_red, 1e-10f);
   const bool conv = sweeps <= 40;
   if (tid == 0) {
     atomicAdd(p.status + 1, (uint32_t)sweeps);
@@ -310,7 +337,7 @@ __global__ void __launch_bounds__(NT) compress_kernel(const CompressParams p) {
 static size_t compress_smem_bytes(int form, int dk, int dv, int R, int W, int nt) {
   const int m = R + W, mp = m + (m & 1);
   size_t f = (size_t)m * dk + (size_t)m * dv + (size_t)mp * (m + 1) + (size_t)mp * (mp + 1) +
-             2 * m + mp + nt / 32 + (form == SEED_KDA ? dk : ((m + 3) & ~3)) + R;
+             2 * m + mp + nt / 32 + (form == SEED_KDA ? dk : ((m + 3) & ~3)) + 2 * m + R;
   return f * sizeof(float) + 16;
 }
 
@@ -371,18 +398,25 @@ struct InitParams {
   int B, L, H, layer, R, W, form, slen;
 };
 
+// The one-sided Jacobi runs over the shorter side of C so that the columns it
+// orthogonalises are at most as many as their length: over the d_v columns of C
+// when d_k >= d_v, else over the d_k columns of C^T.  Either way at most one
+// column is a structural null direction (C vbar = 0), not many.
 template <int DK, int DV, int NT>
 __global__ void __launch_bounds__(NT) init_kernel(const InitParams p) {
   constexpr int NW = NT / 32;
-  constexpr int LDC = DV + 1;   // padded rows of C (= columns of C^T) for the Jacobi
-  constexpr int LDZ = DK + 1;
+  constexpr bool COLS = DK >= DV;       // Jacobi over the columns of C
+  constexpr int NC = COLS ? DV : DK;    // Jacobi columns
+  constexpr int NR = COLS ? DK : DV;    // their length
+  constexpr int LDC = NR + 1;
+  constexpr int LDZ = NC + 1;
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  float* sC = reinterpret_cast<float*>(smem_raw);   // DK columns of length DV (rows of C)
-  float* sZ = sC + DK * LDC;                         // DK x DK
-  float* s_vb = sZ + DK * LDZ;                       // DV
+  float* sC = reinterpret_cast<float*>(smem_raw);   // NC columns of length NR
+  float* sZ = sC + NC * LDC;                         // NC x NC
+  float* s_vb = sZ + NC * LDZ;                       // DV
   float* s_a = s_vb + DV;                            // DK
-  float* sig = s_a + DK;                             // DK
-  float* s_red = sig + DK;                           // NW
+  float* sig = s_a + DK;                             // NC
+  float* s_red = sig + NC;                           // NW
   int* sel = reinterpret_cast<int*>(s_red + NW);     // R
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int units_in_scope = p.layer < 0 ? p.L * p.H : p.H;
@@ -397,12 +431,13 @@ __global__ void __launch_bounds__(NT) init_kernel(const InitParams p) {
   for (int i = tid; i < DV; i += NT) s_vb[i] = p.vbar[((long long)l * p.H + h) * DV + i];
   for (int idx = tid; idx < DK * DV / 4; idx += NT) {
     const float4 x = ld4(S + 4 * idx);
-    const int i = (4 * idx) / DV, j = (4 * idx) - i * DV;
-    float* dst = sC + i * LDC + j;
-    dst[0] = x.x;
-    dst[1] = x.y;
-    dst[2] = x.z;
-    dst[3] = x.w;
+    const int i = (4 * idx) / DV, j = (4 * idx) - i * DV;   // S[i][j .. j+3]
+    const float xv[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (COLS) sC[(j + e) * LDC + i] = xv[e];
+      else sC[i * LDC + j + e] = xv[e];
+    }
   }
   __syncthreads();
   float vv = 0.f;
@@ -417,51 +452,62 @@ __global__ void __launch_bounds__(NT) init_kernel(const InitParams p) {
     if (tid == 0) raise_flag(p.status, SEED_FLAG_ZERO_VBAR);
     return;
   }
-  // a = S vbar / ||vbar||^2 (warp per row), then C = S - a vbar^T in place
-  for (int i = warp; i < DK; i += NW) {
-    float acc = 0.f;
-    for (int j = lane; j < DV; j += 32) acc = fmaf(sC[i * LDC + j], s_vb[j], acc);
-    acc = group_sum<32>(acc) / vbvb;
-    for (int j = lane; j < DV; j += 32) sC[i * LDC + j] = fmaf(-acc, s_vb[j], sC[i * LDC + j]);
-    if (lane == 0) s_a[i] = acc;
+  // a = S vbar / ||vbar||^2, then C = S - a vbar^T in place
+  if (COLS) {
+    for (int i = tid; i < DK; i += NT) {
+      float acc = 0.f;
+      for (int j = 0; j < DV; ++j) acc = fmaf(sC[j * LDC + i], s_vb[j], acc);
+      acc /= vbvb;
+      for (int j = 0; j < DV; ++j) sC[j * LDC + i] = fmaf(-acc, s_vb[j], sC[j * LDC + i]);
+      s_a[i] = acc;
+    }
+  } else {
+    for (int i = warp; i < DK; i += NW) {
+      float acc = 0.f;
+      for (int j = lane; j < DV; j += 32) acc = fmaf(sC[i * LDC + j], s_vb[j], acc);
+      acc = group_sum<32>(acc) / vbvb;
+      for (int j = lane; j < DV; j += 32) sC[i * LDC + j] = fmaf(-acc, s_vb[j], sC[i * LDC + j]);
+      if (lane == 0) s_a[i] = acc;
+    }
   }
   __syncthreads();
-  const float tol = 8.f * sqrtf((float)DV) * 5.9604645e-8f;
-  const int sweeps = jacobi_svd<NT>(sC, LDC, DV, sZ, LDZ, DK, tol, 60, s_red);
+  const float tol = 8.f * sqrtf((float)NR) * 5.9604645e-8f;
+  const int sweeps = jacobi_svd<NT>(sC, LDC, NR, sZ, LDZ, NC, tol, 60, s_red, 1e-12f);
   const bool conv = sweeps <= 60;
   if (tid == 0) {
     atomicAdd(p.status + 3, (uint32_t)sweeps);
     atomicAdd(p.status + 4, 1u);
   }
-  for (int j = tid; j < DK; j += NT) {
+  for (int j = tid; j < NC; j += NT) {
     float s2 = 0.f;
-    for (int i = 0; i < DV; ++i) s2 = fmaf(sC[j * LDC + i], sC[j * LDC + i], s2);
+    for (int i = 0; i < NR; ++i) s2 = fmaf(sC[j * LDC + i], sC[j * LDC + i], s2);
     sig[j] = sqrtf(s2);
   }
   __syncthreads();
-  select_top<NT>(sig, DK, p.R, sel);
+  select_top<NT>(sig, NC, p.R, sel);
   __syncthreads();
   float smax = 0.f;
-  for (int j = 0; j < DK; ++j) smax = fmaxf(smax, sig[j]);
+  for (int j = 0; j < NC; ++j) smax = fmaxf(smax, sig[j]);
   const float szero = (float)max(DK, DV) * 1.1920929e-7f * smax;
 
-  // U[:, r] = Z[:, j] sqrt(s), V[:, r] = (C^T Z)[:, j] / sqrt(s), j the r-th largest
+  // COLS: U[:, r] = (C Z)[:, j] / sqrt(s), V[:, r] = Z[:, j] sqrt(s)
+  // else: U[:, r] = Z[:, j] sqrt(s),       V[:, r] = (C^T Z)[:, j] / sqrt(s)
   float* Ug = p.U + unit * (long long)m * DK;
   float* Vg = p.V + unit * (long long)m * DV;
   bool bad = !conv;
   for (int r = warp; r < p.R; r += NW) {
-    const bool valid = r < DK;
+    const bool valid = r < NC;
     const int j = valid ? sel[r] : 0;
     const float s = valid ? sig[j] : 0.f;
     const bool zero = !(s > szero);
-    const float fu = zero ? 0.f : sqrtf(s), fv = zero ? 0.f : rsqrtf(s);
+    const float fz = zero ? 0.f : sqrtf(s), fc = zero ? 0.f : rsqrtf(s);
     for (int e = lane; e < DK; e += 32) {
-      const float x = fu * sZ[j * LDZ + e];
+      const float x = COLS ? fc * sC[j * LDC + e] : fz * sZ[j * LDZ + e];
       bad |= !isfinite(x);
       Ug[(long long)r * DK + e] = x;
     }
     for (int e = lane; e < DV; e += 32) {
-      const float x = fv * sC[j * LDC + e];
+      const float x = COLS ? fz * sZ[j * LDZ + e] : fc * sC[j * LDC + e];
       bad |= !isfinite(x);
       Vg[(long long)r * DV + e] = x;
     }
@@ -480,7 +526,8 @@ __global__ void __launch_bounds__(NT) init_kernel(const InitParams p) {
 template <int FORM, int DK, int DV>
 static int launch_init_t(const InitParams& p, int blocks, cudaStream_t st) {
   constexpr int NT = 256;
-  const size_t smem = ((size_t)DK * (DV + 1) + (size_t)DK * (DK + 1) + DV + 2 * DK + NT / 32 +
+  constexpr int NC = DK >= DV ? DV : DK, NR = DK >= DV ? DK : DV;
+  const size_t smem = ((size_t)NC * (NR + 1) + (size_t)NC * (NC + 1) + DV + DK + NC + NT / 32 +
                        p.R) * sizeof(float) + 16;
   auto kern = init_kernel<DK, DV, NT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=

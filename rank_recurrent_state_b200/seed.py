@@ -195,10 +195,11 @@ def seed_get_status(ws: Workspace, stream=None) -> int:
 
 
 def seed_get_diagnostics(ws: Workspace, stream=None) -> dict:
-    c = (_lib.c_uint32 * 4)()
+    c = (_lib.c_uint32 * 6)()
     _check("seed_get_diagnostics", _lib.load().seed_get_diagnostics(ws.ptr, _stream(stream), c))
-    return {"compress_sweeps": c[0], "compress_units": c[1], "convert_sweeps": c[2],
-            "convert_units": c[3]}
+    return {"compress_sweeps": c[0], "householder_units": c[1], "convert_sweeps": c[2],
+            "convert_units": c[3], "cholqr_units": c[4], "cholqr_declined": c[5],
+            "compress_units": c[1] + c[4]}
 
 
 # ------------------------------------------------------------------ synthetic workloads

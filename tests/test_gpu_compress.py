@@ -86,11 +86,60 @@ def test_compress_matches_truncated_svd(form, dk, dv, R, W):
 
 def test_repeated_key_takes_the_householder_path():
     diag = _run(FORM_GDN, 128, 128, 16, 16, repeat=True, n=8, seed=7)
-    # the fast path declines every unit (the Householder pass counts its Jacobi
-    # sweeps as well, so both passes' units appear in the counter)
-    assert diag["compress_units"] >= 8
+    assert diag["cholqr_declined"] == 8 and diag["householder_units"] == 8
+
+
+def test_well_conditioned_units_take_the_cholesky_qr_path():
+    diag = _run(FORM_GDN, 128, 128, 16, 16, n=16, seed=11)
+    assert diag["cholqr_units"] == 16 and diag["householder_units"] == 0
 
 
 def test_zero_columns_are_dropped_exactly():
     _run(FORM_GDN, 128, 128, 16, 16, zero_cols=5, n=8, seed=9)
     _run(FORM_KDA, 128, 128, 16, 16, zero_cols=16, n=8, seed=10)
+
+
+def _graded_state(form, n, dk, dv, R, W, rng, lazy):
+    """Columns whose magnitudes span 1 .. 1e-30, as a long-decayed window leaves them:
+    either explicit in the stored U (scale 1) or carried by the lazy decay scales."""
+    m = R + W
+    mags = 10.0 ** (-rng.uniform(0, 30, size=(n, m)))
+    mags[:, -4:] = rng.uniform(0.5, 1.0, size=(n, 4))          # the newest columns
+    U = rng.normal(size=(n, dk, m))
+    U /= np.linalg.norm(U, axis=1, keepdims=True)
+    V = rng.normal(size=(n, dv, m)) * rng.uniform(0.2, 3, size=(n, 1, m))
+    slen = (m + 3) // 4 * 4
+    scale = np.ones((n, slen))
+    if lazy:
+        scale[:, :m] = mags
+    else:
+        U = U * mags[:, None, :]
+    Utrue = U * scale[:, None, :m]
+    return U.astype(np.float32), V.astype(np.float32), scale.astype(np.float32), Utrue
+
+
+@pytest.mark.parametrize("lazy", [False, True])
+@pytest.mark.parametrize("dk,dv,R,W", [(128, 128, 16, 16), (128, 64, 8, 32)])
+def test_graded_spectrum_with_long_decayed_columns(lazy, dk, dv, R, W):
+    import torch
+    from rank_recurrent_state_b200 import seed as S
+    rng = np.random.default_rng(21 + R + W + int(lazy))
+    n, m = 12, R + W
+    U, V, scale, Utrue = _graded_state(FORM_GDN, n, dk, dv, R, W, rng, lazy)
+    d = S.Dims(FORM_GDN, n, 1, 1, dk, dv, R, W)
+    st = S.State.allocate(d, torch.ones(1, 1, dv, device="cuda"))
+    st.U.copy_(torch.from_numpy(np.ascontiguousarray(np.swapaxes(U, 1, 2))).view_as(st.U))
+    st.V.copy_(torch.from_numpy(np.ascontiguousarray(np.swapaxes(V, 1, 2))).view_as(st.V))
+    st.scale.copy_(torch.from_numpy(scale).view_as(st.scale))
+    st.a.zero_()
+    st.ncols.fill_(m)
+    ws = S.Workspace(d)
+    S.seed_compress(d, st, S.SEED_ALL_LAYERS, ws)
+    dense = torch.empty(n, dk, dv, device="cuda")
+    S.seed_state_to_dense(d, st, S.SEED_ALL_LAYERS, dense, ws)
+    assert S.seed_get_status(ws) == 0
+    Up, Vp, _ = ocomp.truncate_product(Utrue.astype(np.float64), V.astype(np.float64), R)
+    ref = np.einsum("nir,njr->nij", Up, Vp)
+    got = dense.cpu().numpy()
+    for u in range(n):
+        assert rel_fro(got[u], ref[u]) <= TOL, (u, rel_fro(got[u], ref[u]))
