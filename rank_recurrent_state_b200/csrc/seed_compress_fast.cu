@@ -315,7 +315,7 @@ __global__ void __launch_bounds__(64) compress_fast_kernel(const FastParams p) {
       const float al = active ? nrm[P] : 0.f, be = active ? nrm[Q] : 0.f;
       // rotation test and parameters with the fast intrinsics: t need not be the
       // exact tangent, the rotation stays orthogonal because c = 1 / sqrt(1 + t^2)
-      if (active && al > tiny && be > tiny && g * g > (tol * tol) * al * be) {
+      if (active && al > tiny && be > tiny && fabsf(g) > tol * sqrtf(al) * sqrtf(be)) {
         const float zeta = __fdividef(be - al, 2.f * g);
         float t;
         if (fabsf(zeta) > 1e18f) t = __fdividef(0.5f, zeta);
