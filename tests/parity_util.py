@@ -71,6 +71,36 @@ def run_oracle(cfg, dev, n_prefill, n_decode):
                           keep_shadow=True)
 
 
+_UNIT_AXIS1 = ("o", "a_t", "sigma", "gap", "tail", "err_open", "sink_dev")
+_SHARED = ("ncols", "comp_steps")
+
+
+def _oracle_chunk(args):
+    from oracle import run as orun
+    cfg, b, l, h, n_prefill, n_decode = args
+    return orun.run_units(cfg, b, l, h, n_prefill=n_prefill, n_decode=n_decode, keep_shadow=True)
+
+
+def run_oracle_units(cfg, b, l, h, n_prefill, n_decode, workers=8, chunk=8):
+    """The oracle on the sampled units (b, l, h), split into chunks run by a pool of
+    spawned processes (units are independent), merged along the unit axis."""
+    import multiprocessing as mp
+    b, l, h = (np.asarray(x, dtype=np.int64) for x in (b, l, h))
+    parts = [(cfg, b[i:i + chunk], l[i:i + chunk], h[i:i + chunk], n_prefill, n_decode)
+             for i in range(0, b.size, chunk)]
+    with mp.get_context("spawn").Pool(min(workers, len(parts))) as pool:
+        outs = pool.map(_oracle_chunk, parts)
+    merged = {}
+    for key in outs[0]:
+        if key in _SHARED:
+            merged[key] = outs[0][key]
+            for o in outs[1:]:
+                assert np.array_equal(np.asarray(o[key]), np.asarray(outs[0][key])), key
+        else:
+            merged[key] = np.concatenate([o[key] for o in outs], axis=1 if key in _UNIT_AXIS1 else 0)
+    return merged
+
+
 def max_decay(cfg, dev, n_decode) -> np.ndarray:
     """Largest per-step contraction factor over the decode run, per sampled unit
     (g for GDN, alpha for Mamba-2, max_i alpha_i for KDA), from the host generator."""
