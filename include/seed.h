@@ -197,6 +197,31 @@ int seed_get_diagnostics(void* ws, void* stream, uint32_t* counters);
 /* Static description of a seed_status code. */
 const char* seed_status_string(int status);
 
+/* ---- Decode step without a caller workspace.  The SEED paper has no counterpart:
+ * this is a library convenience for callers that cannot allocate device memory
+ * (a host program without a device allocator, an engine that fixes every buffer
+ * before serving).  It runs the same kernel as seed_decode_step, with the status
+ * word in a 256-byte array that lives in libseed.so's device image (one per
+ * device, zero at module load); it calls no allocator.
+ *
+ * Arguments as in seed_decode_step, without ws / ws_bytes, plus
+ *   status_out  optional DEVICE pointer (4-byte aligned) that receives, in stream
+ *               order, the SEED_FLAG_* bits this call raised; NULL discards them.
+ * After the launch the call copies the status word to status_out and clears it,
+ * so every call starts from zero.
+ * Returns seed_decode_step's codes, and SEED_ERR_WORKSPACE if the decode step
+ * for these dims needs more workspace than the fixed 256 bytes (no supported
+ * shape does).  Nothing is enqueued when an argument is rejected.
+ * The first call on each device looks up the array's address and may load the
+ * module onto the device: make it before any stream capture on that device.
+ * All calls on a device share the one array: calls that can run at the same time
+ * (other streams, other host threads) race on the status word; serialise them,
+ * or use seed_decode_step with a workspace each.                                  */
+size_t seed_noalloc_workspace_bytes(void);
+int seed_decode_step_noalloc(const seed_dims* dims, const seed_state* state, int32_t layer,
+                             const float* q, const float* k, const float* v, const float* alpha,
+                             const float* beta, float* o, uint32_t* status_out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -58,6 +58,10 @@ SIGNATURES = {
                                                c_void_p, c_void_p]),
     "seed_synth_dense_prefill": (ctypes.c_int, [ctypes.POINTER(seed_dims), seed_synth_key, c_int32, c_int32,
                                                 c_void_p, c_void_p, c_void_p]),
+    "seed_noalloc_workspace_bytes": (c_size_t, []),
+    "seed_decode_step_noalloc": (ctypes.c_int, [ctypes.POINTER(seed_dims), ctypes.POINTER(seed_state),
+                                                c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                                c_void_p, c_void_p, c_void_p]),
 }
 
 _LIB = None

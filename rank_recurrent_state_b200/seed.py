@@ -164,6 +164,20 @@ def seed_decode_step(dims: Dims, state: State, layer: int, q, k, v, alpha, beta,
         _ptr(o), ws.ptr, ws.nbytes, _stream(stream)))
 
 
+def seed_decode_step_noalloc(dims: Dims, state: State, layer: int, q, k, v, alpha, beta, o,
+                             status_out: torch.Tensor | None = None, stream=None) -> None:
+    """seed_decode_step with the library's own fixed device workspace; status_out, if
+    given, is a device int32/uint32 tensor of one element that receives the flags."""
+    d, s = dims.c(), state.c()
+    _check("seed_decode_step_noalloc", _lib.load().seed_decode_step_noalloc(
+        ctypes.byref(d), ctypes.byref(s), layer, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+        _ptr(o), _ptr(status_out), _stream(stream)))
+
+
+def seed_noalloc_workspace_bytes() -> int:
+    return int(_lib.load().seed_noalloc_workspace_bytes())
+
+
 def seed_compress(dims: Dims, state: State, layer: int, ws: Workspace,
                   sigma_out: torch.Tensor | None = None, stream=None) -> None:
     d, s = dims.c(), state.c()

@@ -125,3 +125,11 @@ def test_other_entry_points_validate(lib):
     assert lib.seed_synth_dense_prefill(ctypes.byref(d), key, -1, 0, A, A, None) == -1
     bad_key = _lib.seed_synth_key(0, 0, 0, -1)
     assert lib.seed_synth_dense_prefill(ctypes.byref(d), bad_key, 4, 0, A, A, None) == -1
+
+
+def test_noalloc_decode_step_validates_before_touching_the_device(lib):
+    d, s = _dims(), _state()
+    assert lib.seed_noalloc_workspace_bytes() >= lib.seed_workspace_bytes(ctypes.byref(d))
+    assert lib.seed_decode_step_noalloc(None, ctypes.byref(s), 0, A, A, A, A, A, A, None, None) == -1
+    assert lib.seed_decode_step_noalloc(ctypes.byref(d), ctypes.byref(s), 0, A, A, A, A, A, A,
+                                        0x10002, None) == -3
