@@ -47,6 +47,8 @@ def parse_args(argv=None):
     ap.add_argument("--config", type=int, default=2, help="workload id (2: the full GDN stack)")
     ap.add_argument("--batch", type=int, default=None, help="requests per GPU (default: the workload's)")
     ap.add_argument("--prefill", type=int, default=None, help="prefill tokens (default: the workload's)")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="layers (default: the workload's; fewer only for a small profiling case)")
     ap.add_argument("--input-steps", type=int, default=48,
                     help="distinct pre-generated input steps, cycled (>= 3 W so that a key comes "
                          "back only after its old copy has decayed)")
@@ -232,6 +234,8 @@ def run_reference(args, world, rank):
     cfg = config(args.config)
     if args.batch:
         cfg = cfg.replace(batch=args.batch)
+    if args.layers:
+        cfg = cfg.replace(layers=args.layers)
     if rank != 0:
         return 0
     per = max(1.0, args.cpu_seconds)
@@ -251,6 +255,22 @@ def run_reference(args, world, rank):
 
 # ------------------------------------------------------------------ GPU arm
 
+def compress_rate(d, diag, cmp_ms, clk):
+    """FP32 rate of the compression launches (the FLOP model of roofline.compress_flops,
+    with the measured mean Jacobi sweeps) and its fraction of the CUDA-core FP32 peak
+    at the median SM clock sampled during the timed region."""
+    from rank_recurrent_state_b200 import roofline
+    if not cmp_ms or not diag["compress_units"]:
+        return {}
+    sweeps = diag["compress_sweeps"] / diag["compress_units"]
+    flops = roofline.compress_flops(d.d_k, d.d_v, d.R, d.W, sweeps) * d.units
+    tflops = flops / (sum(cmp_ms) / len(cmp_ms) / 1e3) / 1e12
+    mhz = (clk or {}).get("sm_mhz") or 1965.0
+    peak = roofline.fp32_peak_tflops(mhz)
+    return {"flops_per_unit": flops / d.units, "tflops": tflops, "fp32_peak_tflops": peak,
+            "frac_fp32_peak": tflops / peak}
+
+
 def run_ours(args, world, rank, local):
     import torch
 
@@ -269,6 +289,8 @@ def run_ours(args, world, rank, local):
     cfg = config(args.config)
     if args.batch:
         cfg = cfg.replace(batch=args.batch)
+    if args.layers:
+        cfg = cfg.replace(layers=args.layers)
     B = cfg.batch
     prefill = cfg.n_prefill if args.prefill is None else args.prefill
     run = DeviceRun(cfg, b0=shard(B, rank), device=str(dev), n_prefill=prefill,
@@ -370,7 +392,8 @@ def run_ours(args, world, rank, local):
                      "share_of_step": sum(cmp_ms) / elapsed_ms,
                      "jacobi_sweeps_mean": (diag["compress_sweeps"] / diag["compress_units"]
                                             if diag["compress_units"] else None),
-                     "cholqr_units": diag["cholqr_units"], "householder_units": diag["householder_units"]},
+                     "cholqr_units": diag["cholqr_units"], "householder_units": diag["householder_units"],
+                     **compress_rate(d, diag, cmp_ms, clk.summary())},
         "gpu_launches": len(dec_ms) + len(cmp_ms),
         "status_flags": flags | flags_warm,
         "setup_s": t_setup,

@@ -69,7 +69,8 @@ typedef enum {
 #define SEED_FLAG_BADINDEX 0x20u  /* seed_state_to_dense met a unit index outside the scope;
                                      that output slab was not written                      */
 #define SEED_FLAG_TIMEOUT 0x40u   /* a bounded wait for a bulk copy gave up (1 s); the unit
-                                     was left unchanged                                    */
+                                     being worked on was left unchanged or, in a
+                                     compression, partly written                          */
 
 /* Supported shapes: (d_k, d_v) equal and in {16, 32, 64, 128}, or (128, 64), or
  * (64, 128); R >= 1, W >= 1, R + W <= SEED_MAX_COLS and R + W <= min(d_k, d_v).
@@ -94,8 +95,9 @@ typedef struct {
  *   U      [B][L][H][R+W][d_k]       content factor U, one contiguous d_k column per slot;
  *                                    slot j holds column j, so appends never move data
  *   V      [B][L][H][R+W][d_v]       content factor V, same slots
- *   scale  GDN, Mamba-2: [B][L][H][ceil4(R+W)] per-column decay scales gamma_j: the true
- *                                    U column j is gamma_j * U[:, j] (decay applied lazily);
+ *   scale  GDN, Mamba-2: [B][L][H][ceil4(R+W)] per-column scales gamma_j: the true
+ *                                    U column j is gamma_j * U[:, j] (decay applied lazily,
+ *                                    and a singular value kept by seed_compress);
  *                                    the per-unit stride is R+W rounded up to a multiple of 4
  *          KDA:          [B][L][H][d_k] per-channel decay products P: the true U is
  *                                    Diag(P) U (per-row decay applied lazily)
@@ -156,11 +158,16 @@ int seed_decode_step(const seed_dims* dims, const seed_state* state, int32_t lay
 /* Periodic compression (SEED figures & tables, Figure 1(b): every W steps the
  * factors are compressed back to rank R; SEED summary, Corollary 4 bounds its
  * open-loop error).  For every unit of `layer` (or all layers) whose ncols equals
- * R+W: QR of U and V by Cholesky of the column-equilibrated Gram matrices, the
- * (R+W) x (R+W) core M = R_u R_v^T, a one-sided Jacobi SVD of M, and
- *     U' = Q_u X_R Sigma_R^{1/2},   V' = Q_v Y_R Sigma_R^{1/2}
- * written to slots 0..R-1; scale <- 1; ncols <- R.  The sink a is not touched.
- * Units with ncols != R+W are left unchanged.
+ * R+W: QR of U and V (true U, scales applied), the (R+W) x (R+W) core
+ * M = R_u R_v^T, a one-sided Jacobi SVD M = X Sigma Y^T, and the rank-R truncation
+ * (Q_u X_R) Sigma_R (Q_v Y_R)^T written to slots 0..R-1; ncols <- R.  The sink a
+ * is not touched.  Units with ncols != R+W are left unchanged.
+ * How Sigma_R is stored depends on the path a unit takes (both represent the same
+ * state): R + W <= 32, R <= 16, d_k, d_v in {64, 128} and a well-conditioned,
+ * well-scaled unit take Cholesky QR, which for GDN and Mamba-2 stores the unit
+ * columns Q_u X_R, Q_v Y_R and scale_r = sigma_r (scale 1 beyond R), and for KDA
+ * Sigma^{1/2} on each side with P <- 1; every other unit takes Householder QR,
+ * which stores Sigma^{1/2} on each side and resets the scales to 1.
  *   sigma_out  optional: [units in scope][R] singular values kept (only compressed
  *              units' rows are written)                                              */
 int seed_compress(const seed_dims* dims, const seed_state* state, int32_t layer,

@@ -1,20 +1,25 @@
 // seed_compress_fast.cu -- the compression of units with R + W <= 32, R <= 16.
 //
 // "Shallow Encoding Emits Deep Memories", SEED figures & tables (thelatestinai.com),
-// Figure 1(b): every W steps the factors are compressed back to rank R.  Two warps
-// per unit, everything in shared memory or registers, no Householder sweeps:
+// Figure 1(b): every W steps the factors are compressed back to rank R.  One warp
+// per unit, no Householder sweeps:
 //
-//   1. TMA copies of both panels (one 512-byte bulk copy per column, into rows
-//      padded by 4 floats so that the Gram loops read without bank conflicts);
-//   2. Gram matrices of the column-equilibrated panels, G = Uhat^T Uhat and
-//      Vhat^T Vhat (warp 0 and warp 1 in parallel), and their Cholesky factors
-//      L_u, L_v, so that U = Q_u R_u, V = Q_v R_v with R = L^T D (D the column
-//      norms, and the lazy decay scales for GDN / Mamba-2);
-//   3. the core M = R_u R_v^T = L_u^T D_u D_v L_v (m x m);
-//   4. one-sided Jacobi on M (Hestenes; round-robin pairs split over both warps,
-//      four lanes per pair; column norms carried by the exact update
-//      a' = a - t g, b' = b + t g and recomputed every sweep), M Z = X Sigma;
-//   5. with X_R the R leading left singular vectors of M (orthonormalised once
+//   1. TMA copy of the U panel (one bulk copy per column, into rows padded by 4
+//      floats so that the Gram loop reads without bank conflicts); the Gram
+//      matrix of the column-equilibrated panel, G = Uhat^T Uhat, and its Cholesky
+//      factor L_u in registers; then the V panel into the same buffer, G_v, L_v.
+//      So U = Q_u R_u, V = Q_v R_v with R = L^T D (D the column norms, and the
+//      lazy decay scales for GDN / Mamba-2);
+//   2. the core M = R_u R_v^T = L_u^T D_u D_v L_v (m x m);
+//   3. one-sided Jacobi on M (Hestenes), M Z = X Sigma, with the columns held in
+//      registers: a column pair per two lanes (four when m <= 16), rotations of
+//      Rutishauser applied to scaled columns (true column = s * stored column,
+//      two FMAs per element pair), column norms carried by the exact update and
+//      recomputed every sweep.  Pair order: recursive halving -- all pairs between
+//      the two halves of the columns (a cyclic shift of one half against the
+//      other), then the same within each half, so that each round moves one
+//      column of each pair between lanes instead of two;
+//   4. with X_R the R leading left singular vectors of M (orthonormalised once
 //      more, in descending order, by two passes of Gram-Schmidt):
 //        U' = Q_u X_R Sigma^{1/2} = Uhat (L_u^{-T} X_R Sigma^{1/2})
 //        V' = A^T U' Sigma^{-1}   = V (D_u L_u X_R Sigma^{-1/2})
@@ -27,6 +32,9 @@
 // Householder kernel (seed_compress.cu) then compresses it.  Exactly zero columns
 // (a rank-deficient start, or a decay scale that underflowed) are dropped, which
 // is exact.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "seed_common.cuh"
 #include "seed_launch.h"
 #include "seed_tma.cuh"
@@ -44,8 +52,13 @@ struct FastParams {
 };
 
 constexpr float kCholPivotMin = 1e-2f;
-
-SEED_DEV void pair_sync() { asm volatile("bar.sync 1, 64;" ::: "memory"); }
+constexpr int kFastMaxR = 16;
+constexpr int kJacobiMaxSweeps = 30;
+constexpr unsigned kFull = 0xffffffffu;
+// Stored columns whose largest magnitude lies outside [2^-50, 2^50] (zero allowed)
+// could under- or overflow the float32 Gram; such units go to the Householder path.
+constexpr float kColMin = 8.8817842e-16f;   // 2^-50
+constexpr float kColMax = 1.1258999e15f;    // 2^50
 
 template <int PER>
 struct VecT;
@@ -90,75 +103,292 @@ SEED_DEV float equilibrate_row(float (&g)[MP]) {
   const float n = sqrtf(fmaxf(d, 0.f));
   const float ninv = n > 0.f ? 1.f / n : 0.f;
 #pragma unroll
-  for (int i = 0; i < MP; ++i) g[i] *= __shfl_sync(0xffffffffu, ninv, i) * ninv;
+  for (int i = 0; i < MP; ++i) g[i] *= __shfl_sync(kFull, ninv, i) * ninv;
   return lane < MP ? n : 0.f;
 }
 
 // Right-looking Cholesky in registers, one warp, lane i holding row i of the
 // equilibrated Gram; on return row i of L (lower; the upper part zero).  Column j
 // is dropped (zero) when column j of the panel is zero (norm_j == 0) or the pivot
-// is not positive; a pivot below kCholPivotMin on a nonzero column also sets *bad.
+// is not positive; a pivot below kCholPivotMin on a nonzero column sets `bad`.
 template <int MP>
-SEED_DEV void cholesky_regs(float (&g)[MP], float norm_self, int* bad) {
+SEED_DEV void cholesky_regs(float (&g)[MP], float norm_self, bool& bad) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int j = 0; j < MP; ++j) {
-    const float d = __shfl_sync(0xffffffffu, g[j], j);
-    const bool zero = !(__shfl_sync(0xffffffffu, norm_self, j) > 0.f);
+    const float d = __shfl_sync(kFull, g[j], j);
+    const bool zero = !(__shfl_sync(kFull, norm_self, j) > 0.f);
     bool drop = zero || !(d > 0.f);
     if (!zero && d < kCholPivotMin) {
       drop = true;
-      if (lane == 0) *bad = 1;
+      bad = true;
     }
     const float rs = drop ? 0.f : rsqrtf(d);
     const float lij = lane > j ? g[j] * rs : 0.f;
     g[j] = lane == j ? d * rs : lij;
 #pragma unroll
     for (int k = j + 1; k < MP; ++k) {
-      const float lkj = __shfl_sync(0xffffffffu, lij, k);
+      const float lkj = __shfl_sync(kFull, lij, k);
       if (k <= lane) g[k] = fmaf(-lij, lkj, g[k]);
     }
   }
 }
 
-// Shared memory: the two panels (region A) are only read by the Gram phase; every
-// later buffer aliases region A.  The small per-column arrays live after it.
+// Lanes of one column pair (LP lanes, aligned) sum their partial values.
+template <int LP>
+SEED_DEV float pair_sum(float v) {
+#pragma unroll
+  for (int off = LP / 2; off >= 1; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
+  return v;
+}
+
+SEED_DEV float warp_max(float v) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, off));
+  return v;
+}
+
+// One-sided Jacobi on the MP x MP matrix in sM (column-major, stride LM), in
+// registers.  Slot s = lane / LP holds the column pair (x, y); lane part h holds
+// rows h*NR .. h*NR+NR-1 of both.  The matrix must be scaled so that its squared
+// column norms stay far from the float32 range limits (entries of order one).
+// Returns the sweeps run; `conv` is set when the last sweep rotated nothing.  On
+// return sM holds M Z (columns in place).
+template <int MP, int LM>
+SEED_DEV int jacobi_regs(float* sM, bool& conv) {
+  constexpr int LP = 64 / MP;   // lanes per pair
+  constexpr int NR = MP / LP;   // rows per lane
+  constexpr int NS = MP / 2;    // pair slots
+  static_assert(NR % 4 == 0, "rows per lane must be whole float4s");
+  const int lane = threadIdx.x & 31;
+  const int slot = lane / LP, h = lane % LP;
+  int ix = slot, iy = slot + NS;
+  float x[NR], y[NR];
+#pragma unroll
+  for (int f = 0; f < NR / 4; ++f) {
+    const float4 a = ld4(sM + ix * LM + h * NR + 4 * f);
+    const float4 b = ld4(sM + iy * LM + h * NR + 4 * f);
+    x[4 * f] = a.x; x[4 * f + 1] = a.y; x[4 * f + 2] = a.z; x[4 * f + 3] = a.w;
+    y[4 * f] = b.x; y[4 * f + 1] = b.y; y[4 * f + 2] = b.z; y[4 * f + 3] = b.w;
+  }
+  const float tol = 8.f * sqrtf((float)MP) * 5.9604645e-8f;
+  const float tol2 = tol * tol;
+  float tiny = 0.f;
+  int sweeps = 0;
+  conv = false;
+  for (int sweep = 0; sweep < kJacobiMaxSweeps; ++sweep) {
+    // exact squared norms (the scales are 1 at the start of every sweep)
+    float nx = 0.f, ny = 0.f;
+#pragma unroll
+    for (int i = 0; i < NR; ++i) {
+      nx = fmaf(x[i], x[i], nx);
+      ny = fmaf(y[i], y[i], ny);
+    }
+    nx = pair_sum<LP>(nx);
+    ny = pair_sum<LP>(ny);
+    if (sweep == 0) tiny = 1e-10f * group_sum<32>(nx + ny) * (1.f / LP);
+    // true column = s * stored column; r = 1 / s
+    float sx = 1.f, sy = 1.f, rx = 1.f, ry = 1.f;
+    bool rot = false;
+#pragma unroll 1
+    for (int G = NS; G >= 1; G >>= 1) {
+#pragma unroll 1
+      for (int r = 0; r < G; ++r) {
+        float g0 = 0.f, g1 = 0.f, g2 = 0.f, g3 = 0.f;
+#pragma unroll
+        for (int i = 0; i < NR; i += 4) {
+          g0 = fmaf(x[i], y[i], g0);
+          g1 = fmaf(x[i + 1], y[i + 1], g1);
+          g2 = fmaf(x[i + 2], y[i + 2], g2);
+          g3 = fmaf(x[i + 3], y[i + 3], g3);
+        }
+        const float g = pair_sum<LP>((g0 + g1) + (g2 + g3)) * (sx * sy);
+        if (nx > tiny && ny > tiny && g * g > tol2 * (nx * ny)) {
+          // Rutishauser's rotation, t = sign(d) 2g / (|d| + sqrt(d^2 + 4 g^2)) with
+          // d = |y|^2 - |x|^2 (the smaller root of t^2 + (d / g) t - 1 = 0); the
+          // fast reciprocal only perturbs t, c = 1 / sqrt(1 + t^2) keeps it orthogonal
+          const float d = ny - nx;
+          const float e = fmaf(d, d, 4.f * g * g);
+          const float t0 = __fdividef(2.f * g, fabsf(d) + e * rsqrtf(e));
+          const float t = d >= 0.f ? t0 : -t0;
+          const float u = fmaf(t, t, 1.f);
+          const float c = rsqrtf(u);
+          const float ic = u * c;
+          // x' = c (x - t y), y' = c (y + t x) on the true columns; on the stored
+          // ones xs' = xs - t (sy / sx) ys, ys' = ys + t (sx / sy) xs, s' = c s
+          const float tx = t * sy * rx, ty = t * sx * ry;
+#pragma unroll
+          for (int i = 0; i < NR; ++i) {
+            const float xo = x[i];
+            x[i] = fmaf(-tx, y[i], xo);
+            y[i] = fmaf(ty, xo, y[i]);
+          }
+          sx *= c;
+          sy *= c;
+          rx *= ic;
+          ry *= ic;
+          nx = fmaf(-t, g, nx);
+          ny = fmaf(t, g, ny);
+          rot = true;
+        }
+        if (r + 1 < G) {   // shift the first columns one slot along the group
+          const int gb = slot & ~(G - 1);
+          const int src = (gb + ((slot - gb - 1) & (G - 1))) * LP + h;
+#pragma unroll
+          for (int i = 0; i < NR; ++i) x[i] = __shfl_sync(kFull, x[i], src);
+          ix = __shfl_sync(kFull, ix, src);
+          nx = __shfl_sync(kFull, nx, src);
+          sx = __shfl_sync(kFull, sx, src);
+          rx = __shfl_sync(kFull, rx, src);
+        }
+      }
+      if (G > 1) {   // halve the groups: first halves pair their x's, second halves their y's
+        const int half = G >> 1;
+        const bool first = (slot & half) == 0;
+        const int pl = lane ^ (half * LP);
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+          const float got = __shfl_sync(kFull, first ? y[i] : x[i], pl);
+          if (first) y[i] = got;
+          else x[i] = got;
+        }
+        const int gi = __shfl_sync(kFull, first ? iy : ix, pl);
+        const float gn = __shfl_sync(kFull, first ? ny : nx, pl);
+        const float gs = __shfl_sync(kFull, first ? sy : sx, pl);
+        const float gr = __shfl_sync(kFull, first ? ry : rx, pl);
+        if (first) { iy = gi; ny = gn; sy = gs; ry = gr; }
+        else { ix = gi; nx = gn; sx = gs; rx = gr; }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < NR; ++i) {
+      x[i] *= sx;
+      y[i] *= sy;
+    }
+    sweeps = sweep + 1;
+    if (!__any_sync(kFull, rot)) {
+      conv = true;
+      break;
+    }
+  }
+  __syncwarp();
+#pragma unroll
+  for (int f = 0; f < NR / 4; ++f) {
+    st4(sM + ix * LM + h * NR + 4 * f, make_float4(x[4 * f], x[4 * f + 1], x[4 * f + 2], x[4 * f + 3]));
+    st4(sM + iy * LM + h * NR + 4 * f, make_float4(y[4 * f], y[4 * f + 1], y[4 * f + 2], y[4 * f + 3]));
+  }
+  __syncwarp();
+  return sweeps;
+}
+
+// Chunk c of the panel stream (rows 32c .. 32c+31 of U, then of V) into buffer
+// c & 1: one tensor copy of the box {32 rows, MP columns, 1 unit}, completing on
+// bar[c & 1].  Columns m .. MP-1 lie outside the tensor and arrive as zeros.  In
+// shared memory column j is a 128-byte row whose 16-byte pieces are permuted by
+// the 128-byte swizzle: piece f sits at f ^ (j & 7).
+template <int NCU, int CHUNK>
+SEED_DEV void issue_chunk(int c, float* sA, const CUtensorMap* tmU, const CUtensorMap* tmV, long long unit,
+                          uint64_t* bar) {
+  const int bb = c & 1;
+  const bool isU = c < NCU;
+  const int r0 = 32 * (isU ? c : c - NCU);
+  if ((threadIdx.x & 31) == 0) {
+    mbar_arrive_expect_tx(&bar[bb], (uint32_t)(CHUNK * 4));
+    tma_load_3d(sA + bb * CHUNK, isU ? tmU : tmV, r0, 0, (int)unit, &bar[bb]);
+  }
+}
+
+// Offset (in floats) of element e of column j in a swizzled chunk buffer.
+SEED_DEV int swz(int j, int e) { return j * 32 + ((((e >> 2) ^ (j & 7)) << 2) | (e & 3)); }
+
+// Gram row `lane` of one panel, accumulated over its chunks c0 .. c1-1 as they
+// arrive (issuing chunk c + 2 into a buffer once chunk c is read); also checks the
+// column scale.  FOLD (KDA's U): the products are weighted by P^2 (true U = Diag(P) U).
+// Returns false if a copy did not arrive in time (after waiting for those in flight).
+template <bool FOLD, int NCU, int NCH, int MP, int CHUNK>
+SEED_DEV bool gram_stream(int c0, int c1, float* sA, const CUtensorMap* tmU, const CUtensorMap* tmV,
+                          long long unit, int m, uint64_t* bar, const float* scl, float (&g)[MP], bool& bad) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < MP; ++i) g[i] = 0.f;
+  float mx = 0.f;
+  const int jo = lane < MP ? lane : 0;
+#pragma unroll 1
+  for (int c = c0; c < c1; ++c) {
+    const int bb = c & 1;
+    const uint32_t ph = (uint32_t)(c >> 1) & 1u;
+    if (!__all_sync(kFull, mbar_wait_bounded(&bar[bb], ph, kWaitLimitNs))) {
+      mbar_wait_bounded(&bar[bb], ph, kWaitLimitNs);
+      if (c + 1 < NCH) mbar_wait_bounded(&bar[bb ^ 1], (uint32_t)((c + 1) >> 1) & 1u, kWaitLimitNs);
+      return false;
+    }
+    const float* buf = sA + bb * CHUNK;
+    const int r0 = 32 * (c < NCU ? c : c - NCU);
+#pragma unroll 2
+    for (int f = 0; f < 8; ++f) {
+      float4 o = ld4(buf + jo * 32 + ((f ^ (jo & 7)) << 2));
+      float4 pw = make_float4(1.f, 1.f, 1.f, 1.f);
+      if constexpr (FOLD) {
+        pw = ld4(scl + r0 + 4 * f);
+        o = mul4(o, pw);
+      }
+      mx = fmaxf(mx, fmaxf(fmaxf(fabsf(o.x), fabsf(o.y)), fmaxf(fabsf(o.z), fabsf(o.w))));
+      if constexpr (FOLD) o = mul4(o, pw);
+#pragma unroll
+      for (int i = 0; i < MP; ++i) g[i] += dot4(ld4(buf + i * 32 + ((f ^ (i & 7)) << 2)), o);
+    }
+    __syncwarp();   // every lane has read this chunk before the next copy overwrites it
+    if (c + 2 < NCH) issue_chunk<NCU, CHUNK>(c + 2, sA, tmU, tmV, unit, bar);
+  }
+  if (lane < m && mx > 0.f && (mx < kColMin || mx > kColMax)) bad = true;
+  return true;
+}
+
+// Shared memory.  Region A first holds two 32-row chunk buffers through which the
+// panels stream (U chunks, then V chunks); after the V Gram it holds L_v, then M
+// in place of it, the selected left vectors X and Gram-Schmidt scratch, and at the
+// end the chunks of the panels again.  L_u has its own region, used from the U Gram
+// until the small right factors T_u and T_v replace it.
 template <int FORM, int DK, int DV, int MP>
 struct FastLayout {
-  static constexpr int LDK = DK + 4, LDV = DV + 4, LG = MP + 1, LM = MP + 4;
+  static constexpr int CHUNK = MP * 32;                         // one swizzled chunk (MP x 128 B)
+  static constexpr int LG = MP + 4, LX = MP + 1;
   static constexpr int SL = (FORM == SEED_KDA ? DK : MP);
-  static constexpr int A = MP * LDK + MP * LDV;                 // panels
-  static constexpr int B = 2 * MP * LG + MP * LM + MP * MP;     // L_u, L_v / X, M / T_u, T_v
-  static_assert(B <= A, "aliased buffers must fit in the panel region");
-  static constexpr int SMALL = 6 * MP + SL;                     // nu nv nrm sig csu csv scl
-  static constexpr size_t bytes = (A + SMALL) * sizeof(float) + (MP + 4) * sizeof(int);
+  static constexpr int OFF_M = 0, OFF_X = MP * LG, OFF_P = OFF_X + kFastMaxR * LX;
+  static constexpr int A_CH = 2 * CHUNK, A_B = OFF_P + kFastMaxR * LX;
+  static constexpr int A = ((A_CH > A_B ? A_CH : A_B) + 255) & ~255;   // keeps L_u 1 KB aligned
+  static constexpr int LU = A;                                  // L_u (MP x LG), then T_u | T_v
+  static constexpr int LU_N = (MP * LG > 2 * MP * kFastMaxR ? MP * LG : 2 * MP * kFastMaxR);
+  static constexpr int SMALL = LU + LU_N;                       // nu nv du dv nrm, scl
+  static constexpr int FLOATS = SMALL + 5 * MP + SL;
+  // + 1 KB: the dynamic shared memory is re-aligned to the 1 KB the swizzle needs
+  static constexpr size_t bytes = FLOATS * sizeof(float) + (MP + 4) * sizeof(int) + 1024;
 };
 
 template <int FORM, int DK, int DV, int MP>
-__global__ void __launch_bounds__(64) compress_fast_kernel(const FastParams p) {
+__global__ void __launch_bounds__(32)
+    compress_fast_kernel(const FastParams p, const __grid_constant__ CUtensorMap tmU,
+                         const __grid_constant__ CUtensorMap tmV) {
   using Lay = FastLayout<FORM, DK, DV, MP>;
   constexpr bool KDA = FORM == SEED_KDA;
-  constexpr int LDK = Lay::LDK, LDV = Lay::LDV, LG = Lay::LG, LM = Lay::LM;
-  constexpr int PK = DK / 32, PV = DV / 32;
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  float* sU = reinterpret_cast<float*>(smem_raw);   // region A
-  float* sV = sU + MP * LDK;
-  float* sGu = sU;                                   // region B, after the Grams
-  float* sGv = sGu + MP * LG;                        // L_v, then the selected vectors X
-  float* sM = sGv + MP * LG;                         // the core, then T_u
-  float* sTv = sM + MP * LM;                         // Gram-Schmidt scratch, then T_v
-  float* nu = sU + Lay::A;                           // small arrays
+  constexpr int LG = Lay::LG, LX = Lay::LX, CHUNK = Lay::CHUNK;
+  constexpr int NCU = DK / 32, NCV = DV / 32, NCH = NCU + NCV;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  float* sA = reinterpret_cast<float*>(smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023));
+  float* sM = sA + Lay::OFF_M;       // L_v, then M (column-major), then T_u | T_v
+  float* sX = sA + Lay::OFF_X;       // R x LX
+  float* sP = sA + Lay::OFF_P;       // R x LX scratch
+  float* sLu = sA + Lay::LU;
+  float* nu = sA + Lay::SMALL;
   float* nv = nu + MP;
-  float* nrm = nv + MP;
-  float* sig = nrm + MP;
-  float* csu = sig + MP;
-  float* csv = csu + MP;
-  float* scl = csv + MP;
+  float* du = nv + MP;
+  float* dvv = du + MP;
+  float* nrm = dvv + MP;
+  float* scl = nrm + MP;
   int* sel = reinterpret_cast<int*>(scl + Lay::SL);
-  int* flags = sel + MP;   // [0] ill-conditioned, [1] rotated this sweep
-  __shared__ __align__(8) uint64_t bar;
+  __shared__ __align__(8) uint64_t bar[2];
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int lane = threadIdx.x;
   const int m = p.R + p.W;
   const int per = p.layer < 0 ? p.L * p.H : p.H;
   const int idx = blockIdx.x;
@@ -166,366 +396,326 @@ __global__ void __launch_bounds__(64) compress_fast_kernel(const FastParams p) {
   const long long unit =
       p.layer < 0 ? (long long)idx : ((long long)b * p.L + p.layer) * p.H + rest;
   if (p.ncols[unit] != m) return;   // not due (the fallback kernel flags invalid counts)
-  const float* Ug = p.U + unit * (long long)m * DK;
-  const float* Vg = p.V + unit * (long long)m * DV;
 
-  // 1. panels -> shared memory
-  if (tid == 0) {
-    mbar_init(&bar, 1);
+  // 1. the panels stream through two chunk buffers, 32 rows of every column per
+  //    chunk (one tensor copy each); Gram rows accumulate in registers
+  if (lane == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
     fence_mbar_init();
-    mbar_arrive_expect_tx(&bar, (uint32_t)(m * (DK + DV) * 4));
-    flags[0] = 0;
   }
-  __syncthreads();
-  if (warp == 0 && lane < m) {
-    bulk_g2s(sU + lane * LDK, Ug + (long long)lane * DK, DK * 4, &bar);
-    bulk_g2s(sV + lane * LDV, Vg + (long long)lane * DV, DV * 4, &bar);
-  }
-  for (int e = m * LDK + tid; e < MP * LDK; e += 64) sU[e] = 0.f;
-  for (int e = m * LDV + tid; e < MP * LDV; e += 64) sV[e] = 0.f;
-  for (int e = tid; e < p.slen; e += 64) scl[e] = p.scale[unit * p.slen + e];
-  if (!__syncthreads_and(mbar_wait_bounded(&bar, 0, kWaitLimitNs))) {
-    if (tid == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
-    mbar_wait_bounded(&bar, 0, kWaitLimitNs);
+  for (int e = lane; e < p.slen; e += 32) scl[e] = p.scale[unit * p.slen + e];
+  __syncwarp();
+  issue_chunk<NCU, CHUNK>(0, sA, &tmU, &tmV, unit, bar);
+  issue_chunk<NCU, CHUNK>(1, sA, &tmU, &tmV, unit, bar);
+  bool bad = false;   // ill-conditioned or badly scaled: left for the Householder kernel
+  float g[MP];
+  // U: chunks 0 .. NCU-1, then its Cholesky factor
+  if (!gram_stream<KDA, NCU, NCH, MP, CHUNK>(0, NCU, sA, &tmU, &tmV, unit, m, bar, scl, g, bad)) {
+    if (lane == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
     return;
   }
-  if constexpr (KDA) {   // true U = Diag(P) U
-    for (int e = tid; e < m * DK; e += 64) {
-      const int j = e / DK, r = e - j * DK;
-      sU[j * LDK + r] *= scl[r];
-    }
-    __syncthreads();
-  }
-
-  // column scaling by the largest magnitude (warp 0: U, warp 1: V) so that no
-  // Gram entry is formed from values near the float32 underflow
   {
-    float* Pn = warp == 0 ? sU : sV;
-    const int LD = warp == 0 ? LDK : LDV;
-    const int D = warp == 0 ? DK : DV;
-    float mx = 0.f;
-    if (lane < m) {
-      for (int r = 0; r < D; r += 4) {
-        const float4 x = ld4(Pn + lane * LD + r);
-        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(x.z), fabsf(x.w))));
-      }
-      const float inv = mx > 0.f ? 1.f / mx : 0.f;
-      for (int r = 0; r < D; r += 4) {
-        float4 x = ld4(Pn + lane * LD + r);
-        x.x *= inv; x.y *= inv; x.z *= inv; x.w *= inv;
-        st4(Pn + lane * LD + r, x);
-      }
-    }
-    if (lane < MP) (warp == 0 ? csu : csv)[lane] = mx;
-  }
-  __syncthreads();
-
-  // 2. equilibrated Grams and their Cholesky factors, in registers (warp 0: U,
-  //    warp 1: V); L then stored row-major (ld MP+1) over the panel region
-  {
-    float g[MP];
-    if (warp == 0) gram_row<MP, DK, LDK>(sU, g);
-    else gram_row<MP, DV, LDV>(sV, g);
     const float n = equilibrate_row<MP>(g);
-    if (lane < MP) (warp == 0 ? nu : nv)[lane] = n;
-    cholesky_regs<MP>(g, n, flags);
-    __syncthreads();   // both Grams are read before L overwrites the panels
-    float* G = warp == 0 ? sGu : sGv;
+    if (lane < MP) nu[lane] = n;
+    cholesky_regs<MP>(g, n, bad);
     if (lane < MP) {
 #pragma unroll
-      for (int k = 0; k < MP; ++k) G[lane * LG + k] = g[k];
+      for (int k = 0; k < MP; k += 4) st4(sLu + lane * LG + k, make_float4(g[k], g[k + 1], g[k + 2], g[k + 3]));
     }
   }
-  __syncthreads();
-  if (flags[0]) {   // ill-conditioned: left for the Householder kernel
-    if (tid == 0) atomicAdd(p.status + 6, 1u);
+  // V: chunks NCU .. NCH-1
+  if (!gram_stream<false, NCU, NCH, MP, CHUNK>(NCU, NCH, sA, &tmU, &tmV, unit, m, bar, scl, g, bad)) {
+    if (lane == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
     return;
   }
-
-  // D_u, D_v: true column norms (panel scale times the scaled-column norm, and for
-  // GDN / Mamba-2 the lazy scale gamma_j)
-  if (tid < MP) {
-    const float gj = (KDA || tid >= m) ? 1.f : scl[tid];
-    nrm[tid] = nu[tid] * csu[tid] * gj;   // D_u
-    csv[tid] = nv[tid] * csv[tid];        // D_v
+  {
+    const float n = equilibrate_row<MP>(g);
+    if (lane < MP) nv[lane] = n;
+    cholesky_regs<MP>(g, n, bad);
   }
-  __syncthreads();
-
-  // 3. core M = L_u^T diag(D_u D_v) L_v, column-major (ld LM)
-  for (int e = tid; e < MP * MP; e += 64) {
-    const int j = e / MP, i = e - j * MP;
-    float acc = 0.f;
-    for (int k = max(i, j); k < MP; ++k)
-      acc = fmaf(sGu[k * LG + i] * (nrm[k] * csv[k]), sGv[k * LG + j], acc);
-    sM[j * LM + i] = acc;
+  if (__any_sync(kFull, bad)) {
+    if (lane == 0) atomicAdd(p.status + 6, 1u);
+    return;
   }
-  __syncthreads();
-  if (tid < MP) sig[tid] = nrm[tid];   // keep D_u in sig until the end
-  __syncthreads();
+  // L_v over the (now idle) chunk buffers, row-major
+  if (lane < MP) {
+#pragma unroll
+    for (int k = 0; k < MP; k += 4) st4(sM + lane * LG + k, make_float4(g[k], g[k + 1], g[k + 2], g[k + 3]));
+  }
 
-  // 4. one-sided Jacobi on M: 16 pairs per round, pair pr = warp * 8 + lane / 4,
-  //    lane quarter q holds rows 4 NF q .. of both columns
-  const int pr = warp * 8 + (lane >> 2), qt = lane & 3;
-  const float tol = 8.f * sqrtf((float)MP) * 5.9604645e-8f;
-  float tiny = 0.f;
-  int sweeps = 0;
-  bool converged = false;
-  for (int sweep = 0; sweep < 30; ++sweep) {
-    if (tid < MP) {
-      float s2 = 0.f;
+  // D_u, D_v: true column norms (GDN / Mamba-2: with the lazy scale gamma_j); the
+  // core is formed with w_k = D_u D_v / max(D_u D_v) so that its entries are of
+  // order one, and its singular values are scaled back by wmax
+  float wl = 0.f;
+  if (lane < MP) {
+    const float gj = (KDA || lane >= m) ? 1.f : scl[lane];
+    const float a = nu[lane] * gj, bv = nv[lane];
+    du[lane] = a;
+    dvv[lane] = bv;
+    wl = a * bv;
+  }
+  const float wmax = warp_max(wl);
+  const float winv = wmax > 0.f ? 1.f / wmax : 0.f;
+  __syncwarp();
+
+  // 2. core M = L_u^T diag(w) L_v in place of L_v, column j in lane j:
+  //    M[i][j] = sum_{k >= max(i, j)} L_u[k][i] w_k L_v[k][j]
+  {
+    const int j = lane < MP ? lane : 0;
+    float lv[MP];
 #pragma unroll
-      for (int r = 0; r < MP; r += 4) {
-        const float4 x = ld4(sM + tid * LM + r);
-        s2 += dot4(x, x);
-      }
-      nrm[tid] = s2;
-    }
-    if (tid == 0) flags[1] = 0;
-    pair_sync();
-    if (sweep == 0) {
-      float f2 = 0.f;
-      for (int j = 0; j < MP; ++j) f2 += nrm[j];
-      tiny = 1e-10f * f2;
-    }
-    for (int round = 0; round < MP - 1; ++round) {
-      int P, Q;
-      if (pr == 0) {
-        P = MP - 1;
-        Q = round;
-      } else {
-        P = round + pr;
-        if (P >= MP - 1) P -= MP - 1;
-        Q = round - pr;
-        if (Q < 0) Q += MP - 1;
-      }
-      constexpr int NF = MP / 16;    // float4 per lane per column
-      const bool active = (MP == 32) || pr < MP / 2;   // with MP = 32 every lane has a pair
-      float* xp = sM + P * LM + 4 * NF * qt;
-      float* yp = sM + Q * LM + 4 * NF * qt;
-      float4 xv[NF], yv[NF];
-      float g = 0.f;
+    for (int k = 0; k < MP; ++k) lv[k] = k >= j ? sM[k * LG + j] * (du[k] * dvv[k] * winv) : 0.f;
+    __syncwarp();   // every lane holds its column of L_v before M overwrites it
+    float acc[MP];
 #pragma unroll
-      for (int f = 0; f < NF; ++f) {
-        xv[f] = active ? ld4(xp + 4 * f) : zero4();
-        yv[f] = active ? ld4(yp + 4 * f) : zero4();
-        g += dot4(xv[f], yv[f]);
-      }
-      g += __shfl_xor_sync(0xffffffffu, g, 1);
-      g += __shfl_xor_sync(0xffffffffu, g, 2);
-      const float al = active ? nrm[P] : 0.f, be = active ? nrm[Q] : 0.f;
-      // rotation test and parameters with the fast intrinsics: t need not be the
-      // exact tangent, the rotation stays orthogonal because c = 1 / sqrt(1 + t^2)
-      if (active && al > tiny && be > tiny && fabsf(g) > tol * sqrtf(al) * sqrtf(be)) {
-        const float zeta = __fdividef(be - al, 2.f * g);
-        float t;
-        if (fabsf(zeta) > 1e18f) t = __fdividef(0.5f, zeta);
-        else {
-          const float z1 = fmaf(zeta, zeta, 1.f);
-          t = copysignf(__fdividef(1.f, fabsf(zeta) + z1 * rsqrtf(z1)), zeta);
-        }
-        const float cs = rsqrtf(fmaf(t, t, 1.f));
-        const float sn = cs * t;
+    for (int i = 0; i < MP; ++i) acc[i] = 0.f;
 #pragma unroll
-        for (int f = 0; f < NF; ++f) {
-          const float4 x = xv[f], y = yv[f];
-          float4 a, bb;
-          a.x = cs * x.x - sn * y.x; bb.x = fmaf(sn, x.x, cs * y.x);
-          a.y = cs * x.y - sn * y.y; bb.y = fmaf(sn, x.y, cs * y.y);
-          a.z = cs * x.z - sn * y.z; bb.z = fmaf(sn, x.z, cs * y.z);
-          a.w = cs * x.w - sn * y.w; bb.w = fmaf(sn, x.w, cs * y.w);
-          st4(xp + 4 * f, a);
-          st4(yp + 4 * f, bb);
-        }
-        if (qt == 0) {
-          nrm[P] = al - t * g;
-          nrm[Q] = be + t * g;
-          flags[1] = 1;
-        }
+    for (int k = 0; k < MP; ++k) {
+      const float cf = lv[k];
+#pragma unroll
+      for (int i4 = 0; i4 <= k; i4 += 4) {
+        const float4 l = ld4(sLu + k * LG + i4);
+        acc[i4] = fmaf(cf, l.x, acc[i4]);
+        if (i4 + 1 <= k) acc[i4 + 1] = fmaf(cf, l.y, acc[i4 + 1]);
+        if (i4 + 2 <= k) acc[i4 + 2] = fmaf(cf, l.z, acc[i4 + 2]);
+        if (i4 + 3 <= k) acc[i4 + 3] = fmaf(cf, l.w, acc[i4 + 3]);
       }
-      pair_sync();
     }
-    sweeps = sweep + 1;
-    const int any = flags[1];
-    pair_sync();
-    if (!any) {
-      converged = true;
-      break;
+    if (lane < MP) {
+#pragma unroll
+      for (int i = 0; i < MP; i += 4) st4(sM + lane * LG + i, make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]));
     }
   }
-  if (tid == 0) {
+  __syncwarp();
+
+  // 3. one-sided Jacobi on M
+  bool converged;
+  const int sweeps = jacobi_regs<MP, LG>(sM, converged);
+  if (lane == 0) {
     atomicAdd(p.status + 1, (uint32_t)sweeps);
     atomicAdd(p.status + 5, 1u);
     if (!converged) raise_flag(p.status, SEED_FLAG_NOCONVERGE);
   }
 
-  // 5. singular values = column norms of M Z; the R largest
-  if (tid < MP) {
+  // 4. singular values (of the scaled core) = column norms of M Z; the R largest
+  if (lane < MP) {
     float s2 = 0.f;
 #pragma unroll
     for (int r = 0; r < MP; r += 4) {
-      const float4 x = ld4(sM + tid * LM + r);
+      const float4 x = ld4(sM + lane * LG + r);
       s2 += dot4(x, x);
     }
-    nrm[tid] = sqrtf(s2);
+    nrm[lane] = sqrtf(s2);
   }
-  __syncthreads();
-  if (tid < MP) {
-    const float s = nrm[tid];
+  __syncwarp();
+  if (lane < MP) {
+    const float s = nrm[lane];
     int rank = 0;
     for (int k = 0; k < MP; ++k) {
       const float t = nrm[k];
-      rank += (t > s) || (t == s && k < tid);
+      rank += (t > s) || (t == s && k < lane);
     }
-    if (rank < p.R) sel[rank] = tid;
+    if (rank < p.R) sel[rank] = lane;
   }
-  __syncthreads();
-  float smax = 0.f;
-  for (int j = 0; j < MP; ++j) smax = fmaxf(smax, nrm[j]);
+  __syncwarp();
+  const float smax = warp_max(lane < MP ? nrm[lane] : 0.f);
   const float szero = (float)(DK > DV ? DK : DV) * 1.1920929e-7f * smax;
 
-  // 5b. orthonormalise the selected left vectors x_r = (M Z)_{sel r} / sigma_r in
-  //     descending order (classical Gram-Schmidt, two passes; warp 0, lane = row).
-  //     The Jacobi leaves columns it judged negligible unrotated, so the raw x_r
-  //     need not be orthogonal; with orthonormal x_r the result below is exactly
-  //     the projection of U V^T on their span.  A vector that loses more than half
-  //     its norm to the earlier ones adds no new direction and is dropped.
-  float* sX = sGv;   // R x MP (L_v is no longer needed)
-  float* sP = sTv;   // scratch, R x (MP+1)
-  float* sgk = csu;  // sigma kept for each output column (0: dropped)
-  if (warp == 0) {
+  // 4b. the selected left vectors x_r = (M Z)_{sel r} / sigma_r, stored [r][i].
+  //     Columns whose squared norm the Jacobi judged negligible (below 1e-10 of
+  //     the total) are left unrotated, so they need not be orthogonal to the
+  //     others; when every selected sigma is above 1e-4 sigma_max none of them is
+  //     such a column and the x_r are orthonormal as they are.  Otherwise they are
+  //     orthonormalised in descending order (classical Gram-Schmidt, two passes;
+  //     lane = row), so that the result below is exactly the projection of U V^T on
+  //     their span; a vector that loses more than half its norm to the earlier ones
+  //     adds no new direction and is dropped.
+  float sk = 0.f;   // lane r < R: the scaled sigma kept for output column r (0: dropped)
+  if (nrm[sel[p.R - 1]] > 1e-4f * smax) {
     for (int r = 0; r < p.R; ++r) {
       const int j = sel[r];
       const float sj = nrm[j];
-      float x = (lane < MP && sj > szero) ? sM[j * LM + lane] / sj : 0.f;
+      if (lane < MP) sX[r * LX + lane] = sM[j * LG + lane] / sj;
+      if (lane == r) sk = sj;
+    }
+    __syncwarp();
+  } else {
+    for (int r = 0; r < p.R; ++r) {
+      const int j = sel[r];
+      const float sj = nrm[j];
+      float x = (lane < MP && sj > szero) ? sM[j * LG + lane] / sj : 0.f;
       for (int pass = 0; pass < 2; ++pass) {
         for (int k = 0; k < r; ++k)
-          if (lane < MP) sP[k * (MP + 1) + lane] = x * sX[k * MP + lane];
+          if (lane < MP) sP[k * LX + lane] = x * sX[k * LX + lane];
         __syncwarp();
         float dk = 0.f;
         if (lane < r)
-          for (int i = 0; i < MP; ++i) dk += sP[lane * (MP + 1) + i];
+          for (int i = 0; i < MP; ++i) dk += sP[lane * LX + i];
         __syncwarp();
         for (int k = 0; k < r; ++k) {
-          const float d = __shfl_sync(0xffffffffu, dk, k);
-          if (lane < MP) x = fmaf(-d, sX[k * MP + lane], x);
+          const float d = __shfl_sync(kFull, dk, k);
+          if (lane < MP) x = fmaf(-d, sX[k * LX + lane], x);
         }
       }
       const float nx = sqrtf(group_sum<32>(x * x));
       const bool keep = nx > 0.5f;
       x = keep ? x / nx : 0.f;
-      if (lane < MP) sX[r * MP + lane] = x;
-      if (lane == 0) sgk[r] = keep ? sj : 0.f;
+      if (lane < MP) sX[r * LX + lane] = x;
+      if (lane == r) sk = keep ? sj : 0.f;
       __syncwarp();
     }
   }
-  __syncthreads();
 
-  // 6. small right factors on the raw panels (column r in lane r, stored [k][r]):
-  //    U' = U_raw T_u with T_u = diag(gamma / D_u) L_u^{-T} X_R Sigma^{1/2}
-  //         (KDA: the row decay P is applied to the product instead of gamma)
-  //    V' = V_raw T_v with T_v = D_u L_u X_R Sigma^{-1/2}
-  float* sTu = sM;
-  if (lane < p.R) {
-    const int r = lane;
-    const float s = sgk[r];
-    const bool zero = !(s > 0.f);
-    if (warp == 0) {
+  // 5. small right factors on the stored panels (column r in registers of lane r
+  //    for T_u, of lane 16 + r for T_v).  With sigma = wmax * sk the true value:
+  //      GDN / Mamba-2 (a per-column scale exists): unit columns, the scale = sigma
+  //        U' = U_st T_u, T_u = diag(1 / nu) L_u^{-T} X_R
+  //        V' = V_st T_v, T_v = D_u L_u X_R Sigma^{-1}
+  //      KDA: balanced, Sigma^{1/2} on each side (the row products P applied to U'
+  //        after the product, and reset to 1)
+  //    then stored [k][r] (stride 16) over L_u: T_u first, T_v after it (T_v goes
+  //    through the Gram-Schmidt scratch while the other half still reads L_u)
+  {
+    const int r = lane & 15;
+    const float s = __shfl_sync(kFull, sk, r) * wmax;
+    const bool zero = !(s > 0.f) || r >= p.R;
+    float t[MP];
+    if (lane < 16) {
       // back substitution with L_u^T (upper): t_k = (x_k - sum_{i>k} L_u[i][k] t_i) / L_u[k][k]
-      const float f = zero ? 0.f : sqrtf(s);
+      const float f = zero ? 0.f : (KDA ? sqrtf(s) : 1.f);
+#pragma unroll
       for (int k = MP - 1; k >= 0; --k) {
-        float acc = sX[r * MP + k] * f;
-        for (int i = k + 1; i < MP; ++i) acc = fmaf(-sGu[i * LG + k], sTu[i * MP + r], acc);
-        const float lkk = sGu[k * LG + k];
-        sTu[k * MP + r] = lkk != 0.f ? acc / lkk : 0.f;
+        float acc = zero ? 0.f : sX[r * LX + k] * f;
+#pragma unroll
+        for (int i = k + 1; i < MP; ++i) acc = fmaf(-sLu[i * LG + k], t[i], acc);
+        const float lkk = sLu[k * LG + k];
+        t[k] = lkk != 0.f ? acc / lkk : 0.f;
       }
+#pragma unroll
       for (int k = 0; k < MP; ++k) {
-        const float du = sig[k];
-        const float gk = (KDA || k >= m) ? 1.f : scl[k];
-        sTu[k * MP + r] = du > 0.f ? sTu[k * MP + r] * (gk / du) : 0.f;
+        const float n = nu[k];
+        t[k] = n > 0.f ? t[k] / n : 0.f;
       }
     } else {
-      const float f = zero ? 0.f : rsqrtf(s);
+      const float f = zero ? 0.f : (KDA ? rsqrtf(s) : 1.f / s);
+      float x[MP];
+#pragma unroll
+      for (int i = 0; i < MP; ++i) x[i] = zero ? 0.f : sX[r * LX + i];
+#pragma unroll
       for (int k = 0; k < MP; ++k) {
         float acc = 0.f;
-        for (int i = 0; i <= k; ++i) acc = fmaf(sGu[k * LG + i], sX[r * MP + i], acc);
-        sTv[k * MP + r] = sig[k] * acc * f;   // sig holds D_u
+#pragma unroll
+        for (int i4 = 0; i4 <= k; i4 += 4) {
+          const float4 l = ld4(sLu + k * LG + i4);
+          acc = fmaf(l.x, x[i4], acc);
+          if (i4 + 1 <= k) acc = fmaf(l.y, x[i4 + 1], acc);
+          if (i4 + 2 <= k) acc = fmaf(l.z, x[i4 + 2], acc);
+          if (i4 + 3 <= k) acc = fmaf(l.w, x[i4 + 3], acc);
+        }
+        sP[k * kFastMaxR + r] = du[k] * acc * f;
       }
     }
+    __syncwarp();   // every lane has read L_u and X
+    if (lane < 16) {
+#pragma unroll
+      for (int k = 0; k < MP; ++k) sLu[k * kFastMaxR + r] = t[k];
+    }
+    for (int e = lane; e < MP * kFastMaxR; e += 32) sLu[MP * kFastMaxR + e] = sP[e];
+    __syncwarp();
   }
-  __syncthreads();
+  const float* sTu = sLu;
+  const float* sTv = sLu + MP * kFastMaxR;
 
-  // 7. U' = U_raw T_u (warp 0), V' = V_raw T_v (warp 1), the panels streamed again
-  //    from global memory (read a moment ago, normally still in L2); written to
-  //    slots 0..R-1 after the block has read every stored column
-  constexpr int CH = 16;
-  float accU[CH][PK], accV[CH][PV];
-  bool bad = false;
-  for (int r0 = 0; r0 < p.R; r0 += CH) {
-    if (warp == 0) {
+  // 6. U' = U_st T_u, then V' = V_st T_v: the panels stream through the chunk
+  //    buffers again (read a moment ago, normally still in L2); lane = row of the
+  //    chunk.  A chunk's rows are written after they were read and no other chunk
+  //    holds them, so slots 0..R-1 can be overwritten in place.
+  fence_proxy_async_smem();   // the chunk buffers were written with ordinary stores
+  __syncwarp();
+  issue_chunk<NCU, CHUNK>(0, sA, &tmU, &tmV, unit, bar);
+  issue_chunk<NCU, CHUNK>(1, sA, &tmU, &tmV, unit, bar);
+  bool nonfinite = false;
+  float* Uo = p.U + unit * (long long)m * DK;
+  float* Vo = p.V + unit * (long long)m * DV;
+#pragma unroll 1
+  for (int c = 0; c < NCH; ++c) {
+    const int bb = c & 1;
+    const uint32_t ph = (uint32_t)(NCH / 2 + (c >> 1)) & 1u;
+    if (!__all_sync(kFull, mbar_wait_bounded(&bar[bb], ph, kWaitLimitNs))) {
+      if (lane == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
+      mbar_wait_bounded(&bar[bb], ph, kWaitLimitNs);
+      if (c + 1 < NCH) mbar_wait_bounded(&bar[bb ^ 1], (uint32_t)(NCH / 2 + ((c + 1) >> 1)) & 1u, kWaitLimitNs);
+      return;   // the unit keeps R + W columns; the slots written so far hold partial results
+    }
+    const bool isU = c < NCU;
+    const int r0 = 32 * (isU ? c : c - NCU);
+    const float* buf = sA + bb * CHUNK;
+    const float* T = isU ? sTu : sTv;
+    float acc[kFastMaxR];
 #pragma unroll
-      for (int q = 0; q < CH; ++q)
+    for (int q = 0; q < kFastMaxR; ++q) acc[q] = 0.f;
+#pragma unroll 4
+    for (int k = 0; k < m; ++k) {
+      const float xv = buf[swz(k, lane)];
 #pragma unroll
-        for (int e = 0; e < PK; ++e) accU[q][e] = 0.f;
-      for (int k = 0; k < m; ++k) {
-        const auto u = VecT<PK>::load(Ug + (long long)k * DK + PK * lane);
-#pragma unroll
-        for (int q = 0; q < CH; ++q) {
-          const float tk = (r0 + q < p.R) ? sTu[k * MP + r0 + q] : 0.f;
-#pragma unroll
-          for (int e = 0; e < PK; ++e) accU[q][e] = fmaf(VecT<PK>::get(u, e), tk, accU[q][e]);
-        }
-      }
-      if constexpr (KDA) {
-#pragma unroll
-        for (int e = 0; e < PK; ++e) {
-          const float pe = scl[PK * lane + e];
-#pragma unroll
-          for (int q = 0; q < CH; ++q) accU[q][e] *= pe;
-        }
-      }
-    } else {
-#pragma unroll
-      for (int q = 0; q < CH; ++q)
-#pragma unroll
-        for (int e = 0; e < PV; ++e) accV[q][e] = 0.f;
-      for (int k = 0; k < m; ++k) {
-        const auto v = VecT<PV>::load(Vg + (long long)k * DV + PV * lane);
-#pragma unroll
-        for (int q = 0; q < CH; ++q) {
-          const float tk = (r0 + q < p.R) ? sTv[k * MP + r0 + q] : 0.f;
-#pragma unroll
-          for (int e = 0; e < PV; ++e) accV[q][e] = fmaf(VecT<PV>::get(v, e), tk, accV[q][e]);
-        }
+      for (int q = 0; q < kFastMaxR; q += 4) {
+        const float4 tk = ld4(T + k * kFastMaxR + q);
+        acc[q] = fmaf(xv, tk.x, acc[q]);
+        acc[q + 1] = fmaf(xv, tk.y, acc[q + 1]);
+        acc[q + 2] = fmaf(xv, tk.z, acc[q + 2]);
+        acc[q + 3] = fmaf(xv, tk.w, acc[q + 3]);
       }
     }
-    __syncthreads();   // every stored column of this chunk's range is read
-    float* Uo = p.U + unit * (long long)m * DK;
-    float* Vo = p.V + unit * (long long)m * DV;
+    __syncwarp();   // every lane has read this chunk before the next copy overwrites it
+    if (c + 2 < NCH) issue_chunk<NCU, CHUNK>(c + 2, sA, &tmU, &tmV, unit, bar);
+    const float rowf = (KDA && isU) ? scl[r0 + lane] : 1.f;
+    float* out = (isU ? Uo : Vo) + r0 + lane;
+    const int ld = isU ? DK : DV;
 #pragma unroll
-    for (int q = 0; q < CH; ++q) {
-      if (r0 + q < p.R) {
-        if (warp == 0) {
-#pragma unroll
-          for (int e = 0; e < PK; ++e) {
-            bad |= !isfinite(accU[q][e]);
-            Uo[(long long)(r0 + q) * DK + PK * lane + e] = accU[q][e];
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < PV; ++e) {
-            bad |= !isfinite(accV[q][e]);
-            Vo[(long long)(r0 + q) * DV + PV * lane + e] = accV[q][e];
-          }
-        }
+    for (int q = 0; q < kFastMaxR; ++q) {
+      if (q < p.R) {
+        const float v = acc[q] * rowf;
+        nonfinite |= !isfinite(v);
+        out[(long long)q * ld] = v;
       }
     }
-    __syncthreads();
   }
-  if (p.sigma_out && tid < p.R) p.sigma_out[(long long)idx * p.R + tid] = nrm[sel[tid]];
-  for (int e = tid; e < p.slen; e += 64) p.scale[unit * p.slen + e] = 1.f;
-  __syncthreads();
-  if (tid == 0) p.ncols[unit] = p.R;
-  if (bad) raise_flag(p.status, SEED_FLAG_NONFINITE);
+  const float sig_true = (lane < p.R) ? nrm[sel[lane]] * wmax : 0.f;
+  if (p.sigma_out && lane < p.R) p.sigma_out[(long long)idx * p.R + lane] = sig_true;
+  const float sk_lane = __shfl_sync(kFull, sk, lane & 15);
+  for (int e = lane; e < p.slen; e += 32)   // e < R <= 16 happens only with e == lane
+    p.scale[unit * p.slen + e] = (!KDA && e < p.R) ? sk_lane * wmax : 1.f;
+  if (lane == 0) p.ncols[unit] = p.R;
+  if (__any_sync(kFull, nonfinite) && lane == 0) raise_flag(p.status, SEED_FLAG_NONFINITE);
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !ptr)
+      return nullptr;
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// A factor array [units][m][D] as a 3-D float tensor {D, m, units}; boxes of 32 rows
+// of MP columns of one unit, 128-byte swizzle, zero fill outside (columns >= m).
+static bool make_panel_map(CUtensorMap* tm, const float* base, int D, int m, long long units, int MP) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)m, (cuuint64_t)units};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)m * D * 4};
+  const cuuint32_t box[3] = {32, (cuuint32_t)MP, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int FORM, int DK, int DV, int MP>
@@ -542,7 +732,12 @@ static int launch_fast_t(const FastParams& p, int blocks, cudaStream_t st) {
       return SEED_ERR_CUDA;
     attr_set[dev] = true;
   }
-  kern<<<blocks, 64, Lay::bytes, st>>>(p);
+  const long long units = (long long)p.B * p.L * p.H;
+  const int m = p.R + p.W;
+  CUtensorMap tmU, tmV;
+  if (!make_panel_map(&tmU, p.U, DK, m, units, MP) || !make_panel_map(&tmV, p.V, DV, m, units, MP))
+    return SEED_ERR_CUDA;
+  kern<<<blocks, 32, Lay::bytes, st>>>(p, tmU, tmV);
   return cudaGetLastError() == cudaSuccess ? SEED_OK : SEED_ERR_CUDA;
 }
 
@@ -554,10 +749,11 @@ static int launch_fast_m(const FastParams& p, int blocks, cudaStream_t st) {
 }
 
 // R <= 16: the R new columns are accumulated in registers in one pass over the
-// old ones, so that no output overwrites a column before every column was read.
+// old ones, so that no output overwrites a column before it was read.
 bool compress_fast_supported(const seed_dims& d) {
   const int m = d.R + d.W;
-  return m <= 32 && d.R <= 16 && (d.d_k == 64 || d.d_k == 128) && (d.d_v == 64 || d.d_v == 128);
+  return m <= 32 && d.R <= kFastMaxR && (d.d_k == 64 || d.d_k == 128) &&
+         (d.d_v == 64 || d.d_v == 128);
 }
 
 int launch_compress_fast(const seed_dims& d, const seed_state& s, int layer, float* sigma_out,

@@ -19,78 +19,11 @@
 // P (true U = Diag(P) * stored U); the new column is stored as k / P so that its
 // true value is k.  Both are folded back into U by the compression.
 #include "seed_common.cuh"
+#include "seed_decode.cuh"
 #include "seed_launch.h"
 #include "seed_tma.cuh"
 
 namespace seed {
-
-struct DecodeParams {
-  const float* q;
-  const float* k;
-  const float* v;
-  const float* alpha;
-  const float* beta;
-  float* o;
-  float* a;
-  float* U;
-  float* V;
-  float* scale;
-  int32_t* ncols;
-  const float* vbar;
-  uint32_t* status;
-  int B, L, H, layer, R, W, slen;
-};
-
-// One pipeline stage: everything a unit's step reads.
-template <int FORM, int DK, int DV, int MAXC>
-struct DecodeStage {
-  static constexpr bool KDA = FORM == SEED_KDA;
-  static constexpr int GPAD = (MAXC + 3) & ~3;
-  float U[MAXC * DK];
-  float V[MAXC * DV];
-  float a[DK];
-  float k[DK];
-  float q[DK];
-  float v[DV];
-  float vb[DV];
-  float al[KDA ? DK : 4];
-  float P[KDA ? DK : 4];
-  float gam[GPAD];
-  float g;
-  float beta;
-  int c;
-  int pad;
-};
-
-// Sum of NV per-lane values over the 32 lanes of a warp by recursive halving:
-// 2 NV - 2 shuffles for NV <= 32 instead of 5 NV.  Lane l ends up holding the
-// total of value (l >> (5 - log2 NV)) & (NV - 1).
-template <int NV>
-SEED_DEV float warp_xreduce(float (&v)[NV]) {
-  const int lane = threadIdx.x & 31;
-  int n = NV;
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) {
-    if (n > 1) {
-      const bool hi = (lane & off) != 0;
-#pragma unroll
-      for (int i = 0; i < NV / 2; ++i) {
-        if (i < n / 2) {
-          const float send = hi ? v[i] : v[i + n / 2];
-          const float keep = hi ? v[i + n / 2] : v[i];
-          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-        }
-      }
-      n >>= 1;
-    } else {
-      v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
-    }
-  }
-  return v[0];
-}
-
-template <int NV>
-SEED_DEV constexpr int log2c() { return NV <= 1 ? 0 : 1 + log2c<NV / 2>(); }
 
 constexpr int kConsumerWarps = 4;
 constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
@@ -427,12 +360,12 @@ static int launch_one(const DecodeParams& p, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? SEED_OK : SEED_ERR_CUDA;
 }
 
+// Up to 32 stored columns: one warp per unit (seed_decode_warp.cu); above, this
+// kernel with four consumer warps per unit.
 template <int FORM, int DK, int DV>
 static int launch_cols(const DecodeParams& p, cudaStream_t st) {
   const int maxc = p.R + p.W - 1;
-  if (maxc <= 8) return launch_one<FORM, DK, DV, 8>(p, st);
-  if (maxc <= 16) return launch_one<FORM, DK, DV, 16>(p, st);
-  if (maxc <= 32) return launch_one<FORM, DK, DV, 32>(p, st);
+  if (maxc <= 32) return launch_decode_warp(p, FORM, DK, DV, st);
   if (maxc <= 64) return launch_one<FORM, DK, DV, 64>(p, st);
   return launch_one<FORM, DK, DV, 96>(p, st);
 }

@@ -1,5 +1,5 @@
-// seed_tma.cuh -- TMA bulk copies and mbarriers (inline PTX, sm_90+ / sm_100a).
-// Only non-multicast global -> shared bulk copies are used.
+// seed_tma.cuh -- TMA bulk and tensor copies and mbarriers (inline PTX, sm_100a).
+// Only non-multicast global -> shared copies are used.
 #pragma once
 
 #include <stdint.h>
@@ -16,6 +16,11 @@ SEED_DEV void mbar_init(uint64_t* bar, uint32_t count) {
 
 // Make barrier initialisation visible to the async proxy before any bulk copy uses it.
 SEED_DEV void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+
+// Order this thread's earlier generic-proxy accesses to shared memory before later
+// async-proxy (bulk copy) accesses, e.g. before a copy overwrites a buffer that was
+// just written with ordinary stores.
+SEED_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 SEED_DEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
@@ -34,6 +39,17 @@ SEED_DEV void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
           smem_addr(dst)),
       "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// Tiled 3-D tensor copy global -> shared through a tensor map (no multicast),
+// completing on `bar`; coordinates innermost first.  The innermost coordinate x
+// times the element size must be a multiple of 16 bytes.
+SEED_DEV void tma_load_3d(void* dst, const void* tmap, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+          smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
       : "memory");
 }
 

@@ -53,3 +53,25 @@ def io_bytes(form: int, d_k: int, d_v: int) -> float:
 def mean_columns(R: int, W: int) -> float:
     """Mean column count before a step over one compression window: R + (W - 1) / 2."""
     return R + (W - 1) / 2.0
+
+
+def compress_flops(d_k: int, d_v: int, R: int, W: int, sweeps: float) -> float:
+    """Floating-point operations of one unit's compression by the QR route (the
+    truncation of Figure 1(b) of the SEED figures & tables page), m = R + W:
+
+      Gram matrices of U and V           2 (d_k + d_v) m^2
+      two Cholesky factorisations        2 m^3 / 3
+      core M = R_u R_v^T (triangular)    2 m^3 / 3
+      one-sided Jacobi, per sweep        m (m - 1) / 2 pairs x 6 m
+                                         (a dot product and a rotation of two m-columns)
+      left vectors and small factors     6 m^2 R
+      U' and V' from the stored panels   2 (d_k + d_v) m R
+    """
+    m = R + W
+    return (2.0 * (d_k + d_v) * m * m + 4.0 * m ** 3 / 3.0 + sweeps * (m * (m - 1) / 2.0) * 6.0 * m
+            + 6.0 * m * m * R + 2.0 * (d_k + d_v) * m * R)
+
+
+def fp32_peak_tflops(sm_mhz: float, sms: int = 148) -> float:
+    """FP32 FMA peak of the CUDA cores: SMs x 128 lanes x 2 flops x clock."""
+    return sms * 128 * 2 * sm_mhz * 1e6 / 1e12

@@ -79,7 +79,8 @@ def _run(form, dk, dv, R, W, repeat=False, zero_cols=0, n=24, seed=0):
 
 @pytest.mark.parametrize("form", [FORM_GDN, FORM_KDA, FORM_MAMBA2])
 @pytest.mark.parametrize("dk,dv,R,W", [(128, 128, 16, 16), (128, 64, 8, 8), (64, 64, 4, 12),
-                                       (128, 128, 32, 64), (16, 16, 4, 4), (128, 64, 8, 32)])
+                                       (128, 128, 8, 16), (64, 128, 12, 8), (128, 128, 32, 64),
+                                       (16, 16, 4, 4), (128, 64, 8, 32)])
 def test_compress_matches_truncated_svd(form, dk, dv, R, W):
     _run(form, dk, dv, R, W, seed=dk + R + W + form)
 
