@@ -35,6 +35,12 @@ if ROOT not in sys.path:
 METRIC = "decode head-steps/s and achieved HBM GB/s (% of B200 peak) at R=16,W=16"
 UNIT = "head-steps/s"
 NOMINAL_HBM_GBS = 8000.0
+# DRAM bytes (read + write) of one decode launch of the GDN stack shape, measured by ncu
+# (dram__bytes_read.sum + dram__bytes_write.sum; profiles/decode_warp_kernel_gdn_stack_2layers.md):
+# a full per-layer launch (256 requests x 48 heads) at c = 19 stored columns.  Set to None
+# whenever the decode kernel changes until it is measured again.
+NCU_DECODE_TRAFFIC = {"kernel": "decode_warp_kernel", "form": 0, "d_k": 128, "d_v": 128, "R": 16,
+                      "W": 16, "units": 12288, "c": 19, "bytes": 266.03e6 + 20.66e6}
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -255,6 +261,23 @@ def run_reference(args, world, rank):
 
 # ------------------------------------------------------------------ GPU arm
 
+def decode_kernel_name(d):
+    return "decode_warp_kernel" if d.R + d.W - 1 <= 32 else "decode_step_kernel"
+
+
+def decode_traffic(d, units, cbar):
+    """DRAM bytes per decode launch from the ncu capture, scaled from its units and
+    column count to this launch's by the state + input/output bytes; None when the
+    capture does not match this kernel and shape."""
+    from rank_recurrent_state_b200 import roofline
+    t = NCU_DECODE_TRAFFIC
+    if t is None or decode_kernel_name(d) != t["kernel"] or (d.form, d.d_k, d.d_v, d.R, d.W) != (
+            t["form"], t["d_k"], t["d_v"], t["R"], t["W"]):
+        return None
+    per = lambda c: roofline.lazy_bytes(d.form, d.d_k, d.d_v, c) + roofline.io_bytes(d.form, d.d_k, d.d_v)  # noqa: E731
+    return t["bytes"] / t["units"] * units * per(cbar) / per(t["c"])
+
+
 def compress_rate(d, diag, cmp_ms, clk):
     """FP32 rate of the compression launches (the FLOP model of roofline.compress_flops,
     with the measured mean Jacobi sweeps) and its fraction of the CUDA-core FP32 peak
@@ -380,9 +403,10 @@ def run_ours(args, world, rank, local):
         "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded Philox4x32-10 inputs and prefill, generated on the device)",
         "config": config_obj(cfg, B, world, prefill),
-        "roofline": {"bound": "hbm", "kernel": "decode_step_kernel", "achieved": dec_gbs, "peak": peak,
+        "roofline": {"bound": "hbm", "kernel": decode_kernel_name(d), "achieved": dec_gbs, "peak": peak,
                      "unit": "GB/s", "frac": dec_gbs / peak, "peak_source": f"{peak_kind} copy bandwidth",
-                     "frac_of_nominal_8TBs": dec_gbs / NOMINAL_HBM_GBS, "traffic": None,
+                     "frac_of_nominal_8TBs": dec_gbs / NOMINAL_HBM_GBS,
+                     "traffic": decode_traffic(d, BH, cbar),
                      "algorithmic_bytes_per_head_step_mean": roofline.lazy_bytes(d.form, d.d_k, d.d_v, cbar),
                      "avg_launch_us": 1e3 * sum(dec_ms) / len(dec_ms), "launches": len(dec_ms)},
         "decode_only": {"head_steps_per_s": len(dec_ms) * BH * world / (sum(dec_ms) / 1e3),

@@ -107,16 +107,19 @@ SEED_DEV float equilibrate_row(float (&g)[MP]) {
   return lane < MP ? n : 0.f;
 }
 
-// Right-looking Cholesky in registers, one warp, lane i holding row i of the
-// equilibrated Gram; on return row i of L (lower; the upper part zero).  Column j
-// is dropped (zero) when column j of the panel is zero (norm_j == 0) or the pivot
-// is not positive; a pivot below kCholPivotMin on a nonzero column sets `bad`.
-template <int MP>
-SEED_DEV void cholesky_regs(float (&g)[MP], float norm_self, bool& bad) {
+// Right-looking Cholesky of the equilibrated Gram, one warp, lane i holding row i
+// in registers; row i of L (lower, zero above the diagonal) is written to
+// L[i * LD ..].  The column loop is not unrolled, to keep the code small: after
+// step j every row is shifted down by one register, so that the current column is
+// always g[0].  Column j is dropped (zero) when column j of the panel is zero
+// (norm_j == 0) or the pivot is not positive; a pivot below kCholPivotMin on a
+// nonzero column sets `bad`.
+template <int MP, int LD>
+SEED_DEV void cholesky_rolled(float (&g)[MP], float norm_self, bool& bad, float* L) {
   const int lane = threadIdx.x & 31;
-#pragma unroll
+#pragma unroll 1
   for (int j = 0; j < MP; ++j) {
-    const float d = __shfl_sync(kFull, g[j], j);
+    const float d = __shfl_sync(kFull, g[0], j);
     const bool zero = !(__shfl_sync(kFull, norm_self, j) > 0.f);
     bool drop = zero || !(d > 0.f);
     if (!zero && d < kCholPivotMin) {
@@ -124,13 +127,16 @@ SEED_DEV void cholesky_regs(float (&g)[MP], float norm_self, bool& bad) {
       bad = true;
     }
     const float rs = drop ? 0.f : rsqrtf(d);
-    const float lij = lane > j ? g[j] * rs : 0.f;
-    g[j] = lane == j ? d * rs : lij;
+    const float lij = lane > j ? g[0] * rs : 0.f;
+    if (lane < MP) L[lane * LD + j] = lane == j ? d * rs : lij;
 #pragma unroll
-    for (int k = j + 1; k < MP; ++k) {
-      const float lkj = __shfl_sync(kFull, lij, k);
-      if (k <= lane) g[k] = fmaf(-lij, lkj, g[k]);
+    for (int t = 1; t < MP; ++t) {   // column j + t of the rows below
+      const float lkj = __shfl_sync(kFull, lij, (j + t) & 31);
+      if (j + t <= lane) g[t] = fmaf(-lij, lkj, g[t]);
     }
+#pragma unroll
+    for (int t = 0; t + 1 < MP; ++t) g[t] = g[t + 1];
+    g[MP - 1] = 0.f;
   }
 }
 
@@ -189,7 +195,7 @@ SEED_DEV int jacobi_regs(float* sM, bool& conv) {
     if (sweep == 0) tiny = 1e-10f * group_sum<32>(nx + ny) * (1.f / LP);
     // true column = s * stored column; r = 1 / s
     float sx = 1.f, sy = 1.f, rx = 1.f, ry = 1.f;
-    bool rot = false;
+    bool rot = false, big = false;
 #pragma unroll 1
     for (int G = NS; G >= 1; G >>= 1) {
 #pragma unroll 1
@@ -203,7 +209,9 @@ SEED_DEV int jacobi_regs(float* sM, bool& conv) {
           g3 = fmaf(x[i + 3], y[i + 3], g3);
         }
         const float g = pair_sum<LP>((g0 + g1) + (g2 + g3)) * (sx * sy);
-        if (nx > tiny && ny > tiny && g * g > tol2 * (nx * ny)) {
+        const bool live = nx > tiny && ny > tiny;
+        big |= live && g * g > 1e-6f * (nx * ny);
+        if (live && g * g > tol2 * (nx * ny)) {
           // Rutishauser's rotation, t = sign(d) 2g / (|d| + sqrt(d^2 + 4 g^2)) with
           // d = |y|^2 - |x|^2 (the smaller root of t^2 + (d / g) t - 1 = 0); the
           // fast reciprocal only perturbs t, c = 1 / sqrt(1 + t^2) keeps it orthogonal
@@ -266,7 +274,10 @@ SEED_DEV int jacobi_regs(float* sM, bool& conv) {
       y[i] *= sy;
     }
     sweeps = sweep + 1;
-    if (!__any_sync(kFull, rot)) {
+    // converged when nothing rotated, or when no pair was further from orthogonal
+    // than 1e-3 (relative): quadratic convergence then leaves every pair below the
+    // threshold after this sweep, so the sweep that would only confirm it is skipped
+    if (!__any_sync(kFull, rot) || !__any_sync(kFull, big)) {
       conv = true;
       break;
     }
@@ -303,11 +314,12 @@ SEED_DEV int swz(int j, int e) { return j * 32 + ((((e >> 2) ^ (j & 7)) << 2) | 
 
 // Gram row `lane` of one panel, accumulated over its chunks c0 .. c1-1 as they
 // arrive (issuing chunk c + 2 into a buffer once chunk c is read); also checks the
-// column scale.  FOLD (KDA's U): the products are weighted by P^2 (true U = Diag(P) U).
+// column scale.  fold (KDA's U): the products are weighted by P^2 (true U = Diag(P) U).
 // Returns false if a copy did not arrive in time (after waiting for those in flight).
-template <bool FOLD, int NCU, int NCH, int MP, int CHUNK>
-SEED_DEV bool gram_stream(int c0, int c1, float* sA, const CUtensorMap* tmU, const CUtensorMap* tmV,
-                          long long unit, int m, uint64_t* bar, const float* scl, float (&g)[MP], bool& bad) {
+template <bool KDA, int NCU, int NCH, int MP, int CHUNK>
+SEED_DEV bool gram_stream(int c0, int c1, bool fold, float* sA, const CUtensorMap* tmU,
+                          const CUtensorMap* tmV, long long unit, int m, uint64_t* bar, const float* scl,
+                          float (&g)[MP], bool& bad) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int i = 0; i < MP; ++i) g[i] = 0.f;
@@ -324,18 +336,21 @@ SEED_DEV bool gram_stream(int c0, int c1, float* sA, const CUtensorMap* tmU, con
     }
     const float* buf = sA + bb * CHUNK;
     const int r0 = 32 * (c < NCU ? c : c - NCU);
-#pragma unroll 2
+#pragma unroll 1
     for (int f = 0; f < 8; ++f) {
       float4 o = ld4(buf + jo * 32 + ((f ^ (jo & 7)) << 2));
       float4 pw = make_float4(1.f, 1.f, 1.f, 1.f);
-      if constexpr (FOLD) {
+      if (KDA && fold) {
         pw = ld4(scl + r0 + 4 * f);
         o = mul4(o, pw);
       }
       mx = fmaxf(mx, fmaxf(fmaxf(fabsf(o.x), fabsf(o.y)), fmaxf(fabsf(o.z), fabsf(o.w))));
-      if constexpr (FOLD) o = mul4(o, pw);
+      if (KDA && fold) o = mul4(o, pw);
 #pragma unroll
-      for (int i = 0; i < MP; ++i) g[i] += dot4(ld4(buf + i * 32 + ((f ^ (i & 7)) << 2)), o);
+      for (int i = 0; i < MP; ++i) {
+        const float4 b4 = ld4(buf + i * 32 + ((f ^ (i & 7)) << 2));
+        g[i] = fmaf(b4.x, o.x, fmaf(b4.y, o.y, fmaf(b4.z, o.z, fmaf(b4.w, o.w, g[i]))));
+      }
     }
     __syncwarp();   // every lane has read this chunk before the next copy overwrites it
     if (c + 2 < NCH) issue_chunk<NCU, CHUNK>(c + 2, sA, tmU, tmV, unit, bar);
@@ -410,38 +425,30 @@ __global__ void __launch_bounds__(32)
   issue_chunk<NCU, CHUNK>(1, sA, &tmU, &tmV, unit, bar);
   bool bad = false;   // ill-conditioned or badly scaled: left for the Householder kernel
   float g[MP];
-  // U: chunks 0 .. NCU-1, then its Cholesky factor
-  if (!gram_stream<KDA, NCU, NCH, MP, CHUNK>(0, NCU, sA, &tmU, &tmV, unit, m, bar, scl, g, bad)) {
+  // U: chunks 0 .. NCU-1, then its Cholesky factor (to its own region)
+  if (!gram_stream<KDA, NCU, NCH, MP, CHUNK>(0, NCU, true, sA, &tmU, &tmV, unit, m, bar, scl, g, bad)) {
     if (lane == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
     return;
   }
   {
     const float n = equilibrate_row<MP>(g);
     if (lane < MP) nu[lane] = n;
-    cholesky_regs<MP>(g, n, bad);
-    if (lane < MP) {
-#pragma unroll
-      for (int k = 0; k < MP; k += 4) st4(sLu + lane * LG + k, make_float4(g[k], g[k + 1], g[k + 2], g[k + 3]));
-    }
+    cholesky_rolled<MP, LG>(g, n, bad, sLu);
   }
-  // V: chunks NCU .. NCH-1
-  if (!gram_stream<false, NCU, NCH, MP, CHUNK>(NCU, NCH, sA, &tmU, &tmV, unit, m, bar, scl, g, bad)) {
+  // V: chunks NCU .. NCH-1; L_v over the chunk buffers once the last one is read
+  if (!gram_stream<KDA, NCU, NCH, MP, CHUNK>(NCU, NCH, false, sA, &tmU, &tmV, unit, m, bar, scl, g, bad)) {
     if (lane == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
     return;
   }
   {
     const float n = equilibrate_row<MP>(g);
     if (lane < MP) nv[lane] = n;
-    cholesky_regs<MP>(g, n, bad);
+    __syncwarp();   // every lane has read the last V chunk before L_v overwrites it
+    cholesky_rolled<MP, LG>(g, n, bad, sM);
   }
   if (__any_sync(kFull, bad)) {
     if (lane == 0) atomicAdd(p.status + 6, 1u);
     return;
-  }
-  // L_v over the (now idle) chunk buffers, row-major
-  if (lane < MP) {
-#pragma unroll
-    for (int k = 0; k < MP; k += 4) st4(sM + lane * LG + k, make_float4(g[k], g[k + 1], g[k + 2], g[k + 3]));
   }
 
   // D_u, D_v: true column norms (GDN / Mamba-2: with the lazy scale gamma_j); the
@@ -460,28 +467,25 @@ __global__ void __launch_bounds__(32)
   __syncwarp();
 
   // 2. core M = L_u^T diag(w) L_v in place of L_v, column j in lane j:
-  //    M[i][j] = sum_{k >= max(i, j)} L_u[k][i] w_k L_v[k][j]
+  //    M[i][j] = sum_{k >= max(i, j)} L_u[k][i] w_k L_v[k][j]   (L_u, L_v lower triangular)
   {
     const int j = lane < MP ? lane : 0;
-    float lv[MP];
-#pragma unroll
-    for (int k = 0; k < MP; ++k) lv[k] = k >= j ? sM[k * LG + j] * (du[k] * dvv[k] * winv) : 0.f;
-    __syncwarp();   // every lane holds its column of L_v before M overwrites it
     float acc[MP];
 #pragma unroll
     for (int i = 0; i < MP; ++i) acc[i] = 0.f;
-#pragma unroll
+#pragma unroll 2
     for (int k = 0; k < MP; ++k) {
-      const float cf = lv[k];
+      const float cf = sM[k * LG + j] * (du[k] * dvv[k] * winv);
 #pragma unroll
-      for (int i4 = 0; i4 <= k; i4 += 4) {
+      for (int i4 = 0; i4 < MP; i4 += 4) {
         const float4 l = ld4(sLu + k * LG + i4);
         acc[i4] = fmaf(cf, l.x, acc[i4]);
-        if (i4 + 1 <= k) acc[i4 + 1] = fmaf(cf, l.y, acc[i4 + 1]);
-        if (i4 + 2 <= k) acc[i4 + 2] = fmaf(cf, l.z, acc[i4 + 2]);
-        if (i4 + 3 <= k) acc[i4 + 3] = fmaf(cf, l.w, acc[i4 + 3]);
+        acc[i4 + 1] = fmaf(cf, l.y, acc[i4 + 1]);
+        acc[i4 + 2] = fmaf(cf, l.z, acc[i4 + 2]);
+        acc[i4 + 3] = fmaf(cf, l.w, acc[i4 + 3]);
       }
     }
+    __syncwarp();   // every lane has read L_v before M overwrites it
     if (lane < MP) {
 #pragma unroll
       for (int i = 0; i < MP; i += 4) st4(sM + lane * LG + i, make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]));
@@ -567,61 +571,64 @@ __global__ void __launch_bounds__(32)
     }
   }
 
-  // 5. small right factors on the stored panels (column r in registers of lane r
-  //    for T_u, of lane 16 + r for T_v).  With sigma = wmax * sk the true value:
+  // 5. small right factors on the stored panels, lane k holding row k of both:
+  //    with sigma_r = wmax * sk_r the true singular value,
   //      GDN / Mamba-2 (a per-column scale exists): unit columns, the scale = sigma
   //        U' = U_st T_u, T_u = diag(1 / nu) L_u^{-T} X_R
   //        V' = V_st T_v, T_v = D_u L_u X_R Sigma^{-1}
   //      KDA: balanced, Sigma^{1/2} on each side (the row products P applied to U'
   //        after the product, and reset to 1)
-  //    then stored [k][r] (stride 16) over L_u: T_u first, T_v after it (T_v goes
-  //    through the Gram-Schmidt scratch while the other half still reads L_u)
+  //    then stored [k][r] (stride 16) over L_u: T_u first, T_v after it
   {
-    const int r = lane & 15;
-    const float s = __shfl_sync(kFull, sk, r) * wmax;
-    const bool zero = !(s > 0.f) || r >= p.R;
-    float t[MP];
-    if (lane < 16) {
-      // back substitution with L_u^T (upper): t_k = (x_k - sum_{i>k} L_u[i][k] t_i) / L_u[k][k]
-      const float f = zero ? 0.f : (KDA ? sqrtf(s) : 1.f);
+    float fu[kFastMaxR], fv[kFastMaxR];
 #pragma unroll
-      for (int k = MP - 1; k >= 0; --k) {
-        float acc = zero ? 0.f : sX[r * LX + k] * f;
+    for (int r = 0; r < kFastMaxR; ++r) {
+      const float sr = __shfl_sync(kFull, sk, r) * wmax;
+      const bool zero = !(sr > 0.f) || r >= p.R;
+      fu[r] = zero ? 0.f : (KDA ? sqrtf(sr) : 1.f);
+      fv[r] = zero ? 0.f : (KDA ? rsqrtf(sr) : 1.f / sr);
+    }
+    const int k = lane < MP ? lane : 0;
+    float bu[kFastMaxR], bv[kFastMaxR];
 #pragma unroll
-        for (int i = k + 1; i < MP; ++i) acc = fmaf(-sLu[i * LG + k], t[i], acc);
-        const float lkk = sLu[k * LG + k];
-        t[k] = lkk != 0.f ? acc / lkk : 0.f;
-      }
+    for (int r = 0; r < kFastMaxR; ++r) {
+      bu[r] = (lane < MP && r < p.R) ? sX[r * LX + k] * fu[r] : 0.f;
+      bv[r] = 0.f;
+    }
+    // T_v rows: (L_u X_R^T)_k = sum_{i <= k} L_u[k][i] x_r[i]  (L_u[k][i] = 0 above the diagonal)
+#pragma unroll 2
+    for (int i = 0; i < MP; ++i) {
+      const float l = sLu[k * LG + i];
 #pragma unroll
-      for (int k = 0; k < MP; ++k) {
-        const float n = nu[k];
-        t[k] = n > 0.f ? t[k] / n : 0.f;
-      }
-    } else {
-      const float f = zero ? 0.f : (KDA ? rsqrtf(s) : 1.f / s);
-      float x[MP];
+      for (int r = 0; r < kFastMaxR; ++r) bv[r] = fmaf(l, sX[r * LX + i], bv[r]);
+    }
+    // T_u: back substitution with L_u^T by columns: once row kk is final, remove its
+    // part from every row above it
+#pragma unroll 1
+    for (int kk = MP - 1; kk >= 0; --kk) {
+      const float lkk = sLu[kk * LG + kk];
+      const float rl = lkk != 0.f ? 1.f / lkk : 0.f;
+      const float lk = sLu[kk * LG + k];   // L_u[kk][k], used by rows k < kk
 #pragma unroll
-      for (int i = 0; i < MP; ++i) x[i] = zero ? 0.f : sX[r * LX + i];
-#pragma unroll
-      for (int k = 0; k < MP; ++k) {
-        float acc = 0.f;
-#pragma unroll
-        for (int i4 = 0; i4 <= k; i4 += 4) {
-          const float4 l = ld4(sLu + k * LG + i4);
-          acc = fmaf(l.x, x[i4], acc);
-          if (i4 + 1 <= k) acc = fmaf(l.y, x[i4 + 1], acc);
-          if (i4 + 2 <= k) acc = fmaf(l.z, x[i4 + 2], acc);
-          if (i4 + 3 <= k) acc = fmaf(l.w, x[i4 + 3], acc);
-        }
-        sP[k * kFastMaxR + r] = du[k] * acc * f;
+      for (int r = 0; r < kFastMaxR; ++r) {
+        if (lane == kk) bu[r] *= rl;
+        const float tk = __shfl_sync(kFull, bu[r], kk);
+        if (lane < kk) bu[r] = fmaf(-lk, tk, bu[r]);
       }
     }
-    __syncwarp();   // every lane has read L_u and X
-    if (lane < 16) {
+    const float nk = lane < MP ? nu[k] : 0.f;
+    const float rn = nk > 0.f ? 1.f / nk : 0.f;
+    const float dk = lane < MP ? du[k] : 0.f;
+    __syncwarp();   // every lane has read L_u
+    if (lane < MP) {
 #pragma unroll
-      for (int k = 0; k < MP; ++k) sLu[k * kFastMaxR + r] = t[k];
+      for (int r = 0; r < kFastMaxR; r += 4) {
+        st4(sLu + k * kFastMaxR + r, make_float4(bu[r] * rn, bu[r + 1] * rn, bu[r + 2] * rn, bu[r + 3] * rn));
+        st4(sLu + MP * kFastMaxR + k * kFastMaxR + r,
+            make_float4(dk * bv[r] * fv[r], dk * bv[r + 1] * fv[r + 1], dk * bv[r + 2] * fv[r + 2],
+                        dk * bv[r + 3] * fv[r + 3]));
+      }
     }
-    for (int e = lane; e < MP * kFastMaxR; e += 32) sLu[MP * kFastMaxR + e] = sP[e];
     __syncwarp();
   }
   const float* sTu = sLu;

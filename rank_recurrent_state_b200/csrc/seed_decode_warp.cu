@@ -151,17 +151,23 @@ __global__ void __launch_bounds__(32) decode_warp_kernel(const DecodeParams p) {
     const int u = u0 + NSW * stride;
     if (u < n_units) c_next = p.ncols[unit_index(p, u)];
   }
+  // the scalars of the current unit, loaded one unit ahead
+  float g_cur = (KDA || u0 >= n_units) ? 1.f : p.alpha[u0];
+  float b_cur = u0 < n_units ? p.beta[u0] : 0.f;
 
   for (int i = 0, u = u0; u < n_units; ++i, u += stride) {
     const int s = NSW == 1 ? 0 : (i & 1);
     const uint32_t ph = (uint32_t)(i / NSW) & 1u;
     const int c = s == 0 ? c_s0 : c_s1;
     const long long unit = unit_index(p, u);
-    const float g = KDA ? 1.f : p.alpha[u];
-    const float be = p.beta[u];
+    const float g = g_cur, be = b_cur;
     const int u_next = u + NSW * stride;
     const int u_after = u_next + stride;
     const int c_after = u_after < n_units ? p.ncols[unit_index(p, u_after)] : 0;
+    if (u + stride < n_units) {
+      g_cur = KDA ? 1.f : p.alpha[u + stride];
+      b_cur = p.beta[u + stride];
+    }
 
     if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full[s], ph, kWaitLimitNs))) {
       if (lane == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);

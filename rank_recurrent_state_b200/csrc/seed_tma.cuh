@@ -71,14 +71,25 @@ SEED_DEV uint64_t global_ns() {
 
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s
 
-// Bounded wait for the phase with the given parity: polls without blocking, with
-// a short sleep between polls, and gives up after `limit_ns` of wall time.
+// Like mbar_test_wait, but the thread may be suspended for a while (a time the
+// hardware chooses) until the phase completes; returns false if it has not.
+SEED_DEV bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(phase)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity: suspending tries, and gives up
+// after `limit_ns` of wall time.
 SEED_DEV bool mbar_wait_bounded(uint64_t* bar, uint32_t phase, uint64_t limit_ns) {
   if (mbar_test_wait(bar, phase)) return true;
   const uint64_t t0 = global_ns();
-  while (!mbar_test_wait(bar, phase)) {
+  while (!mbar_try_wait(bar, phase)) {
     if (global_ns() - t0 > limit_ns) return false;
-    __nanosleep(32);
   }
   return true;
 }
