@@ -312,19 +312,56 @@ SEED_DEV void issue_chunk(int c, float* sA, const CUtensorMap* tmU, const CUtens
 // Offset (in floats) of element e of column j in a swizzled chunk buffer.
 SEED_DEV int swz(int j, int e) { return j * 32 + ((((e >> 2) ^ (j & 7)) << 2) | (e & 3)); }
 
-// Gram row `lane` of one panel, accumulated over its chunks c0 .. c1-1 as they
-// arrive (issuing chunk c + 2 into a buffer once chunk c is read); also checks the
-// column scale.  fold (KDA's U): the products are weighted by P^2 (true U = Diag(P) U).
-// Returns false if a copy did not arrive in time (after waiting for those in flight).
-template <bool KDA, int NCU, int NCH, int MP, int CHUNK>
+// Tensor-core products in float32 accuracy: x = hi + lo with hi = tf32(x) and
+// lo = tf32(x - hi), and a b ~ hi_a hi_b + hi_a lo_b + lo_a hi_b (the dropped
+// lo_a lo_b is below 2^-21 of a b), each term one warp-level mma.sync m16n8k8 with
+// float32 accumulation.
+SEED_DEV void tf32_split(float x, uint32_t& hi, uint32_t& lo) {
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
+  const float r = x - __uint_as_float(hi);
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(lo) : "f"(r));
+}
+
+SEED_DEV void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+SEED_DEV void mma3_tf32(float (&d)[4], const uint32_t (&ah)[4], const uint32_t (&al)[4], uint32_t bh0,
+                        uint32_t bh1, uint32_t bl0, uint32_t bl1) {
+  mma_tf32(d, ah, bl0, bl1);
+  mma_tf32(d, al, bh0, bh1);
+  mma_tf32(d, ah, bh0, bh1);
+}
+
+// Gram matrix of one panel, accumulated over its chunks c0 .. c1-1 as they arrive
+// (chunk c + 2 is issued into a buffer once chunk c is read) with tensor-core tiles:
+// G = P^T P as (MP x 32-row chunk) x (32-row chunk x MP) products, the upper block
+// triangle only (m16n8 tiles with n-tile >= 2 m-tile), mirrored when written to Gs
+// (row-major, stride LG); then lane i loads row i of G into g.  The A operand of
+// an m-tile is made of the B operands of n-tiles 2 mt and 2 mt + 1 (the same panel
+// columns).  fold (KDA's U): entries weighted by P (true U = Diag(P) U).  Also
+// checks the column scale.  Returns false if a copy did not arrive in time (after
+// waiting for those in flight).
+template <bool KDA, int NCU, int NCH, int MP, int CHUNK, int LG>
 SEED_DEV bool gram_stream(int c0, int c1, bool fold, float* sA, const CUtensorMap* tmU,
                           const CUtensorMap* tmV, long long unit, int m, uint64_t* bar, const float* scl,
-                          float (&g)[MP], bool& bad) {
-  const int lane = threadIdx.x & 31;
+                          float* Gs, float (&g)[MP], bool& bad) {
+  constexpr int NT = MP / 8, MT = MP / 16;
+  const int lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
+  float acc[MT][NT][4];
 #pragma unroll
-  for (int i = 0; i < MP; ++i) g[i] = 0.f;
-  float mx = 0.f;
-  const int jo = lane < MP ? lane : 0;
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+  float mx[NT];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) mx[nt] = 0.f;
 #pragma unroll 1
   for (int c = c0; c < c1; ++c) {
     const int bb = c & 1;
@@ -337,25 +374,63 @@ SEED_DEV bool gram_stream(int c0, int c1, bool fold, float* sA, const CUtensorMa
     const float* buf = sA + bb * CHUNK;
     const int r0 = 32 * (c < NCU ? c : c - NCU);
 #pragma unroll 1
-    for (int f = 0; f < 8; ++f) {
-      float4 o = ld4(buf + jo * 32 + ((f ^ (jo & 7)) << 2));
-      float4 pw = make_float4(1.f, 1.f, 1.f, 1.f);
-      if (KDA && fold) {
-        pw = ld4(scl + r0 + 4 * f);
-        o = mul4(o, pw);
-      }
-      mx = fmaxf(mx, fmaxf(fmaxf(fabsf(o.x), fabsf(o.y)), fmaxf(fabsf(o.z), fabsf(o.w))));
-      if (KDA && fold) o = mul4(o, pw);
+    for (int ks = 0; ks < 4; ++ks) {
+      uint32_t bh[NT][2], bl[NT][2];
 #pragma unroll
-      for (int i = 0; i < MP; ++i) {
-        const float4 b4 = ld4(buf + i * 32 + ((f ^ (i & 7)) << 2));
-        g[i] = fmaf(b4.x, o.x, fmaf(b4.y, o.y, fmaf(b4.z, o.z, fmaf(b4.w, o.w, g[i]))));
+      for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int row = ks * 8 + tq + 4 * h;
+          float x = buf[swz(nt * 8 + gq, row)];
+          if (KDA && fold) x *= scl[r0 + row];   // both operands carry P: P^2 in the product
+          mx[nt] = fmaxf(mx[nt], fabsf(x));
+          tf32_split(x, bh[nt][h], bl[nt][h]);
+        }
+      }
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        const uint32_t ah[4] = {bh[2 * mt][0], bh[2 * mt + 1][0], bh[2 * mt][1], bh[2 * mt + 1][1]};
+        const uint32_t al[4] = {bl[2 * mt][0], bl[2 * mt + 1][0], bl[2 * mt][1], bl[2 * mt + 1][1]};
+#pragma unroll
+        for (int nt = 2 * mt; nt < NT; ++nt)
+          mma3_tf32(acc[mt][nt], ah, al, bh[nt][0], bh[nt][1], bl[nt][0], bl[nt][1]);
       }
     }
     __syncwarp();   // every lane has read this chunk before the next copy overwrites it
     if (c + 2 < NCH) issue_chunk<NCU, CHUNK>(c + 2, sA, tmU, tmV, unit, bar);
   }
-  if (lane < m && mx > 0.f && (mx < kColMin || mx > kColMax)) bad = true;
+  // largest magnitude of column nt * 8 + gq, over the four lanes of the group
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    float v = fmaxf(mx[nt], __shfl_xor_sync(kFull, mx[nt], 1));
+    v = fmaxf(v, __shfl_xor_sync(kFull, v, 2));
+    if (nt * 8 + gq < m && v > 0.f && (v < kColMin || v > kColMax)) bad = true;
+  }
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+    for (int nt = 2 * mt; nt < NT; ++nt) {
+      const int row = mt * 16 + gq, col = nt * 8 + 2 * tq;
+      Gs[row * LG + col] = acc[mt][nt][0];
+      Gs[row * LG + col + 1] = acc[mt][nt][1];
+      Gs[(row + 8) * LG + col] = acc[mt][nt][2];
+      Gs[(row + 8) * LG + col + 1] = acc[mt][nt][3];
+      if (nt >= 2 * mt + 2) {   // off the diagonal blocks: the transposed entries too
+        Gs[col * LG + row] = acc[mt][nt][0];
+        Gs[(col + 1) * LG + row] = acc[mt][nt][1];
+        Gs[col * LG + row + 8] = acc[mt][nt][2];
+        Gs[(col + 1) * LG + row + 8] = acc[mt][nt][3];
+      }
+    }
+  }
+  __syncwarp();
+  const int i = lane < MP ? lane : 0;
+#pragma unroll
+  for (int k = 0; k < MP; k += 4) {
+    const float4 v = ld4(Gs + i * LG + k);
+    g[k] = v.x; g[k + 1] = v.y; g[k + 2] = v.z; g[k + 3] = v.w;
+  }
+  __syncwarp();   // every lane has its row before Gs is overwritten
   return true;
 }
 
@@ -426,7 +501,7 @@ __global__ void __launch_bounds__(32)
   bool bad = false;   // ill-conditioned or badly scaled: left for the Householder kernel
   float g[MP];
   // U: chunks 0 .. NCU-1, then its Cholesky factor (to its own region)
-  if (!gram_stream<KDA, NCU, NCH, MP, CHUNK>(0, NCU, true, sA, &tmU, &tmV, unit, m, bar, scl, g, bad)) {
+  if (!gram_stream<KDA, NCU, NCH, MP, CHUNK, LG>(0, NCU, true, sA, &tmU, &tmV, unit, m, bar, scl, sLu, g, bad)) {
     if (lane == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
     return;
   }
@@ -436,7 +511,7 @@ __global__ void __launch_bounds__(32)
     cholesky_rolled<MP, LG>(g, n, bad, sLu);
   }
   // V: chunks NCU .. NCH-1; L_v over the chunk buffers once the last one is read
-  if (!gram_stream<KDA, NCU, NCH, MP, CHUNK>(NCU, NCH, false, sA, &tmU, &tmV, unit, m, bar, scl, g, bad)) {
+  if (!gram_stream<KDA, NCU, NCH, MP, CHUNK, LG>(NCU, NCH, false, sA, &tmU, &tmV, unit, m, bar, scl, sM, g, bad)) {
     if (lane == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
     return;
   }
@@ -659,32 +734,59 @@ __global__ void __launch_bounds__(32)
     const int r0 = 32 * (isU ? c : c - NCU);
     const float* buf = sA + bb * CHUNK;
     const float* T = isU ? sTu : sTv;
-    float acc[kFastMaxR];
+    // out (32 rows x 16) = chunk (32 rows x MP) T (MP x 16): m16n8k8 tiles, rows
+    // mt * 16 + .., output columns nt * 8 + ..; columns >= m are zero in both
+    const int gq = lane >> 2, tq = lane & 3;
+    float acc[2][2][4];
 #pragma unroll
-    for (int q = 0; q < kFastMaxR; ++q) acc[q] = 0.f;
-#pragma unroll 4
-    for (int k = 0; k < m; ++k) {
-      const float xv = buf[swz(k, lane)];
+    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-      for (int q = 0; q < kFastMaxR; q += 4) {
-        const float4 tk = ld4(T + k * kFastMaxR + q);
-        acc[q] = fmaf(xv, tk.x, acc[q]);
-        acc[q + 1] = fmaf(xv, tk.y, acc[q + 1]);
-        acc[q + 2] = fmaf(xv, tk.z, acc[q + 2]);
-        acc[q + 3] = fmaf(xv, tk.w, acc[q + 3]);
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < MP / 8; ++ks) {
+      const int k = ks * 8 + tq;
+      uint32_t bh[2][2], bl[2][2];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        tf32_split(T[k * kFastMaxR + nt * 8 + gq], bh[nt][0], bl[nt][0]);
+        tf32_split(T[(k + 4) * kFastMaxR + nt * 8 + gq], bh[nt][1], bl[nt][1]);
+      }
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        const int r = mt * 16 + gq;
+        uint32_t ah[4], al[4];
+        tf32_split(buf[swz(k, r)], ah[0], al[0]);
+        tf32_split(buf[swz(k, r + 8)], ah[1], al[1]);
+        tf32_split(buf[swz(k + 4, r)], ah[2], al[2]);
+        tf32_split(buf[swz(k + 4, r + 8)], ah[3], al[3]);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) mma3_tf32(acc[mt][nt], ah, al, bh[nt][0], bh[nt][1], bl[nt][0], bl[nt][1]);
       }
     }
     __syncwarp();   // every lane has read this chunk before the next copy overwrites it
     if (c + 2 < NCH) issue_chunk<NCU, CHUNK>(c + 2, sA, &tmU, &tmV, unit, bar);
-    const float rowf = (KDA && isU) ? scl[r0 + lane] : 1.f;
-    float* out = (isU ? Uo : Vo) + r0 + lane;
+    float* out = (isU ? Uo : Vo) + r0;
     const int ld = isU ? DK : DV;
 #pragma unroll
-    for (int q = 0; q < kFastMaxR; ++q) {
-      if (q < p.R) {
-        const float v = acc[q] * rowf;
-        nonfinite |= !isfinite(v);
-        out[(long long)q * ld] = v;
+    for (int mt = 0; mt < 2; ++mt) {
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int r = mt * 16 + gq + 8 * hh;
+        const float rowf = (KDA && isU) ? scl[r0 + r] : 1.f;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int q = nt * 8 + 2 * tq + e;
+            if (q < p.R) {
+              const float v = acc[mt][nt][2 * hh + e] * rowf;
+              nonfinite |= !isfinite(v);
+              out[(long long)q * ld + r] = v;
+            }
+          }
+        }
       }
     }
   }

@@ -12,8 +12,9 @@
 // it, so the copies of one warp overlap the arithmetic of the others.  Each lane
 // holds d_k / 32 rows of every U column and d_v / 32 rows of every V column:
 //   1. U^T q and U^T k by partial dot products over the lane's rows, summed over
-//      the warp eight columns at a time by a transposed (recursive-halving)
-//      reduction;
+//      the warp sixteen columns at a time by a transposed (recursive-halving)
+//      reduction that leaves one dot per lane, which that lane scales into the
+//      column's coefficient for step 3;
 //   2. the scalars k^T a, a^T q, k^T q, v^T vbar, vbar^T vbar the same way;
 //   3. y_k = V (g gamma (.) U^T k) and y_q = V (g gamma (.) U^T q), each lane for
 //      its own rows, no reduction;
@@ -100,7 +101,7 @@ SEED_DEV void issue_unit(const DecodeParams& p, DecodeStage<FORM, DK, DV, MAXC>&
 template <int FORM, int DK, int DV, int MAXC, int NSW>
 struct WarpDecodeLayout {
   using Stage = DecodeStage<FORM, DK, DV, MAXC>;
-  static constexpr int NCH = (MAXC + 7) / 8;   // column chunks of eight
+  static constexpr int NCH = (MAXC + 31) / 32 * 4;   // coefficient pairs, in units of 8
   static constexpr size_t OFF_BAR = NSW * sizeof(Stage);
   static constexpr size_t OFF_DOT = OFF_BAR + 16 * ((NSW * 8 + 15) / 16);
   static constexpr size_t bytes = OFF_DOT + 2 * NCH * 8 * sizeof(float);
@@ -114,14 +115,12 @@ __global__ void __launch_bounds__(32) decode_warp_kernel(const DecodeParams p) {
   constexpr bool M2 = FORM == SEED_MAMBA2;
   constexpr int PK = DK >= 32 ? DK / 32 : 1;   // U rows per lane (d_k = 16: half the lanes)
   constexpr int PV = DV >= 32 ? DV / 32 : 1;
-  constexpr int NV = M2 ? 8 : 16;              // partial dots per chunk of eight columns
-  constexpr int SH = 5 - log2c<NV>();
+  constexpr int CPS = M2 ? 32 : 16;            // columns per warp reduction
   static_assert(NSW == 1 || NSW == 2, "one or two stages per warp");
   extern __shared__ __align__(128) unsigned char smem_raw[];
   Stage* stages = reinterpret_cast<Stage*>(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + Lay::OFF_BAR);
-  float* s_dq = reinterpret_cast<float*>(smem_raw + Lay::OFF_DOT);
-  float* s_dk = s_dq + Lay::NCH * 8;
+  float* s_f = reinterpret_cast<float*>(smem_raw + Lay::OFF_DOT);   // [MAXC][2]
 
   const int lane = threadIdx.x;
   const bool kact = DK >= 32 || lane < DK;
@@ -199,26 +198,26 @@ __global__ void __launch_bounds__(32) decode_warp_kernel(const DecodeParams p) {
         kk[e] = kr[e] * pp;
         qq[e] = qr[e] * pp;
       }
-      for (int ch = 0; ch * 8 < c; ++ch) {
-        float dv[NV];
+      // 16 columns per reduction (32 for Mamba-2, which has no erase): lane l ends up
+      // with dot number l; it turns it into the column's y coefficient
+      // g gamma_j (U^T q)_j or g gamma_j (U^T k)_j, stored as (q, k) pairs
+      for (int c0 = 0; c0 < c; c0 += CPS) {
+        float dv[32];
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          const int j = ch * 8 + t;
+        for (int t = 0; t < CPS; ++t) {
+          const int j = c0 + t;
           float ue[PK];
 #pragma unroll
           for (int e = 0; e < PK; ++e) ue[e] = 0.f;
           if (j < c && kact) ldv<PK>(S.U + j * DK + lane * PK, ue);
           dv[t] = dotv<PK>(ue, qq);
-          if constexpr (!M2) dv[8 + t] = dotv<PK>(ue, kk);
+          if constexpr (!M2) dv[16 + t] = dotv<PK>(ue, kk);
         }
-        const float tot = warp_xreduce<NV>(dv);
-        if ((lane & ((1 << SH) - 1)) == 0) {
-          const int idx = (lane >> SH) & (NV - 1);
-          const int j = ch * 8 + (idx & 7);
-          if (j < c) {
-            if (idx < 8) s_dq[j] = tot;
-            else s_dk[j] = tot;
-          }
+        const float tot = warp_xreduce<32>(dv);
+        const int j = c0 + (M2 ? lane : (lane & 15));
+        if (j < c) {
+          const float f = KDA ? 1.f : g * S.gam[j];
+          s_f[2 * j + (M2 ? 0 : (lane >> 4))] = f * tot;
         }
       }
       // 2. scalars: k^T a', a'^T q, k^T q (a' = alpha (.) a for KDA), v^T vbar, vbar^T vbar
@@ -248,7 +247,7 @@ __global__ void __launch_bounds__(32) decode_warp_kernel(const DecodeParams p) {
       const float kq = __shfl_sync(0xffffffffu, tot, 8);
       const float vvb = __shfl_sync(0xffffffffu, tot, 12);
       const float vbvb = __shfl_sync(0xffffffffu, tot, 16);
-      __syncwarp();   // the column dots are in s_dq / s_dk
+      __syncwarp();   // the column coefficients are in s_f
       if (!(vbvb > 0.f)) {
         if (lane == 0) raise_flag(p.status, SEED_FLAG_ZERO_VBAR);
       } else {
@@ -264,13 +263,11 @@ __global__ void __launch_bounds__(32) decode_warp_kernel(const DecodeParams p) {
 #pragma unroll
           for (int e = 0; e < PV; ++e) ve[e] = 0.f;
           if (vact) ldv<PV>(S.V + j * DV + lane * PV, ve);
-          const float f = KDA ? 1.f : g * S.gam[j];
-          const float fq = f * s_dq[j];
-          const float fk = M2 ? 0.f : f * s_dk[j];
+          const float2 f2 = *reinterpret_cast<const float2*>(s_f + 2 * j);   // (q, k) coefficients
 #pragma unroll
           for (int e = 0; e < PV; ++e) {
-            if constexpr (!M2) yk[e] = fmaf(fk, ve[e], yk[e]);
-            yq[e] = fmaf(fq, ve[e], yq[e]);
+            if constexpr (!M2) yk[e] = fmaf(f2.y, ve[e], yk[e]);
+            yq[e] = fmaf(f2.x, ve[e], yq[e]);
           }
         }
         // 4. sink update, new column pair, read-out
@@ -318,7 +315,7 @@ __global__ void __launch_bounds__(32) decode_warp_kernel(const DecodeParams p) {
         if (__any_sync(0xffffffffu, bad) && lane == 0) raise_flag(p.status, SEED_FLAG_NONFINITE);
       }
     }
-    // every read of the stage (and of s_dq / s_dk) is above: refill the stage
+    // every read of the stage (and of s_f) is above: refill the stage
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0 && u_next < n_units) issue_unit<FORM, DK, DV, MAXC>(p, stages[s], &full[s], u_next, c_next, m);
