@@ -6,11 +6,14 @@
 //
 // With at most 32 stored columns a unit is small enough for one warp, and a warp
 // that owns a unit needs no block-level synchronisation at all.  Every warp of a
-// persistent grid (one warp per block) owns NSW shared-memory stages; lane 0 fills
-// a stage with TMA bulk copies (cp.async.bulk, completion on the stage's mbarrier,
-// no multicast) for the warp's next unit as soon as the warp has finished reading
-// it, so the copies of one warp overlap the arithmetic of the others.  Each lane
-// holds d_k / 32 rows of every U column and d_v / 32 rows of every V column:
+// persistent grid (one warp per block) owns one shared-memory stage sized for the
+// R + W - 1 columns a unit holds at most before a step; lane 0 fills it with two
+// TMA bulk copies (cp.async.bulk of the stored U and V columns, completion on the
+// stage's mbarrier, no multicast) for the warp's next unit as soon as the warp has
+// read the current one, so the copies of one warp overlap the arithmetic of the
+// others.  The per-unit vectors (k, q, a, v, vbar, the decay scales, g, beta) go
+// straight from HBM into each lane's registers with coalesced loads issued one unit
+// ahead, so that they cost neither stage space nor copies:
 //   1. U^T q and U^T k by partial dot products over the lane's rows, summed over
 //      the warp sixteen columns at a time by a transposed (recursive-halving)
 //      reduction that leaves one dot per lane, which that lane scales into the
@@ -65,138 +68,130 @@ SEED_DEV long long unit_index(const DecodeParams& p, int u) {
   return ((long long)b * p.L + p.layer) * p.H + h;
 }
 
-// Lane 0: the bulk copies of unit u (c stored columns) into stage S, completing on
-// bar.  A unit with an invalid column count gets no copies (the wait still ends).
-template <int FORM, int DK, int DV, int MAXC>
-SEED_DEV void issue_unit(const DecodeParams& p, DecodeStage<FORM, DK, DV, MAXC>& S, uint64_t* bar,
-                         int u, int c, int m) {
-  constexpr bool KDA = FORM == SEED_KDA;
-  const long long unit = unit_index(p, u);
-  const int h = u % p.H;
-  const bool valid = c >= 0 && c < m;
-  uint32_t bytes = 0;
-  if (valid) {
-    bytes = (uint32_t)(c * (DK + DV) + 3 * DK + 2 * DV) * 4u;
-    bytes += KDA ? 2u * DK * 4u : (uint32_t)((c + 3) & ~3) * 4u;
-  }
-  mbar_arrive_expect_tx(bar, bytes);
-  if (!valid) return;
-  if (c > 0) {
-    bulk_g2s(S.U, p.U + unit * (long long)m * DK, (uint32_t)(c * DK * 4), bar);
-    bulk_g2s(S.V, p.V + unit * (long long)m * DV, (uint32_t)(c * DV * 4), bar);
-  }
-  bulk_g2s(S.a, p.a + unit * DK, DK * 4, bar);
-  bulk_g2s(S.k, p.k + (long long)u * DK, DK * 4, bar);
-  bulk_g2s(S.q, p.q + (long long)u * DK, DK * 4, bar);
-  bulk_g2s(S.v, p.v + (long long)u * DV, DV * 4, bar);
-  bulk_g2s(S.vb, p.vbar + ((long long)p.layer * p.H + h) * DV, DV * 4, bar);
-  if constexpr (KDA) {
-    bulk_g2s(S.al, p.alpha + (long long)u * DK, DK * 4, bar);
-    bulk_g2s(S.P, p.scale + unit * DK, DK * 4, bar);
-  } else if (c > 0) {
-    bulk_g2s(S.gam, p.scale + unit * p.slen, (uint32_t)((c + 3) & ~3) * 4u, bar);
-  }
-}
-
-template <int FORM, int DK, int DV, int MAXC, int NSW>
-struct WarpDecodeLayout {
-  using Stage = DecodeStage<FORM, DK, DV, MAXC>;
-  static constexpr int NCH = (MAXC + 31) / 32 * 4;   // coefficient pairs, in units of 8
-  static constexpr size_t OFF_BAR = NSW * sizeof(Stage);
-  static constexpr size_t OFF_DOT = OFF_BAR + 16 * ((NSW * 8 + 15) / 16);
-  static constexpr size_t bytes = OFF_DOT + 2 * NCH * 8 * sizeof(float);
+// The per-unit vectors one lane needs, in registers: its d_k / 32 rows of k, q, a
+// (KDA: alpha, P) and d_v / 32 rows of v, vbar; the decay scales of the columns
+// whose coefficients it forms (j = lane & 15 and 16 + (lane & 15); Mamba-2: j =
+// lane); and the unit's g (alpha) and beta.
+template <int FORM, int DK, int DV>
+struct UnitVecs {
+  static constexpr int PK = DK >= 32 ? DK / 32 : 1, PV = DV >= 32 ? DV / 32 : 1;
+  float k[PK], q[PK], a[PK], al[PK], P[PK], v[PV], vb[PV];
+  float gam_lo, gam_hi, g, be;
 };
 
-template <int FORM, int DK, int DV, int MAXC, int NSW>
+template <int FORM, int DK, int DV>
+SEED_DEV void load_vecs(const DecodeParams& p, int u, int c, UnitVecs<FORM, DK, DV>& r) {
+  constexpr bool KDA = FORM == SEED_KDA, M2 = FORM == SEED_MAMBA2;
+  constexpr int PK = UnitVecs<FORM, DK, DV>::PK, PV = UnitVecs<FORM, DK, DV>::PV;
+  const int lane = threadIdx.x & 31;
+  const long long unit = unit_index(p, u);
+  const int h = u % p.H;
+#pragma unroll
+  for (int e = 0; e < PK; ++e) r.k[e] = r.q[e] = r.a[e] = 0.f, r.al[e] = r.P[e] = 1.f;
+#pragma unroll
+  for (int e = 0; e < PV; ++e) r.v[e] = r.vb[e] = 0.f;
+  if (DK >= 32 || lane < DK) {
+    ldv<PK>(p.k + (long long)u * DK + lane * PK, r.k);
+    ldv<PK>(p.q + (long long)u * DK + lane * PK, r.q);
+    ldv<PK>(p.a + unit * DK + lane * PK, r.a);
+    if constexpr (KDA) {
+      ldv<PK>(p.alpha + (long long)u * DK + lane * PK, r.al);
+      ldv<PK>(p.scale + unit * DK + lane * PK, r.P);
+    }
+  }
+  if (DV >= 32 || lane < DV) {
+    ldv<PV>(p.v + (long long)u * DV + lane * PV, r.v);
+    ldv<PV>(p.vbar + ((long long)p.layer * p.H + h) * DV + lane * PV, r.vb);
+  }
+  r.gam_lo = r.gam_hi = 1.f;
+  if constexpr (!KDA) {
+    const int j0 = M2 ? lane : (lane & 15), j1 = 16 + (lane & 15);
+    if (j0 < c) r.gam_lo = p.scale[unit * p.slen + j0];
+    if (!M2 && j1 < c) r.gam_hi = p.scale[unit * p.slen + j1];
+  }
+  r.g = KDA ? 1.f : p.alpha[u];
+  r.be = p.beta[u];
+}
+
+// Lane 0: the bulk copies of the c stored columns of U and of V of unit u into the
+// stage (U at sU, V at sV), completing on bar.  A unit with an invalid column count
+// gets no copies (the wait still ends).
+template <int DK, int DV>
+SEED_DEV void issue_unit(const DecodeParams& p, float* sU, float* sV, uint64_t* bar, int u, int c, int m) {
+  const bool valid = c > 0 && c < m;
+  mbar_arrive_expect_tx(bar, valid ? (uint32_t)(c * (DK + DV)) * 4u : 0u);
+  if (!valid) return;
+  const long long unit = unit_index(p, u);
+  bulk_g2s(sU, p.U + unit * (long long)m * DK, (uint32_t)(c * DK * 4), bar);
+  bulk_g2s(sV, p.V + unit * (long long)m * DV, (uint32_t)(c * DV * 4), bar);
+}
+
+// Shared memory of one warp: the stage (U columns, then V columns, each sized for
+// the R + W - 1 columns a unit can hold before a step), the column coefficients and
+// the stage's mbarrier.
+__host__ __device__ constexpr size_t warp_stage_floats(int maxc, int dk, int dv) {
+  return (size_t)maxc * (dk + dv);
+}
+constexpr int kCoefFloats = 2 * 32;
+
+template <int FORM, int DK, int DV, int MAXC>
 __global__ void __launch_bounds__(32) decode_warp_kernel(const DecodeParams p) {
-  using Lay = WarpDecodeLayout<FORM, DK, DV, MAXC, NSW>;
-  using Stage = typename Lay::Stage;
+  using Vecs = UnitVecs<FORM, DK, DV>;
   constexpr bool KDA = FORM == SEED_KDA;
   constexpr bool M2 = FORM == SEED_MAMBA2;
-  constexpr int PK = DK >= 32 ? DK / 32 : 1;   // U rows per lane (d_k = 16: half the lanes)
-  constexpr int PV = DV >= 32 ? DV / 32 : 1;
+  constexpr int PK = Vecs::PK, PV = Vecs::PV;
   constexpr int CPS = M2 ? 32 : 16;            // columns per warp reduction
-  static_assert(NSW == 1 || NSW == 2, "one or two stages per warp");
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  Stage* stages = reinterpret_cast<Stage*>(smem_raw);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + Lay::OFF_BAR);
-  float* s_f = reinterpret_cast<float*>(smem_raw + Lay::OFF_DOT);   // [MAXC][2]
+  const int m = p.R + p.W;
+  const int maxc = m - 1;
+  float* sU = reinterpret_cast<float*>(smem_raw);
+  float* sV = sU + (size_t)maxc * DK;
+  float* s_f = sU + warp_stage_floats(maxc, DK, DV);   // [32][2] column coefficients (q, k)
+  uint64_t* full = reinterpret_cast<uint64_t*>(s_f + kCoefFloats);
 
   const int lane = threadIdx.x;
   const bool kact = DK >= 32 || lane < DK;
   const bool vact = DV >= 32 || lane < DV;
   const int n_units = p.B * p.H;
-  const int m = p.R + p.W;
   const int stride = gridDim.x;
   const int u0 = blockIdx.x;
   if (lane == 0) {
-    for (int s = 0; s < NSW; ++s) mbar_init(&full[s], 1);
+    mbar_init(full, 1);
     fence_mbar_init();
   }
   __syncwarp();
 
-  // prime the stages with the warp's first units
-  int c_s0 = 0, c_s1 = 0;
-#pragma unroll
-  for (int k = 0; k < NSW; ++k) {
-    const int u = u0 + k * stride;
-    const int c = u < n_units ? p.ncols[unit_index(p, u)] : 0;
-    if (k == 0) c_s0 = c;
-    else c_s1 = c;
-    if (lane == 0 && u < n_units) issue_unit<FORM, DK, DV, MAXC>(p, stages[k], &full[k], u, c, m);
-  }
-  int c_next = 0;   // column count of the unit that will refill the current stage
-  {
-    const int u = u0 + NSW * stride;
-    if (u < n_units) c_next = p.ncols[unit_index(p, u)];
-  }
-  // the scalars of the current unit, loaded one unit ahead
-  float g_cur = (KDA || u0 >= n_units) ? 1.f : p.alpha[u0];
-  float b_cur = u0 < n_units ? p.beta[u0] : 0.f;
+  // the first unit: its columns to the stage, its vectors to registers
+  int c = p.ncols[unit_index(p, u0)];
+  if (lane == 0) issue_unit<DK, DV>(p, sU, sV, full, u0, c, m);
+  Vecs cur, nxt;
+  load_vecs<FORM, DK, DV>(p, u0, c, cur);
+  int c_next = u0 + stride < n_units ? p.ncols[unit_index(p, u0 + stride)] : 0;
 
   for (int i = 0, u = u0; u < n_units; ++i, u += stride) {
-    const int s = NSW == 1 ? 0 : (i & 1);
-    const uint32_t ph = (uint32_t)(i / NSW) & 1u;
-    const int c = s == 0 ? c_s0 : c_s1;
     const long long unit = unit_index(p, u);
-    const float g = g_cur, be = b_cur;
-    const int u_next = u + NSW * stride;
-    const int u_after = u_next + stride;
-    const int c_after = u_after < n_units ? p.ncols[unit_index(p, u_after)] : 0;
-    if (u + stride < n_units) {
-      g_cur = KDA ? 1.f : p.alpha[u + stride];
-      b_cur = p.beta[u + stride];
-    }
+    const int u_next = u + stride;
+    // the next unit's vectors and the column count after it, while this one waits
+    if (u_next < n_units) load_vecs<FORM, DK, DV>(p, u_next, c_next, nxt);
+    const int c_after = u_next + stride < n_units ? p.ncols[unit_index(p, u_next + stride)] : 0;
+    const float g = cur.g, be = cur.be;
 
-    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full[s], ph, kWaitLimitNs))) {
+    if (!__all_sync(0xffffffffu, mbar_wait_bounded(full, (uint32_t)i & 1u, kWaitLimitNs))) {
       if (lane == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
-      for (int k = 0; k < NSW; ++k)   // let the copies in flight land before the block exits
-        mbar_wait_bounded(&full[(s + k) % NSW], (uint32_t)((i + k) / NSW) & 1u, kWaitLimitNs);
+      mbar_wait_bounded(full, (uint32_t)i & 1u, kWaitLimitNs);   // let the copies land before exit
       return;
     }
-    const Stage& S = stages[s];
     if (c < 0 || c >= m) {
       if (lane == 0) raise_flag(p.status, c == m ? SEED_FLAG_FULL : SEED_FLAG_BADCOLS);
     } else {
       // 1. dots of the stored U columns with q and k (KDA: with P+ (.) q and P+ (.) k,
       //    P+ = P (.) alpha, the dots of the decayed true columns)
-      float kr[PK], qr[PK], kk[PK], qq[PK], ar[PK], alr[PK], pr[PK];
-#pragma unroll
-      for (int e = 0; e < PK; ++e) kr[e] = qr[e] = ar[e] = 0.f, alr[e] = pr[e] = 1.f;
-      if (kact) {
-        ldv<PK>(S.k + lane * PK, kr);
-        ldv<PK>(S.q + lane * PK, qr);
-        ldv<PK>(S.a + lane * PK, ar);
-        if constexpr (KDA) {
-          ldv<PK>(S.al + lane * PK, alr);
-          ldv<PK>(S.P + lane * PK, pr);
-        }
-      }
+      float kk[PK], qq[PK];
 #pragma unroll
       for (int e = 0; e < PK; ++e) {
-        const float pp = KDA ? pr[e] * alr[e] : 1.f;
-        kk[e] = kr[e] * pp;
-        qq[e] = qr[e] * pp;
+        const float pp = KDA ? cur.P[e] * cur.al[e] : 1.f;
+        kk[e] = cur.k[e] * pp;
+        qq[e] = cur.q[e] * pp;
       }
       // 16 columns per reduction (32 for Mamba-2, which has no erase): lane l ends up
       // with dot number l; it turns it into the column's y coefficient
@@ -209,37 +204,30 @@ __global__ void __launch_bounds__(32) decode_warp_kernel(const DecodeParams p) {
           float ue[PK];
 #pragma unroll
           for (int e = 0; e < PK; ++e) ue[e] = 0.f;
-          if (j < c && kact) ldv<PK>(S.U + j * DK + lane * PK, ue);
+          if (j < c && kact) ldv<PK>(sU + j * DK + lane * PK, ue);
           dv[t] = dotv<PK>(ue, qq);
           if constexpr (!M2) dv[16 + t] = dotv<PK>(ue, kk);
         }
         const float tot = warp_xreduce<32>(dv);
         const int j = c0 + (M2 ? lane : (lane & 15));
         if (j < c) {
-          const float f = KDA ? 1.f : g * S.gam[j];
+          const float f = KDA ? 1.f : g * (c0 == 0 ? cur.gam_lo : cur.gam_hi);
           s_f[2 * j + (M2 ? 0 : (lane >> 4))] = f * tot;
         }
       }
       // 2. scalars: k^T a', a'^T q, k^T q (a' = alpha (.) a for KDA), v^T vbar, vbar^T vbar
-      float vr[PV], vbr[PV];
-#pragma unroll
-      for (int e = 0; e < PV; ++e) vr[e] = vbr[e] = 0.f;
-      if (vact) {
-        ldv<PV>(S.v + lane * PV, vr);
-        ldv<PV>(S.vb + lane * PV, vbr);
-      }
       float sc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int e = 0; e < PK; ++e) {
-        const float ae = KDA ? alr[e] * ar[e] : ar[e];
-        sc[0] = fmaf(kr[e], ae, sc[0]);
-        sc[1] = fmaf(ae, qr[e], sc[1]);
-        sc[2] = fmaf(kr[e], qr[e], sc[2]);
+        const float ae = KDA ? cur.al[e] * cur.a[e] : cur.a[e];
+        sc[0] = fmaf(cur.k[e], ae, sc[0]);
+        sc[1] = fmaf(ae, cur.q[e], sc[1]);
+        sc[2] = fmaf(cur.k[e], cur.q[e], sc[2]);
       }
 #pragma unroll
       for (int e = 0; e < PV; ++e) {
-        sc[3] = fmaf(vr[e], vbr[e], sc[3]);
-        sc[4] = fmaf(vbr[e], vbr[e], sc[4]);
+        sc[3] = fmaf(cur.v[e], cur.vb[e], sc[3]);
+        sc[4] = fmaf(cur.vb[e], cur.vb[e], sc[4]);
       }
       const float tot = warp_xreduce<8>(sc);   // lane 4 i holds scalar i
       const float ka = __shfl_sync(0xffffffffu, tot, 0);
@@ -262,7 +250,7 @@ __global__ void __launch_bounds__(32) decode_warp_kernel(const DecodeParams p) {
           float ve[PV];
 #pragma unroll
           for (int e = 0; e < PV; ++e) ve[e] = 0.f;
-          if (vact) ldv<PV>(S.V + j * DV + lane * PV, ve);
+          if (vact) ldv<PV>(sV + j * DV + lane * PV, ve);
           const float2 f2 = *reinterpret_cast<const float2*>(s_f + 2 * j);   // (q, k) coefficients
 #pragma unroll
           for (int e = 0; e < PV; ++e) {
@@ -281,9 +269,9 @@ __global__ void __launch_bounds__(32) decode_warp_kernel(const DecodeParams p) {
           float ncol[PV], oe[PV];
 #pragma unroll
           for (int e = 0; e < PV; ++e) {
-            const float eps = vr[e] - omega * vbr[e];
+            const float eps = cur.v[e] - omega * cur.vb[e];
             ncol[e] = M2 ? be * eps : be * (eps - yk[e]);
-            oe[e] = fmaf(vbr[e], apq, yq[e]) + ncol[e] * kq;
+            oe[e] = fmaf(cur.vb[e], apq, yq[e]) + ncol[e] * kq;
             bad |= !(isfinite(ncol[e]) && isfinite(oe[e]));
           }
           stv<PV>(p.V + unit * (long long)m * DV + (long long)c * DV + lane * PV, ncol);
@@ -294,13 +282,13 @@ __global__ void __launch_bounds__(32) decode_warp_kernel(const DecodeParams p) {
 #pragma unroll
           for (int e = 0; e < PK; ++e) {
             if constexpr (KDA) {
-              pn[e] = pr[e] * alr[e];
-              anew[e] = fmaf(alr[e], ar[e], coef * kr[e]);
-              unew[e] = kr[e] / pn[e];
+              pn[e] = cur.P[e] * cur.al[e];
+              anew[e] = fmaf(cur.al[e], cur.a[e], coef * cur.k[e]);
+              unew[e] = cur.k[e] / pn[e];
               bad |= !isfinite(unew[e]);
             } else {
-              anew[e] = fmaf(g, ar[e], coef * kr[e]);
-              unew[e] = kr[e];
+              anew[e] = fmaf(g, cur.a[e], coef * cur.k[e]);
+              unew[e] = cur.k[e];
             }
             bad |= !isfinite(anew[e]);
           }
@@ -309,56 +297,64 @@ __global__ void __launch_bounds__(32) decode_warp_kernel(const DecodeParams p) {
           if constexpr (KDA) stv<PK>(p.scale + unit * DK + lane * PK, pn);
         }
         if constexpr (!KDA) {
-          for (int j = lane; j <= c; j += 32) p.scale[unit * p.slen + j] = j < c ? g * S.gam[j] : 1.f;
+          // gamma_j of column j = lane: gam_lo for lanes < 16 (and every lane for
+          // Mamba-2), gam_hi above; the new column's scale is 1
+          const float gl = (M2 || lane < 16) ? cur.gam_lo : cur.gam_hi;
+          for (int j = lane; j <= c; j += 32) p.scale[unit * p.slen + j] = j < c ? g * gl : 1.f;
         }
         if (lane == 0) p.ncols[unit] = c + 1;
         if (__any_sync(0xffffffffu, bad) && lane == 0) raise_flag(p.status, SEED_FLAG_NONFINITE);
       }
     }
-    // every read of the stage (and of s_f) is above: refill the stage
-    fence_proxy_async_smem();
+    // every read of the stage (and of s_f) is above and complete (its values were
+    // consumed); only bulk copies write the stage, so no proxy fence is needed
     __syncwarp();
-    if (lane == 0 && u_next < n_units) issue_unit<FORM, DK, DV, MAXC>(p, stages[s], &full[s], u_next, c_next, m);
-    if (s == 0) c_s0 = c_next;
-    else c_s1 = c_next;
+    if (lane == 0 && u_next < n_units) issue_unit<DK, DV>(p, sU, sV, full, u_next, c_next, m);
+    cur = nxt;
+    c = c_next;
     c_next = c_after;
   }
 }
 
-template <int FORM, int DK, int DV, int MAXC, int NSW>
+template <int FORM, int DK, int DV, int MAXC>
 static int launch_warp_t(const DecodeParams& p, cudaStream_t st) {
-  using Lay = WarpDecodeLayout<FORM, DK, DV, MAXC, NSW>;
-  auto kern = decode_warp_kernel<FORM, DK, DV, MAXC, NSW>;
+  auto kern = decode_warp_kernel<FORM, DK, DV, MAXC>;
+  const int maxc = p.R + p.W - 1;
+  const size_t smem = warp_stage_floats(maxc, DK, DV) * sizeof(float) + kCoefFloats * sizeof(float) + 16;
+  // per device: the shared-memory opt-in (for the largest stage), and the resident
+  // blocks per SM for each stage size
   constexpr int kMaxDev = 64;
-  static int grid_per_sm[kMaxDev] = {0};
+  static bool attr_set[kMaxDev] = {false};
   static int sm_count[kMaxDev] = {0};
+  static int grid_per_sm[kMaxDev][MAXC + 1] = {};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return SEED_ERR_CUDA;
-  if (grid_per_sm[dev] == 0) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::bytes) !=
-        cudaSuccess)
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev || maxc > MAXC) return SEED_ERR_CUDA;
+  if (!attr_set[dev]) {
+    const size_t smax = warp_stage_floats(MAXC, DK, DV) * sizeof(float) + kCoefFloats * sizeof(float) + 16;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smax) != cudaSuccess)
       return SEED_ERR_CUDA;
-    int n = 0, sms = 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    if (cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return SEED_ERR_CUDA;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 32, Lay::bytes) != cudaSuccess)
-      return SEED_ERR_CUDA;
-    sm_count[dev] = sms;
-    grid_per_sm[dev] = n > 0 ? n : 1;
+    attr_set[dev] = true;
+  }
+  if (grid_per_sm[dev][maxc] == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 32, smem) != cudaSuccess) return SEED_ERR_CUDA;
+    grid_per_sm[dev][maxc] = n > 0 ? n : 1;
   }
   const int units = p.B * p.H;
-  int grid = grid_per_sm[dev] * sm_count[dev];
+  int grid = grid_per_sm[dev][maxc] * sm_count[dev];
   if (grid > units) grid = units;
-  kern<<<grid, 32, Lay::bytes, st>>>(p);
+  kern<<<grid, 32, smem, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? SEED_OK : SEED_ERR_CUDA;
 }
 
 template <int FORM, int DK, int DV>
 static int launch_warp_dims(const DecodeParams& p, cudaStream_t st) {
   const int maxc = p.R + p.W - 1;
-  if (maxc <= 8) return launch_warp_t<FORM, DK, DV, 8, 1>(p, st);
-  if (maxc <= 16) return launch_warp_t<FORM, DK, DV, 16, 1>(p, st);
-  return launch_warp_t<FORM, DK, DV, 32, 1>(p, st);
+  if (maxc <= 8) return launch_warp_t<FORM, DK, DV, 8>(p, st);
+  if (maxc <= 16) return launch_warp_t<FORM, DK, DV, 16>(p, st);
+  return launch_warp_t<FORM, DK, DV, 32>(p, st);
 }
 
 bool decode_warp_supported(const seed_dims& d) { return d.R + d.W - 1 <= 32; }
