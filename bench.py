@@ -40,7 +40,7 @@ NOMINAL_HBM_GBS = 8000.0
 # a full per-layer launch (256 requests x 48 heads) at c = 19 stored columns.  Set to None
 # whenever the decode kernel changes until it is measured again.
 NCU_DECODE_TRAFFIC = {"kernel": "decode_warp_kernel", "form": 0, "d_k": 128, "d_v": 128, "R": 16,
-                      "W": 16, "units": 12288, "c": 19, "bytes": 266.03e6 + 20.66e6}
+                      "W": 16, "units": 12288, "c": 19, "bytes": 266.031e6 + 19.914e6}
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -58,6 +58,9 @@ def parse_args(argv=None):
     ap.add_argument("--input-steps", type=int, default=48,
                     help="distinct pre-generated input steps, cycled (>= 3 W so that a key comes "
                          "back only after its old copy has decayed)")
+    ap.add_argument("--ragged", action="store_true",
+                    help="ragged compression schedules: requests joined at different times, a "
+                         "compression launch after every step compresses the units that are due")
     ap.add_argument("--dense-steps", type=int, default=8)
     ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -225,13 +228,17 @@ def cpu_oracle_rate(cfg, seconds: float, rank_seed: int = 0) -> dict:
             "affinity_cores": len(os.sched_getaffinity(0))}
 
 
-def config_obj(cfg, batch, world, prefill):
+def config_obj(cfg, batch, world, prefill, ragged=False):
+    schedule = ("ragged: request b joined W-1-floor(bW/B) steps before the others; a compression "
+                "launch after every step compresses the units that are due" if ragged else
+                "lockstep: every unit compresses after steps W, 2W, ...")
     return {"workload": f"{cfg.name}: {cfg.layers} GDN layers x {cfg.heads} heads, "
                         f"d_k=d_v={cfg.d_k}, R={cfg.R}, W={cfg.W}" if cfg.form == 0 else cfg.name,
             "form": {0: "gdn", 1: "kda", 2: "mamba2"}[cfg.form], "layers": cfg.layers,
             "heads": cfg.heads, "d_k": cfg.d_k, "d_v": cfg.d_v, "R": cfg.R, "W": cfg.W,
             "batch_per_gpu": batch, "global_batch": batch * world, "prefill_tokens": prefill,
             "parallelism": f"dp{world} (requests sharded, no collective)",
+            "schedule": schedule,
             "l2": "inputs and state larger than L2 (no flush needed)"}
 
 
@@ -317,10 +324,12 @@ def run_ours(args, world, rank, local):
     B = cfg.batch
     prefill = cfg.n_prefill if args.prefill is None else args.prefill
     run = DeviceRun(cfg, b0=shard(B, rank), device=str(dev), n_prefill=prefill,
-                    keep_dense=not args.no_dense)
+                    keep_dense=not args.no_dense and not args.ragged, ragged=args.ragged)
     d = run.dims
     t_setup = time.perf_counter()
     run.prefill_and_convert()
+    if args.ragged:
+        run.lead_in(S.alloc_step_inputs(d, dev))
     torch.cuda.synchronize()
     t_setup = time.perf_counter() - t_setup
 
@@ -351,13 +360,13 @@ def run_ours(args, world, rank, local):
             qq, kk, vv, aa, bb = inputs(t, l)
             if ev is not None:
                 ev["dec"].append((torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-                                  run.c))
+                                  roofline.mean_columns(d.R, d.W) if args.ragged else run.c))
                 ev["dec"][-1][0].record(stream)
             S.seed_decode_step(d, run.state, l, qq, kk, vv, aa, bb, o[l], run.ws, stream)
             if ev is not None:
                 ev["dec"][-1][1].record(stream)
         run.c += 1
-        if run.c == d.m:
+        if run.c == d.m or args.ragged:
             if ev is not None:
                 ev["cmp"].append((torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)))
                 ev["cmp"][-1][0].record(stream)
@@ -402,7 +411,7 @@ def run_ours(args, world, rank, local):
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded Philox4x32-10 inputs and prefill, generated on the device)",
-        "config": config_obj(cfg, B, world, prefill),
+        "config": config_obj(cfg, B, world, prefill, args.ragged),
         "roofline": {"bound": "hbm", "kernel": decode_kernel_name(d), "achieved": dec_gbs, "peak": peak,
                      "unit": "GB/s", "frac": dec_gbs / peak, "peak_source": f"{peak_kind} copy bandwidth",
                      "frac_of_nominal_8TBs": dec_gbs / NOMINAL_HBM_GBS,
@@ -466,34 +475,64 @@ def run_ours(args, world, rank, local):
         for t in range(Ph):
             hq[t].copy_(q[t]); hk[t].copy_(k[t]); hv[t].copy_(v[t]); ha[t].copy_(alpha[t]); hb[t].copy_(beta[t])
         ho = torch.empty(L, BH, d.d_v, dtype=torch.float32, pin_memory=True)
-        sq, sk, sv = torch.empty_like(q[0, 0]), torch.empty_like(k[0, 0]), torch.empty_like(v[0, 0])
-        sa, sb = torch.empty_like(alpha[0, 0]), torch.empty_like(beta[0, 0])
-        h2d = L * (sq.numel() + sk.numel() + sv.numel() + sa.numel() + sb.numel()) * 4   # as copied
+        # inputs copied in on their own stream into two alternating device buffers, each
+        # layer's o copied out on a third stream as soon as it is written, so that the
+        # transfers (host memory and PCIe bound) overlap the decode launches
+        nb = 2
+        bufs = [(torch.empty_like(q[0, 0]), torch.empty_like(k[0, 0]), torch.empty_like(v[0, 0]),
+                 torch.empty_like(alpha[0, 0]), torch.empty_like(beta[0, 0])) for _ in range(nb)]
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(nb)]
+        ev_free = [torch.cuda.Event() for _ in range(nb)]
+        ev_dec = [torch.cuda.Event() for _ in range(L)]
+        ev_out = [torch.cuda.Event() for _ in range(L)]
+        h2d = L * sum(x.numel() for x in bufs[0]) * 4   # as copied
         d2h = o.numel() * 4
         torch.cuda.synchronize()
         barrier(world, dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
+        s_in.wait_stream(stream)
+        s_out.wait_stream(stream)
+        n = 0
         for s in range(args.e2e_steps):
             t = s % Ph
             for l in range(L):
-                sq.copy_(hq[t, l], non_blocking=True); sk.copy_(hk[t, l], non_blocking=True)
-                sv.copy_(hv[t, l], non_blocking=True); sa.copy_(ha[t, l], non_blocking=True)
-                sb.copy_(hb[t, l], non_blocking=True)
-                S.seed_decode_step(d, run.state, l, sq, sk, sv, sa if kda else sa[:BH], sb[:BH], o[l],
+                bi = n % nb
+                bq, bk, bv, ba, bb = bufs[bi]
+                with torch.cuda.stream(s_in):
+                    if n >= nb:
+                        s_in.wait_event(ev_free[bi])
+                    bq.copy_(hq[t, l], non_blocking=True); bk.copy_(hk[t, l], non_blocking=True)
+                    bv.copy_(hv[t, l], non_blocking=True); ba.copy_(ha[t, l], non_blocking=True)
+                    bb.copy_(hb[t, l], non_blocking=True)
+                    ev_in[bi].record(s_in)
+                stream.wait_event(ev_in[bi])
+                if s > 0:
+                    stream.wait_event(ev_out[l])   # last step's o of this layer is out
+                S.seed_decode_step(d, run.state, l, bq, bk, bv, ba if kda else ba[:BH], bb[:BH], o[l],
                                    run.ws, stream)
+                ev_free[bi].record(stream)
+                ev_dec[l].record(stream)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(ev_dec[l])
+                    ho[l].copy_(o[l], non_blocking=True)
+                    ev_out[l].record(s_out)
+                n += 1
             run.c += 1
             if run.c == d.m:
                 S.seed_compress(d, run.state, S.SEED_ALL_LAYERS, run.ws, stream=stream)
                 run.c = d.R
-            ho.copy_(o, non_blocking=True)
+        stream.wait_stream(s_out)
+        stream.wait_stream(s_in)
         e1.record(stream)
         torch.cuda.synchronize()
         barrier(world, dev)
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         line["e2e"] = {"value": args.e2e_steps * units * world / (e2e_ms / 1e3), "unit": UNIT,
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                       "note": "pinned host buffers; every step copies its inputs in and its o out"}
+                       "note": "pinned host buffers; every step copies its inputs in and its o out "
+                               "(copies on their own streams, overlapping the decode launches)"}
         line["status_flags"] |= S.seed_get_status(run.ws)
 
     if rank == 0 and world == 1 and not args.no_cpu:
