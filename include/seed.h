@@ -181,6 +181,21 @@ int seed_state_to_dense(const seed_dims* dims, const seed_state* state, int32_t 
                         const int32_t* units, int32_t n_units, float* S_out, void* ws,
                         size_t ws_bytes, void* stream);
 
+/* Energies of the stored states (SEED figures & tables, Figure 3 (f)-(g): the sink
+ * holds most of a state's energy; Figure 12 (f): the content energy beyond rank R).
+ * For the listed units of `layer` (or all layers; units and n_units as in
+ * seed_state_to_dense, NULL = every unit in scope), out[n][4] (float32) receives
+ *     [0] ||a vbar^T||_F^2   [1] ||U V^T||_F^2 (true U)   [2] 2 <a vbar^T, U V^T>_F
+ *     [3] ||S||_F^2 = [0] + [1] + [2]
+ * The sink's share of the state's energy is [0] / [3]; the content C = S - a vbar^T
+ * has energy [1] + [2] (the cross term vanishes up to rounding: every update keeps
+ * V^T vbar = 0), so with the kept singular values sigma_1..R of the content (returned
+ * by the conversion and the compression) the energy beyond rank R is
+ * [1] + [2] - sum sigma_i^2.  Reads the state only.                                  */
+int seed_state_energy(const seed_dims* dims, const seed_state* state, int32_t layer,
+                      const int32_t* units, int32_t n_units, float* out, void* ws, size_t ws_bytes,
+                      void* stream);
+
 /* The dense-state step that SEED replaces, kept as the in-run comparison: every
  * decode step loads and stores whole recurrent states (SEED abstract, readsearch.ai).
  * One step of `layer` on a dense state S [B][L][H][d_k][d_v] with the form's dense

@@ -40,6 +40,8 @@ typedef struct {
 
 #define SEED_PHASE_PREFILL 0
 #define SEED_PHASE_DECODE 1
+#define SEED_PHASE_LEADIN 2   /* decode steps a request took before the others joined it
+                                 (ragged compression schedules); t counts them from 0 */
 
 /* vbar [L][H][d_v] for every head. */
 int seed_synth_vbar(const seed_dims* dims, seed_synth_key key, float* vbar, void* stream);

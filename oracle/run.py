@@ -8,7 +8,8 @@ Per unit (request b, layer l, head h), following SEED figures & tables
      appends one column pair,
   4. after the step that brings the column count to R + W, the factors are
      compressed back to rank R (``compress.truncate_qr_core``): with decode steps
-     counted from 1 this is after steps W, 2W, 3W, ... ("every W steps").
+     counted from 1 this is after steps W, 2W, 3W, ... ("every W steps"); a
+     request that joined j steps earlier (ragged schedules) is j steps ahead.
 An open-loop dense shadow S_t^exact runs the dense recurrence on the same inputs
 from the uncompressed prefill state, for Lemma 1 and Corollary 4 checks.
 """
@@ -22,8 +23,12 @@ from workloads import philox
 from . import compress, convert, factored, recurrences
 
 
-def run_units(cfg, b, l, h, n_prefill=None, n_decode=None, keep_shadow=True):
+def run_units(cfg, b, l, h, n_prefill=None, n_decode=None, keep_shadow=True, lead_in=0):
     """Run the sampled units (1-D arrays b, l, h) and return a dict of trajectories.
+
+    With lead_in = j > 0 the units first take j lead-in decode steps (inputs of
+    philox.PHASE_LEADIN, t = 0 .. j-1, outputs not kept), as a request that joined
+    the batch j steps before the others; the trajectories below start after them.
 
     Keys: o (T, n, d_v); a_t (T, n, d_k); ncols (T,) after each step;
     comp_steps (list of 1-based steps after which a compression ran);
@@ -34,6 +39,8 @@ def run_units(cfg, b, l, h, n_prefill=None, n_decode=None, keep_shadow=True):
     and, with keep_shadow, S_exact (final open-loop dense state),
     err_open (T, n) ||S~_t - S_t^exact||_F and sink_dev (T, n) max |a_t - sink(S_t^exact)|.
     """
+    if not 0 <= lead_in < cfg.W:
+        raise ValueError("lead_in must lie in [0, W)")
     b, l, h = (np.atleast_1d(np.asarray(x, dtype=np.int64)) for x in (b, l, h))
     T = cfg.n_decode if n_decode is None else n_decode
     S0 = recurrences.dense_prefill(cfg, b, l, h, n_prefill)
@@ -46,6 +53,17 @@ def run_units(cfg, b, l, h, n_prefill=None, n_decode=None, keep_shadow=True):
     o_all, a_all, ncols_all, sig, gaps, comp_steps = [], [], [], [], [], []
     err_open, sink_dev = [], []
     ncols = cfg.R
+    # ragged schedules: a request that joined `lead_in` steps before the others has
+    # taken that many decode steps (inputs of the lead-in phase) before step 0, so
+    # it holds R + lead_in columns and compresses after steps W - lead_in, 2W - lead_in, ...
+    for j in range(lead_in):
+        inp = recurrences.f64(philox.token_inputs(cfg, b, l, h, j, philox.PHASE_LEADIN))
+        a, U, V, _ = factored.step(cfg.form, a, U, V, vb, inp["q"], inp["k"], inp["v"],
+                                   inp["alpha"], inp["beta"])
+        ncols += 1
+        if keep_shadow:
+            S_exact = recurrences.dense_step(cfg.form, S_exact, inp["k"], inp["v"],
+                                             inp["alpha"], inp["beta"])
     for t in range(T):
         inp = recurrences.f64(philox.token_inputs(cfg, b, l, h, t, philox.PHASE_DECODE))
         a, U, V, o = factored.step(cfg.form, a, U, V, vb, inp["q"], inp["k"], inp["v"],

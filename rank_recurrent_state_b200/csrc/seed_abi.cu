@@ -144,6 +144,26 @@ int seed_state_to_dense(const seed_dims* dims, const seed_state* state, int32_t 
                                as_stream(stream));
 }
 
+int seed_state_energy(const seed_dims* dims, const seed_state* state, int32_t layer,
+                      const int32_t* units, int32_t n_units, float* out, void* ws, size_t ws_bytes,
+                      void* stream) {
+  SEED_TRY(check_dims(dims));
+  SEED_TRY(check_layer(dims, layer, true));
+  SEED_TRY(check_state(state));
+  SEED_TRY(check_ptr(out));
+  SEED_TRY(check_ws(ws, ws_bytes));
+  const long long scope = (long long)dims->batch * dims->heads * (layer < 0 ? dims->layers : 1);
+  if (units) {
+    if (n_units < 0 || n_units > scope) return SEED_ERR_INVALID_ARG;
+    if (n_units == 0) return SEED_OK;
+    SEED_TRY(check_ptr(units));
+  } else {
+    n_units = (int32_t)scope;
+  }
+  return seed::launch_state_energy(*dims, *state, layer, units, n_units, out, status_word(ws),
+                                   as_stream(stream));
+}
+
 int seed_dense_step(const seed_dims* dims, float* S, int32_t layer, const float* q, const float* k,
                     const float* v, const float* alpha, const float* beta, float* o, void* ws,
                     size_t ws_bytes, void* stream) {
@@ -212,7 +232,8 @@ int seed_synth_token_inputs(const seed_dims* dims, seed_synth_key key, int32_t p
                             float* alpha, float* beta, void* stream) {
   SEED_TRY(check_dims(dims));
   SEED_TRY(check_layer(dims, layer, false));
-  if (phase != SEED_PHASE_PREFILL && phase != SEED_PHASE_DECODE) return SEED_ERR_INVALID_ARG;
+  if (phase != SEED_PHASE_PREFILL && phase != SEED_PHASE_DECODE && phase != SEED_PHASE_LEADIN)
+    return SEED_ERR_INVALID_ARG;
   if (t < 0 || key.b0 < 0) return SEED_ERR_INVALID_ARG;
   SEED_TRY(check_ptr(vbar));
   SEED_TRY(check_opt_ptr(q));

@@ -35,6 +35,9 @@ int launch_init_from_dense(const seed_dims& d, const seed_state& s, int layer, c
 int launch_to_dense(const seed_dims& d, const seed_state& s, int layer, const int32_t* units,
                     int n_units, float* S_out, uint32_t* status, cudaStream_t st);
 
+int launch_state_energy(const seed_dims& d, const seed_state& s, int layer, const int32_t* units,
+                        int n_units, float* out, uint32_t* status, cudaStream_t st);
+
 int launch_dense_step(const seed_dims& d, float* S, int layer, const float* q, const float* k,
                       const float* v, const float* alpha, const float* beta, float* o,
                       uint32_t* status, cudaStream_t st);

@@ -2,7 +2,9 @@
 
 prefill (synthetic, dense) -> seed_state_init_from_dense -> per step and layer:
 seed_synth_token_inputs + seed_decode_step, and seed_compress after the step that
-fills R + W columns ("every W steps", decode steps counted from 1).
+fills R + W columns ("every W steps", decode steps counted from 1).  With ragged
+schedules the requests joined at different times (a lead-in of up to W - 1 steps)
+and seed_compress runs after every step, compressing the units that are due.
 
 Every step of the path runs in libseed's kernels; this module only allocates
 tensors, orders the calls and tracks the (uniform) column count on the host.
@@ -19,7 +21,7 @@ class DeviceRun:
     """One workload resident on the device: v̄, the stored state and a workspace."""
 
     def __init__(self, cfg, batch: int | None = None, b0: int = 0, device: str = "cuda",
-                 n_prefill: int | None = None, keep_dense: bool = False):
+                 n_prefill: int | None = None, keep_dense: bool = False, ragged: bool = False):
         self.cfg = cfg
         self.dims = S.Dims.from_config(cfg, batch)
         self.key = S.synth_key(cfg, b0)
@@ -35,6 +37,12 @@ class DeviceRun:
         self.c = 0
         self.t = 0
         self.keep_dense = keep_dense
+        # ragged schedules: request b (global index) joined phi_b steps before the
+        # others, phi_b = W - 1 - floor(b W / B) for the workload's B requests, so the
+        # requests still in their lead-in at lead-in step j are a prefix of the batch
+        self.ragged = ragged
+        gb = torch.arange(b0, b0 + self.dims.batch)
+        self.phase = (cfg.W - 1 - (gb * cfg.W) // cfg.batch).clamp(min=0) if ragged else torch.zeros_like(gb)
 
     # ------------------------------------------------------------------ setup
     def prefill_and_convert(self, layer_chunk: int | None = None) -> None:
@@ -57,6 +65,22 @@ class DeviceRun:
         self.c = d.R
         self.t = 0
 
+    def lead_in(self, buf: dict) -> None:
+        """Ragged schedules: request b takes phi_b decode steps (lead-in inputs, t = 0 ..
+        phi_b - 1) before step 0, launched over the batch prefix still leading in."""
+        d = self.dims
+        for j in range(self.cfg.W - 1):
+            nb = int((self.phase > j).sum())
+            if nb == 0:
+                break
+            dj = S.Dims(d.form, nb, d.layers, d.heads, d.d_k, d.d_v, d.R, d.W)
+            bj = {k: (None if x is None else x[:nb]) for k, x in buf.items()}
+            for l in range(d.layers):
+                S.seed_synth_token_inputs(dj, self.key, S.SEED_PHASE_LEADIN, j, l, self.vbar,
+                                          bj["q"], bj["k"], bj["v"], bj["alpha"], bj["beta"])
+                S.seed_decode_step(dj, self.state, l, bj["q"], bj["k"], bj["v"], bj["alpha"], bj["beta"],
+                                   bj["o"], self.ws)
+
     # ------------------------------------------------------------------ decode
     def gen_inputs(self, t: int, layer: int, buf: dict) -> None:
         S.seed_synth_token_inputs(self.dims, self.key, S.SEED_PHASE_DECODE, t, layer, self.vbar,
@@ -78,6 +102,9 @@ class DeviceRun:
                 outs[l] = buf["o"].clone()
         self.c += 1
         self.t += 1
+        if self.ragged:   # some request is due after every step: only its units compress
+            S.seed_compress(d, self.state, S.SEED_ALL_LAYERS, self.ws, sigma_out=sigma)
+            return True
         if self.c == d.m:
             S.seed_compress(d, self.state, S.SEED_ALL_LAYERS, self.ws, sigma_out=sigma)
             self.c = d.R

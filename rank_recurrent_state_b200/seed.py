@@ -18,7 +18,7 @@ from . import _lib
 
 SEED_GDN, SEED_KDA, SEED_MAMBA2 = 0, 1, 2
 SEED_ALL_LAYERS = -1
-SEED_PHASE_PREFILL, SEED_PHASE_DECODE = 0, 1
+SEED_PHASE_PREFILL, SEED_PHASE_DECODE, SEED_PHASE_LEADIN = 0, 1, 2
 SEED_MAX_COLS = 96
 
 FLAG_FULL = 0x1
@@ -191,6 +191,16 @@ def seed_state_to_dense(dims: Dims, state: State, layer: int, S_out: torch.Tenso
     n = 0 if units is None else int(units.numel())
     _check("seed_state_to_dense", _lib.load().seed_state_to_dense(
         ctypes.byref(d), ctypes.byref(s), layer, _ptr(units), n, _ptr(S_out), ws.ptr, ws.nbytes,
+        _stream(stream)))
+
+
+def seed_state_energy(dims: Dims, state: State, layer: int, out: torch.Tensor, ws: Workspace,
+                      units: torch.Tensor | None = None, stream=None) -> None:
+    """out [n][4]: sink energy, content energy, cross term, total (see seed.h)."""
+    d, s = dims.c(), state.c()
+    n = 0 if units is None else int(units.numel())
+    _check("seed_state_energy", _lib.load().seed_state_energy(
+        ctypes.byref(d), ctypes.byref(s), layer, _ptr(units), n, _ptr(out), ws.ptr, ws.nbytes,
         _stream(stream)))
 
 

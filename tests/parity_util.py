@@ -65,6 +65,56 @@ def run_device(cfg, sample_units, n_prefill, n_decode, batch=None):
                 b=b, l=l, h=h)
 
 
+def run_device_ragged(cfg, sample_units, n_prefill, n_decode, batch=None):
+    """Like run_device, with ragged compression schedules: requests joined the batch at
+    different times (DeviceRun's lead-in) and every step ends with a compression of the
+    units that are due.  Returns the trajectories of the sampled units plus, per unit,
+    its lead-in length ``phase``; ``comp_steps`` and ``sigma`` are per unit (lists)."""
+    import torch
+    from rank_recurrent_state_b200 import seed as S
+    from rank_recurrent_state_b200.pipeline import DeviceRun
+
+    run = DeviceRun(cfg, batch=batch, n_prefill=n_prefill, ragged=True)
+    d = run.dims
+    run.prefill_and_convert()
+    su = np.asarray(sample_units, dtype=np.int64)
+    b, rem = np.divmod(su, d.layers * d.heads)
+    l, h = np.divmod(rem, d.heads)
+    units_t = torch.as_tensor(su, dtype=torch.int32, device=run.device)
+    conv = run.sigma_conv.reshape(-1, d.R)[units_t.long()].cpu().numpy()
+    S0 = run.to_dense(units_t).cpu().numpy()
+    buf = S.alloc_step_inputs(d, run.device)
+    run.lead_in(buf)
+    outs = [None] * d.layers
+    sig = torch.zeros(d.units, d.R, dtype=torch.float32, device=run.device)
+    o_traj, ncols_traj, sig_traj = [], [], []
+    for t in range(n_decode):
+        run.step(buf, outs=outs, sigma=sig)
+        o_traj.append(np.stack([outs[li][bi, hi].cpu().numpy() for bi, li, hi in zip(b, l, h)]))
+        ncols_traj.append(run.state.ncols.reshape(-1)[units_t.long()].cpu().numpy())
+        sig_traj.append(sig[units_t.long()].cpu().numpy())
+    torch.cuda.synchronize()
+    ncols = np.array(ncols_traj)
+    comp = [[t + 1 for t in range(n_decode) if ncols[t, u] == cfg.R] for u in range(su.size)]
+    sigma = [np.array([sig_traj[t - 1][u] for t in comp[u]]) for u in range(su.size)]
+    return dict(o=np.array(o_traj), ncols=ncols, comp_steps=comp, sigma=sigma,
+                S=run.to_dense(units_t).cpu().numpy(),
+                a=run.state.a.reshape(-1, d.d_k)[units_t.long()].cpu().numpy(), S_conv=S0,
+                conv_sigma=conv, flags=run.status(), b=b, l=l, h=h,
+                phase=run.phase[torch.as_tensor(b)].cpu().numpy())
+
+
+def ragged_group(dev, idx):
+    """The device trajectories of the sampled units idx (one lead-in length), in the
+    layout compare() takes."""
+    comp = dev["comp_steps"][idx[0]]
+    assert all(dev["comp_steps"][u] == comp for u in idx)
+    sig = np.stack([dev["sigma"][u] for u in idx], axis=1) if comp else np.zeros((0, len(idx), 0))
+    return dict(o=dev["o"][:, idx], ncols=dev["ncols"][:, idx], comp_steps=comp, sigma=sig, S=dev["S"][idx],
+                a=dev["a"][idx], S_conv=dev["S_conv"][idx], conv_sigma=dev["conv_sigma"][idx],
+                flags=dev["flags"], b=dev["b"][idx], l=dev["l"][idx], h=dev["h"][idx])
+
+
 def run_oracle(cfg, dev, n_prefill, n_decode):
     from oracle import run as orun
     return orun.run_units(cfg, dev["b"], dev["l"], dev["h"], n_prefill=n_prefill, n_decode=n_decode,

@@ -121,7 +121,7 @@ def test_other_entry_points_validate(lib):
     assert lib.seed_get_status(None, None, ctypes.byref(flags)) == -5
     assert lib.seed_get_status(A, None, None) == -1
     key = _lib.seed_synth_key(0, 0, 0, 0)
-    assert lib.seed_synth_token_inputs(ctypes.byref(d), key, 2, 0, 0, A, A, A, A, A, A, None) == -1
+    assert lib.seed_synth_token_inputs(ctypes.byref(d), key, 3, 0, 0, A, A, A, A, A, A, None) == -1
     assert lib.seed_synth_dense_prefill(ctypes.byref(d), key, -1, 0, A, A, None) == -1
     bad_key = _lib.seed_synth_key(0, 0, 0, -1)
     assert lib.seed_synth_dense_prefill(ctypes.byref(d), bad_key, 4, 0, A, A, None) == -1

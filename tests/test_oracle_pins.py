@@ -300,6 +300,30 @@ def test_compression_schedule_every_w_steps(tiny_run):
     np.testing.assert_array_equal(r["ncols"], expect)
 
 
+@pytest.mark.parametrize("lead_in", [1, 3])
+def test_ragged_schedule_lead_in(lead_in):
+    """A request that joined j steps earlier holds R + j columns at step 0 and compresses
+    after steps W - j, 2W - j, ...; Lemma 1 and Corollary 4 still hold over its whole run
+    (the lead-in steps included), and its lead-in inputs differ from its decode inputs."""
+    cfg = config(0)
+    r = run.run_units(cfg, [0, 0], [0, 0], [0, 1], lead_in=lead_in)
+    assert r["comp_steps"] == list(range(cfg.W - lead_in, cfg.n_decode + 1, cfg.W))
+    expect = [cfg.R + ((t + 1 + lead_in) % cfg.W) for t in range(cfg.n_decode)]
+    np.testing.assert_array_equal(r["ncols"], expect)
+    assert np.max(r["sink_dev"]) < 1e-12 * max(1.0, np.max(np.abs(r["a_t"])))
+    inp = philox.token_inputs(cfg, 0, 0, np.array([0, 1])[:, None], np.arange(cfg.n_decode)[None, :],
+                              philox.PHASE_DECODE)
+    lead = philox.token_inputs(cfg, 0, 0, np.array([0, 1])[:, None], np.arange(lead_in)[None, :],
+                               philox.PHASE_LEADIN)
+    g_bar = max(float(np.max(inp["alpha"])), float(np.max(lead["alpha"])))
+    bound = np.max(r["tail"], axis=0) / (1.0 - g_bar ** cfg.W)
+    assert np.all(np.max(r["err_open"], axis=0) <= bound)
+    assert not np.allclose(lead["k"][:, 0], inp["k"][:, 0])
+    # without lead-in the same call is the lockstep schedule
+    r0 = run.run_units(cfg, [0, 0], [0, 0], [0, 1], lead_in=0)
+    assert r0["comp_steps"] == list(range(cfg.W, cfg.n_decode + 1, cfg.W))
+
+
 def test_lemma1_sink_is_exact_across_compressions(tiny_run):
     """a_t equals the sink coefficient of the never-compressed dense state at every step."""
     _, r = tiny_run

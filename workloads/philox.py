@@ -14,8 +14,9 @@ regenerated independently on the host and on the device:
 
 ``block`` indexes the group of four 32-bit words inside one field vector,
 ``field`` names the quantity (q, k, v, alpha, beta, v̄ ...), ``phase`` is 0 for
-prefill tokens and 1 for decode steps, ``t`` is the token index inside the
-phase, and ``unit`` is the global unit index ((b * L) + l) * H + h (per-head
+prefill tokens, 1 for decode steps and 2 for the lead-in steps of a request that
+joined the batch earlier (ragged compression schedules), ``t`` is the token index
+inside the phase, and ``unit`` is the global unit index ((b * L) + l) * H + h (per-head
 quantities use l * H + h with t = 0).
 
 Transforms, all evaluated in float64 and rounded to float32 once at the end:
@@ -46,7 +47,7 @@ _SH = np.uint64(32)
 # field ids (low byte of counter word 1)
 F_Q, F_K, F_V, F_ALPHA, F_BETA = 0, 1, 2, 3, 4
 F_VBAR_DIR, F_VBAR_NORM, F_A = 8, 9, 10
-PHASE_PREFILL, PHASE_DECODE = 0, 1
+PHASE_PREFILL, PHASE_DECODE, PHASE_LEADIN = 0, 1, 2
 
 _TWO_PI = 2.0 * np.pi
 _U_SCALE = 2.0 ** -32
