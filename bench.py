@@ -58,6 +58,8 @@ def parse_args(argv=None):
     ap.add_argument("--input-steps", type=int, default=48,
                     help="distinct pre-generated input steps, cycled (>= 3 W so that a key comes "
                          "back only after its old copy has decayed)")
+    ap.add_argument("--factors", default="f32", choices=["f32", "f16", "bf16"],
+                    help="storage format of the factors U and V (arithmetic stays f32)")
     ap.add_argument("--ragged", action="store_true",
                     help="ragged compression schedules: requests joined at different times, a "
                          "compression launch after every step compresses the units that are due")
@@ -228,7 +230,7 @@ def cpu_oracle_rate(cfg, seconds: float, rank_seed: int = 0) -> dict:
             "affinity_cores": len(os.sched_getaffinity(0))}
 
 
-def config_obj(cfg, batch, world, prefill, ragged=False):
+def config_obj(cfg, batch, world, prefill, ragged=False, factors="f32"):
     schedule = ("ragged: request b joined W-1-floor(bW/B) steps before the others; a compression "
                 "launch after every step compresses the units that are due" if ragged else
                 "lockstep: every unit compresses after steps W, 2W, ...")
@@ -239,6 +241,8 @@ def config_obj(cfg, batch, world, prefill, ragged=False):
             "batch_per_gpu": batch, "global_batch": batch * world, "prefill_tokens": prefill,
             "parallelism": f"dp{world} (requests sharded, no collective)",
             "schedule": schedule,
+            "factors": factors + (" (U and V stored in 16 bits, rounded to nearest when written)"
+                                  if factors != "f32" else ""),
             "l2": "inputs and state larger than L2 (no flush needed)"}
 
 
@@ -278,8 +282,8 @@ def decode_traffic(d, units, cbar):
     capture does not match this kernel and shape."""
     from rank_recurrent_state_b200 import roofline
     t = NCU_DECODE_TRAFFIC
-    if t is None or decode_kernel_name(d) != t["kernel"] or (d.form, d.d_k, d.d_v, d.R, d.W) != (
-            t["form"], t["d_k"], t["d_v"], t["R"], t["W"]):
+    if t is None or decode_kernel_name(d) != t["kernel"] or (d.form, d.d_k, d.d_v, d.R, d.W, d.factors) != (
+            t["form"], t["d_k"], t["d_v"], t["R"], t["W"], t.get("factors", 0)):
         return None
     per = lambda c: roofline.lazy_bytes(d.form, d.d_k, d.d_v, c) + roofline.io_bytes(d.form, d.d_k, d.d_v)  # noqa: E731
     return t["bytes"] / t["units"] * units * per(cbar) / per(t["c"])
@@ -324,8 +328,10 @@ def run_ours(args, world, rank, local):
     B = cfg.batch
     prefill = cfg.n_prefill if args.prefill is None else args.prefill
     run = DeviceRun(cfg, b0=shard(B, rank), device=str(dev), n_prefill=prefill,
-                    keep_dense=not args.no_dense and not args.ragged, ragged=args.ragged)
+                    keep_dense=not args.no_dense and not args.ragged, ragged=args.ragged,
+                    factors=S.FACTOR_NAMES[args.factors])
     d = run.dims
+    fb = 4 if args.factors == "f32" else 2   # bytes per stored U / V value
     t_setup = time.perf_counter()
     run.prefill_and_convert()
     if args.ragged:
@@ -400,7 +406,7 @@ def run_ours(args, world, rank, local):
     units = d.units
     value = args.steps * units * world / (elapsed_ms / 1e3)
     dec_ms = [a.elapsed_time(b) for a, b, _ in ev["dec"]]
-    dec_bytes = [BH * roofline.lazy_bytes(d.form, d.d_k, d.d_v, c) for _, _, c in ev["dec"]]
+    dec_bytes = [BH * roofline.lazy_bytes(d.form, d.d_k, d.d_v, c, fb) for _, _, c in ev["dec"]]
     cmp_ms = [a.elapsed_time(b) for a, b in ev["cmp"]]
     dec_gbs = sum(dec_bytes) / (sum(dec_ms) / 1e3) / 1e9
     peak, peak_kind = measured_peak_hbm()
@@ -411,12 +417,12 @@ def run_ours(args, world, rank, local):
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded Philox4x32-10 inputs and prefill, generated on the device)",
-        "config": config_obj(cfg, B, world, prefill, args.ragged),
+        "config": config_obj(cfg, B, world, prefill, args.ragged, args.factors),
         "roofline": {"bound": "hbm", "kernel": decode_kernel_name(d), "achieved": dec_gbs, "peak": peak,
                      "unit": "GB/s", "frac": dec_gbs / peak, "peak_source": f"{peak_kind} copy bandwidth",
                      "frac_of_nominal_8TBs": dec_gbs / NOMINAL_HBM_GBS,
                      "traffic": decode_traffic(d, BH, cbar),
-                     "algorithmic_bytes_per_head_step_mean": roofline.lazy_bytes(d.form, d.d_k, d.d_v, cbar),
+                     "algorithmic_bytes_per_head_step_mean": roofline.lazy_bytes(d.form, d.d_k, d.d_v, cbar, fb),
                      "avg_launch_us": 1e3 * sum(dec_ms) / len(dec_ms), "launches": len(dec_ms)},
         "decode_only": {"head_steps_per_s": len(dec_ms) * BH * world / (sum(dec_ms) / 1e3),
                         "GBps": dec_gbs},
@@ -458,8 +464,9 @@ def run_ours(args, world, rank, local):
         line["speedup_vs_dense"] = {
             "decode_only": line["decode_only"]["head_steps_per_s"] / line["dense"]["head_steps_per_s"],
             "with_compress": value / line["dense"]["head_steps_per_s"],
-            "byte_ratio_lazy": roofline.dense_bytes(d.d_k, d.d_v) / roofline.lazy_bytes(d.form, d.d_k, d.d_v, cbar),
-            "byte_ratio_explicit": roofline.dense_bytes(d.d_k, d.d_v) / roofline.explicit_bytes(d.d_k, d.d_v, cbar)}
+            "byte_ratio_lazy": roofline.dense_bytes(d.d_k, d.d_v) / roofline.lazy_bytes(d.form, d.d_k, d.d_v, cbar, fb),
+            "byte_ratio_explicit": roofline.dense_bytes(d.d_k, d.d_v) / roofline.explicit_bytes(d.d_k, d.d_v, cbar,
+                                                                                                 fb)}
         del run.dense
         run.dense = None
         torch.cuda.empty_cache()

@@ -29,7 +29,8 @@
  *    caller's workspace; kernels never trap.  Read them with seed_get_status.
  *  - Units: one unit is one (request b, layer l, head h).  State arrays are
  *    request-major: unit index u = ((b * layers) + l) * heads + h.
- *  - Precision: float32 storage and arithmetic throughout.
+ *  - Precision: float32 arithmetic throughout; float32 storage, except that the
+ *    content factors U and V may be stored in 16 bits (seed_dims.factors).
  */
 #ifndef SEED_H_
 #define SEED_H_
@@ -78,6 +79,19 @@ typedef enum {
 #define SEED_MAX_COLS 96
 #define SEED_ALL_LAYERS (-1)
 
+/* Storage format of the content factors U and V (seed_dims.factors).  The SEED
+ * figures & tables page, Table 9 (and Table 4's 16-bit rows), keeps the shallow
+ * state's factors in fp16 or bf16, rounded when a compression writes them, with the
+ * same drift as fp32; the SEED summary's key points add that fp16 factors halve the
+ * state's bytes again.  Here every value written to U or V -- a conversion's or a
+ * compression's result and every appended column pair -- is rounded to the nearest
+ * value of the format, ties to even; all arithmetic stays float32, and the sink a,
+ * the scales and the column counts stay float32 / int32.  A 16-bit factor array
+ * holds 2-byte elements in the layout below (pointers still 16-byte aligned).
+ * A value beyond the format's range is stored as +-inf and raises
+ * SEED_FLAG_NONFINITE (fp16's largest finite value is 65504).                      */
+typedef enum { SEED_FACTORS_F32 = 0, SEED_FACTORS_F16 = 1, SEED_FACTORS_BF16 = 2 } seed_factors;
+
 /* Problem dimensions: batch of requests x layers x heads, head dims, rank, window. */
 typedef struct {
   int32_t form;   /* seed_form */
@@ -88,11 +102,13 @@ typedef struct {
   int32_t d_v;    /* value dimension */
   int32_t R;      /* rank kept after a compression */
   int32_t W;      /* steps between compressions; a unit holds at most R + W columns */
+  int32_t factors; /* seed_factors: element type of U and V (0 = float32)          */
 } seed_dims;
 
 /* The stored state of all B x L x H units (device pointers, caller-owned).
  *   a      [B][L][H][d_k]            sink coefficient a
- *   U      [B][L][H][R+W][d_k]       content factor U, one contiguous d_k column per slot;
+ *   U      [B][L][H][R+W][d_k]       content factor U (element type: dims->factors), one
+ *                                    contiguous d_k column per slot;
  *                                    slot j holds column j, so appends never move data
  *   V      [B][L][H][R+W][d_v]       content factor V, same slots
  *   scale  GDN, Mamba-2: [B][L][H][ceil4(R+W)] per-column scales gamma_j: the true
@@ -107,8 +123,8 @@ typedef struct {
  * returns it.  seed_scale_len() gives the per-unit length of `scale`.               */
 typedef struct {
   float* a;
-  float* U;
-  float* V;
+  void* U;   /* float, or 16-bit elements (dims->factors) */
+  void* V;
   float* scale;
   int32_t* ncols;
   const float* vbar;

@@ -21,6 +21,8 @@ Modules:
   compress     rank-R truncation: plain SVD of U V^T, and the QR + core-SVD route
   convert      end-of-prefill conversion of a dense state
   bytes_model  the analytical byte account (Table 17) behind Table 2
+  precision    rounding to the 16-bit factor formats (Table 9)
+  diagnostics  sink and content energies (Figures 3 and 12)
   run          whole trajectories (prefill, convert, decode, compress) for sampled units
 
 Parity pins: every function above is pinned in tests/test_oracle_pins.py to a
@@ -29,4 +31,4 @@ recurrence, Lemma 1's sink recurrence, Eckart-Young by brute force, Corollary 4,
 the delta-rule write, closed-form unrolled sums, Table 2's byte values).
 """
 
-from . import bytes_model, compress, convert, factored, recurrences, run  # noqa: F401
+from . import bytes_model, compress, convert, diagnostics, factored, precision, recurrences, run  # noqa: F401

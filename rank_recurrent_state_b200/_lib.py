@@ -20,7 +20,7 @@ c_float_p = ctypes.POINTER(ctypes.c_float)
 
 class seed_dims(ctypes.Structure):
     _fields_ = [("form", c_int32), ("batch", c_int32), ("layers", c_int32), ("heads", c_int32),
-                ("d_k", c_int32), ("d_v", c_int32), ("R", c_int32), ("W", c_int32)]
+                ("d_k", c_int32), ("d_v", c_int32), ("R", c_int32), ("W", c_int32), ("factors", c_int32)]
 
 
 class seed_state(ctypes.Structure):

@@ -18,6 +18,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 int check_dims(const seed_dims* d) {
   if (!d) return SEED_ERR_INVALID_ARG;
   if (d->form < SEED_GDN || d->form > SEED_MAMBA2) return SEED_ERR_INVALID_ARG;
+  if (d->factors < SEED_FACTORS_F32 || d->factors > SEED_FACTORS_BF16) return SEED_ERR_INVALID_ARG;
   if (d->batch < 1 || d->layers < 1 || d->heads < 1 || d->R < 1 || d->W < 1)
     return SEED_ERR_INVALID_ARG;
   if (!seed::decode_dims_supported(d->d_k, d->d_v)) return SEED_ERR_SHAPE;

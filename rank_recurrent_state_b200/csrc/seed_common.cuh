@@ -1,8 +1,13 @@
 // seed_common.cuh -- device helpers shared by the libseed kernels.
 #pragma once
 
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <string.h>
+
+#include <type_traits>
 
 #include "../../include/seed.h"
 
@@ -28,6 +33,75 @@ SEED_DEV float4 fma4(float s, float4 x, float4 y) {
 SEED_DEV float4 zero4() { return make_float4(0.f, 0.f, 0.f, 0.f); }
 SEED_DEV bool finite4(float4 v) {
   return isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w);
+}
+
+// ------------------------------------------------------------------ factor storage
+// U and V hold float32 or 16-bit values (seed_factors); every kernel computes in
+// float32, converting when it reads a factor and rounding to nearest, ties to even,
+// when it writes one.
+SEED_DEV float fac_to_f(float x) { return x; }
+SEED_DEV float fac_to_f(__half x) { return __half2float(x); }
+SEED_DEV float fac_to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+SEED_DEV T fac_from_f(float x) {
+  if constexpr (std::is_same<T, __half>::value) return __float2half_rn(x);
+  else if constexpr (std::is_same<T, __nv_bfloat16>::value) return __float2bfloat16_rn(x);
+  else return x;
+}
+
+// The value x has once stored as T.
+template <typename T>
+SEED_DEV float fac_round(float x) { return fac_to_f(fac_from_f<T>(x)); }
+
+// P consecutive factor values (P = 1, 2, 4) at p, aligned to P * sizeof(T).
+template <typename T, int P>
+SEED_DEV void fac_ld(const T* p, float (&e)[P]) {
+  static_assert(P == 1 || P == 2 || P == 4, "P");
+  if constexpr (std::is_same<T, float>::value) {
+    if constexpr (P == 4) {
+      const float4 t = *reinterpret_cast<const float4*>(p);
+      e[0] = t.x; e[1] = t.y; e[2] = t.z; e[3] = t.w;
+    } else if constexpr (P == 2) {
+      const float2 t = *reinterpret_cast<const float2*>(p);
+      e[0] = t.x; e[1] = t.y;
+    } else {
+      e[0] = *p;
+    }
+  } else {
+    using W = typename std::conditional<P == 4, uint2, typename std::conditional<P == 2, uint32_t, uint16_t>::type>::type;
+    const W raw = *reinterpret_cast<const W*>(p);
+    T t[P];
+    memcpy(t, &raw, sizeof(raw));
+#pragma unroll
+    for (int i = 0; i < P; ++i) e[i] = fac_to_f(t[i]);
+  }
+}
+
+template <typename T, int P>
+SEED_DEV void fac_st(T* p, const float (&e)[P]) {
+  static_assert(P == 1 || P == 2 || P == 4, "P");
+  if constexpr (std::is_same<T, float>::value) {
+    if constexpr (P == 4) *reinterpret_cast<float4*>(p) = make_float4(e[0], e[1], e[2], e[3]);
+    else if constexpr (P == 2) *reinterpret_cast<float2*>(p) = make_float2(e[0], e[1]);
+    else *p = e[0];
+  } else {
+    using W = typename std::conditional<P == 4, uint2, typename std::conditional<P == 2, uint32_t, uint16_t>::type>::type;
+    T t[P];
+#pragma unroll
+    for (int i = 0; i < P; ++i) t[i] = fac_from_f<T>(e[i]);
+    W raw;
+    memcpy(&raw, t, sizeof(raw));
+    *reinterpret_cast<W*>(p) = raw;
+  }
+}
+
+SEED_DEV float4 fac_ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+template <typename T>
+SEED_DEV float4 fac_ld4(const T* p) {
+  float e[4];
+  fac_ld<T, 4>(p, e);
+  return make_float4(e[0], e[1], e[2], e[3]);
 }
 
 template <int WIDTH>

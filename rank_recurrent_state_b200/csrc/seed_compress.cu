@@ -105,8 +105,8 @@ SEED_DEV void apply_q_warp(const float* A, int n, int m, const float* tau, float
 
 // ------------------------------------------------------------------ compress
 struct CompressParams {
-  float* U;
-  float* V;
+  void* U;   // element type: the kernel's factor type
+  void* V;
   float* scale;
   int32_t* ncols;
   float* sigma_out;
@@ -131,7 +131,7 @@ SEED_DEV int select_top(const float* sig, int n, int R, int* sel) {
 
 // One unit whose column count is R + W (checked by the caller), whole CTA.
 // `phase` is the parity of this unit's use of the CTA's mbarrier.
-template <int FORM, int DK, int DV, int NT>
+template <int FORM, int DK, int DV, int NT, typename TS>
 __device__ void compress_unit(const CompressParams& p, long long unit, long long srow,
                               unsigned char* smem_raw, uint64_t& bar, uint32_t phase) {
   constexpr int NW = NT / 32;
@@ -154,21 +154,34 @@ __device__ void compress_unit(const CompressParams& p, long long unit, long long
   int* sel = reinterpret_cast<int*>(cs_v + m);               // R
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-  // 1. panels -> shared memory (TMA bulk copies, no multicast)
-  if (tid == 0) {
-    mbar_arrive_expect_tx(&bar, (uint32_t)(m * (DK + DV) * sizeof(float)));
-    bulk_g2s(sU, p.U + unit * (long long)m * DK, (uint32_t)(m * DK * sizeof(float)), &bar);
-    bulk_g2s(sV, p.V + unit * (long long)m * DV, (uint32_t)(m * DV * sizeof(float)), &bar);
+  // 1. panels -> shared memory as float32 (TMA bulk copies, no multicast; 16-bit
+  //    factors are read and widened by the threads)
+  constexpr bool F32 = std::is_same<TS, float>::value;
+  if constexpr (F32) {
+    if (tid == 0) {
+      mbar_arrive_expect_tx(&bar, (uint32_t)(m * (DK + DV) * sizeof(float)));
+      bulk_g2s(sU, static_cast<const float*>(p.U) + unit * (long long)m * DK, (uint32_t)(m * DK * sizeof(float)),
+               &bar);
+      bulk_g2s(sV, static_cast<const float*>(p.V) + unit * (long long)m * DV, (uint32_t)(m * DV * sizeof(float)),
+               &bar);
+    }
+  } else {
+    const TS* Us = static_cast<const TS*>(p.U) + unit * (long long)m * DK;
+    const TS* Vs = static_cast<const TS*>(p.V) + unit * (long long)m * DV;
+    for (int idx = tid; idx < m * DK; idx += NT) sU[idx] = fac_to_f(Us[idx]);
+    for (int idx = tid; idx < m * DV; idx += NT) sV[idx] = fac_to_f(Vs[idx]);
   }
   const int slen = p.slen;
   for (int i = tid; i < slen; i += NT) s_scale[i] = p.scale[unit * slen + i];
   __syncthreads();
   // every thread polls, and the outcome is made uniform so no barrier below diverges
-  if (!__syncthreads_and(mbar_wait_bounded(&bar, phase, kWaitLimitNs))) {
-    if (tid == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
-    mbar_wait_bounded(&bar, phase, kWaitLimitNs);
-    __syncthreads();
-    return;
+  if constexpr (F32) {
+    if (!__syncthreads_and(mbar_wait_bounded(&bar, phase, kWaitLimitNs))) {
+      if (tid == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
+      mbar_wait_bounded(&bar, phase, kWaitLimitNs);
+      __syncthreads();
+      return;
+    }
   }
   // KDA's per-row decay is folded into the panel (P >= 0.85^W stays far from
   // underflow); the per-column decay of GDN / Mamba-2 stays a column factor
@@ -236,8 +249,8 @@ __device__ void compress_unit(const CompressParams& p, long long unit, long long
   const float szero = (float)max(DK, DV) * 1.1920929e-7f * smax;
 
   // 4. U' = Q_u (M Z)_R Sigma^{-1/2}, V' = Q_v Z_R Sigma^{1/2}: warp per output column
-  float* Ug = p.U + unit * (long long)m * DK;
-  float* Vg = p.V + unit * (long long)m * DV;
+  TS* Ug = static_cast<TS*>(p.U) + unit * (long long)m * DK;
+  TS* Vg = static_cast<TS*>(p.V) + unit * (long long)m * DV;
   bool bad = !conv;
   for (int task = warp; task < 2 * p.R; task += NW) {
     const bool isU = task < p.R;
@@ -259,8 +272,8 @@ __device__ void compress_unit(const CompressParams& p, long long unit, long long
       for (int q = 0; q < PER; ++q) {
         const int e = lane + 32 * q;
         if (e < DK) {
-          bad |= !isfinite(y[q]);
-          Ug[(long long)r * DK + e] = y[q];
+          bad |= !isfinite(fac_round<TS>(y[q]));
+          Ug[(long long)r * DK + e] = fac_from_f<TS>(y[q]);
         }
       }
     } else {
@@ -276,8 +289,8 @@ __device__ void compress_unit(const CompressParams& p, long long unit, long long
       for (int q = 0; q < PER; ++q) {
         const int e = lane + 32 * q;
         if (e < DV) {
-          bad |= !isfinite(y[q]);
-          Vg[(long long)r * DV + e] = y[q];
+          bad |= !isfinite(fac_round<TS>(y[q]));
+          Vg[(long long)r * DV + e] = fac_from_f<TS>(y[q]);
         }
       }
     }
@@ -295,7 +308,7 @@ __device__ void compress_unit(const CompressParams& p, long long unit, long long
 // Scans the scope in chunks of NT units, collects those holding R + W columns and
 // compresses them one after the other with the whole CTA.  A modest grid suffices:
 // after the fast kernel this pass normally finds nothing left to do.
-template <int FORM, int DK, int DV, int NT>
+template <int FORM, int DK, int DV, int NT, typename TS>
 __global__ void __launch_bounds__(NT) compress_kernel(const CompressParams p) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t bar;
@@ -327,7 +340,7 @@ __global__ void __launch_bounds__(NT) compress_kernel(const CompressParams p) {
       const long long i2 = base + s_list[k];
       const long long b = i2 / per, rest = i2 - b * per;
       const long long unit = p.layer < 0 ? i2 : (b * p.L + p.layer) * p.H + rest;
-      compress_unit<FORM, DK, DV, NT>(p, unit, i2, smem_raw, bar, phase);
+      compress_unit<FORM, DK, DV, NT, TS>(p, unit, i2, smem_raw, bar, phase);
       phase ^= 1u;
     }
     __syncthreads();
@@ -341,11 +354,11 @@ static size_t compress_smem_bytes(int form, int dk, int dv, int R, int W, int nt
   return f * sizeof(float) + 16;
 }
 
-template <int FORM, int DK, int DV>
-static int launch_compress_t(const CompressParams& p, int blocks, cudaStream_t st) {
+template <int FORM, int DK, int DV, typename TS>
+static int launch_compress_tt(const CompressParams& p, int blocks, cudaStream_t st) {
   constexpr int NT = 128;
   const size_t smem = compress_smem_bytes(FORM, DK, DV, p.R, p.W, NT);
-  auto kern = compress_kernel<FORM, DK, DV, NT>;
+  auto kern = compress_kernel<FORM, DK, DV, NT, TS>;
   if (smem > 48 * 1024) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
@@ -354,6 +367,16 @@ static int launch_compress_t(const CompressParams& p, int blocks, cudaStream_t s
   const int grid = (blocks + NT - 1) / NT < 1184 ? (blocks + NT - 1) / NT : 1184;
   kern<<<grid, NT, smem, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? SEED_OK : SEED_ERR_CUDA;
+}
+
+template <int FORM, int DK, int DV>
+static int launch_compress_t(const CompressParams& p, int blocks, int factors, cudaStream_t st) {
+  switch (factors) {
+    case SEED_FACTORS_F32: return launch_compress_tt<FORM, DK, DV, float>(p, blocks, st);
+    case SEED_FACTORS_F16: return launch_compress_tt<FORM, DK, DV, __half>(p, blocks, st);
+    case SEED_FACTORS_BF16: return launch_compress_tt<FORM, DK, DV, __nv_bfloat16>(p, blocks, st);
+  }
+  return SEED_ERR_INVALID_ARG;
 }
 
 #define SEED_DISPATCH_DIMS(FN, FORM, ...)                                     \
@@ -377,9 +400,9 @@ int launch_compress(const seed_dims& d, const seed_state& s, int layer, float* s
                    d.batch, d.layers, d.heads, layer, d.R, d.W, scale_len(d)};
   const int blocks = d.batch * d.heads * (layer < 0 ? d.layers : 1);
   switch (d.form) {
-    case SEED_GDN: SEED_DISPATCH_DIMS(launch_compress_t, SEED_GDN, p, blocks, st);
-    case SEED_KDA: SEED_DISPATCH_DIMS(launch_compress_t, SEED_KDA, p, blocks, st);
-    case SEED_MAMBA2: SEED_DISPATCH_DIMS(launch_compress_t, SEED_MAMBA2, p, blocks, st);
+    case SEED_GDN: SEED_DISPATCH_DIMS(launch_compress_t, SEED_GDN, p, blocks, d.factors, st);
+    case SEED_KDA: SEED_DISPATCH_DIMS(launch_compress_t, SEED_KDA, p, blocks, d.factors, st);
+    case SEED_MAMBA2: SEED_DISPATCH_DIMS(launch_compress_t, SEED_MAMBA2, p, blocks, d.factors, st);
   }
   return SEED_ERR_INVALID_ARG;
 }
@@ -388,21 +411,21 @@ int launch_compress(const seed_dims& d, const seed_state& s, int layer, float* s
 struct InitParams {
   const float* S;
   float* a;
-  float* U;
-  float* V;
+  void* U;   // element type: the kernel's factor type
+  void* V;
   float* scale;
   int32_t* ncols;
   const float* vbar;
   float* sigma_out;
   uint32_t* status;
-  int B, L, H, layer, R, W, form, slen;
+  int B, L, H, layer, R, W, form, slen, factors;
 };
 
 // The one-sided Jacobi runs over the shorter side of C so that the columns it
 // orthogonalises are at most as many as their length: over the d_v columns of C
 // when d_k >= d_v, else over the d_k columns of C^T.  Either way at most one
 // column is a structural null direction (C vbar = 0), not many.
-template <int DK, int DV, int NT>
+template <int DK, int DV, int NT, typename TS>
 __global__ void __launch_bounds__(NT) init_kernel(const InitParams p) {
   constexpr int NW = NT / 32;
   constexpr bool COLS = DK >= DV;       // Jacobi over the columns of C
@@ -492,8 +515,8 @@ __global__ void __launch_bounds__(NT) init_kernel(const InitParams p) {
 
   // COLS: U[:, r] = (C Z)[:, j] / sqrt(s), V[:, r] = Z[:, j] sqrt(s)
   // else: U[:, r] = Z[:, j] sqrt(s),       V[:, r] = (C^T Z)[:, j] / sqrt(s)
-  float* Ug = p.U + unit * (long long)m * DK;
-  float* Vg = p.V + unit * (long long)m * DV;
+  TS* Ug = static_cast<TS*>(p.U) + unit * (long long)m * DK;
+  TS* Vg = static_cast<TS*>(p.V) + unit * (long long)m * DV;
   bool bad = !conv;
   for (int r = warp; r < p.R; r += NW) {
     const bool valid = r < NC;
@@ -503,13 +526,13 @@ __global__ void __launch_bounds__(NT) init_kernel(const InitParams p) {
     const float fz = zero ? 0.f : sqrtf(s), fc = zero ? 0.f : rsqrtf(s);
     for (int e = lane; e < DK; e += 32) {
       const float x = COLS ? fc * sC[j * LDC + e] : fz * sZ[j * LDZ + e];
-      bad |= !isfinite(x);
-      Ug[(long long)r * DK + e] = x;
+      bad |= !isfinite(fac_round<TS>(x));
+      Ug[(long long)r * DK + e] = fac_from_f<TS>(x);
     }
     for (int e = lane; e < DV; e += 32) {
       const float x = COLS ? fz * sZ[j * LDZ + e] : fc * sC[j * LDC + e];
-      bad |= !isfinite(x);
-      Vg[(long long)r * DV + e] = x;
+      bad |= !isfinite(fac_round<TS>(x));
+      Vg[(long long)r * DV + e] = fac_from_f<TS>(x);
     }
     if (p.sigma_out && lane == 0) p.sigma_out[(long long)blockIdx.x * p.R + r] = s;
   }
@@ -523,13 +546,13 @@ __global__ void __launch_bounds__(NT) init_kernel(const InitParams p) {
   if (bad && conv) raise_flag(p.status, SEED_FLAG_NONFINITE);
 }
 
-template <int FORM, int DK, int DV>
-static int launch_init_t(const InitParams& p, int blocks, cudaStream_t st) {
+template <int DK, int DV, typename TS>
+static int launch_init_tt(const InitParams& p, int blocks, cudaStream_t st) {
   constexpr int NT = 256;
   constexpr int NC = DK >= DV ? DV : DK, NR = DK >= DV ? DK : DV;
   const size_t smem = ((size_t)NC * (NR + 1) + (size_t)NC * (NC + 1) + DV + DK + NC + NT / 32 +
                        p.R) * sizeof(float) + 16;
-  auto kern = init_kernel<DK, DV, NT>;
+  auto kern = init_kernel<DK, DV, NT, TS>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return SEED_ERR_CUDA;
@@ -537,10 +560,20 @@ static int launch_init_t(const InitParams& p, int blocks, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? SEED_OK : SEED_ERR_CUDA;
 }
 
+template <int FORM, int DK, int DV>
+static int launch_init_t(const InitParams& p, int blocks, cudaStream_t st) {
+  switch (p.factors) {
+    case SEED_FACTORS_F32: return launch_init_tt<DK, DV, float>(p, blocks, st);
+    case SEED_FACTORS_F16: return launch_init_tt<DK, DV, __half>(p, blocks, st);
+    case SEED_FACTORS_BF16: return launch_init_tt<DK, DV, __nv_bfloat16>(p, blocks, st);
+  }
+  return SEED_ERR_INVALID_ARG;
+}
+
 int launch_init_from_dense(const seed_dims& d, const seed_state& s, int layer, const float* S,
                            float* sigma_out, uint32_t* status, cudaStream_t st) {
   InitParams p{S, s.a, s.U, s.V, s.scale, s.ncols, s.vbar, sigma_out, status,
-               d.batch, d.layers, d.heads, layer, d.R, d.W, d.form, scale_len(d)};
+               d.batch, d.layers, d.heads, layer, d.R, d.W, d.form, scale_len(d), d.factors};
   const int blocks = d.batch * d.heads * (layer < 0 ? d.layers : 1);
   SEED_DISPATCH_DIMS(launch_init_t, 0, p, blocks, st);
 }
@@ -548,18 +581,18 @@ int launch_init_from_dense(const seed_dims& d, const seed_state& s, int layer, c
 // ------------------------------------------------------------------ to_dense
 struct ToDenseParams {
   const float* a;
-  const float* U;
-  const float* V;
+  const void* U;   // element type: the kernel's factor type
+  const void* V;
   const float* scale;
   const int32_t* ncols;
   const float* vbar;
   const int32_t* units;
   float* S;
   uint32_t* status;
-  int B, L, H, layer, R, W, form, slen;
+  int B, L, H, layer, R, W, form, slen, factors;
 };
 
-template <int DK, int DV, int NT>
+template <int DK, int DV, int NT, typename TS>
 __global__ void __launch_bounds__(NT) to_dense_kernel(const ToDenseParams p) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const int m = p.R + p.W;
@@ -586,9 +619,10 @@ __global__ void __launch_bounds__(NT) to_dense_kernel(const ToDenseParams p) {
   for (int idx = threadIdx.x; idx < c * DK; idx += NT) {
     const int j = idx / DK, i = idx - j * DK;
     const float sc = kda ? p.scale[unit * DK + i] : p.scale[unit * p.slen + j];
-    sU[idx] = sc * p.U[unit * (long long)m * DK + idx];
+    sU[idx] = sc * fac_to_f(static_cast<const TS*>(p.U)[unit * (long long)m * DK + idx]);
   }
-  for (int idx = threadIdx.x; idx < c * DV; idx += NT) sV[idx] = p.V[unit * (long long)m * DV + idx];
+  for (int idx = threadIdx.x; idx < c * DV; idx += NT)
+    sV[idx] = fac_to_f(static_cast<const TS*>(p.V)[unit * (long long)m * DV + idx]);
   for (int i = threadIdx.x; i < DK; i += NT) s_a[i] = p.a[unit * DK + i];
   for (int i = threadIdx.x; i < DV; i += NT) s_vb[i] = p.vbar[((long long)l * p.H + h) * DV + i];
   __syncthreads();
@@ -601,11 +635,11 @@ __global__ void __launch_bounds__(NT) to_dense_kernel(const ToDenseParams p) {
   }
 }
 
-template <int FORM, int DK, int DV>
-static int launch_to_dense_t(const ToDenseParams& p, int blocks, cudaStream_t st) {
+template <int DK, int DV, typename TS>
+static int launch_to_dense_tt(const ToDenseParams& p, int blocks, cudaStream_t st) {
   constexpr int NT = 256;
   const size_t smem = ((size_t)(p.R + p.W) * (DK + DV) + DK + DV) * sizeof(float);
-  auto kern = to_dense_kernel<DK, DV, NT>;
+  auto kern = to_dense_kernel<DK, DV, NT, TS>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return SEED_ERR_CUDA;
@@ -613,10 +647,20 @@ static int launch_to_dense_t(const ToDenseParams& p, int blocks, cudaStream_t st
   return cudaGetLastError() == cudaSuccess ? SEED_OK : SEED_ERR_CUDA;
 }
 
+template <int FORM, int DK, int DV>
+static int launch_to_dense_t(const ToDenseParams& p, int blocks, cudaStream_t st) {
+  switch (p.factors) {
+    case SEED_FACTORS_F32: return launch_to_dense_tt<DK, DV, float>(p, blocks, st);
+    case SEED_FACTORS_F16: return launch_to_dense_tt<DK, DV, __half>(p, blocks, st);
+    case SEED_FACTORS_BF16: return launch_to_dense_tt<DK, DV, __nv_bfloat16>(p, blocks, st);
+  }
+  return SEED_ERR_INVALID_ARG;
+}
+
 int launch_to_dense(const seed_dims& d, const seed_state& s, int layer, const int32_t* units,
                     int n_units, float* S_out, uint32_t* status, cudaStream_t st) {
   ToDenseParams p{s.a, s.U, s.V, s.scale, s.ncols, s.vbar, units, S_out, status,
-                  d.batch, d.layers, d.heads, layer, d.R, d.W, d.form, scale_len(d)};
+                  d.batch, d.layers, d.heads, layer, d.R, d.W, d.form, scale_len(d), d.factors};
   SEED_DISPATCH_DIMS(launch_to_dense_t, 0, p, n_units, st);
 }
 

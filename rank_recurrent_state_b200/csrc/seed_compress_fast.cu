@@ -42,8 +42,8 @@
 namespace seed {
 
 struct FastParams {
-  float* U;
-  float* V;
+  void* U;   // element type: the kernel's factor type
+  void* V;
   float* scale;
   int32_t* ncols;
   float* sigma_out;
@@ -312,6 +312,74 @@ SEED_DEV void issue_chunk(int c, float* sA, const CUtensorMap* tmU, const CUtens
 // Offset (in floats) of element e of column j in a swizzled chunk buffer.
 SEED_DEV int swz(int j, int e) { return j * 32 + ((((e >> 2) ^ (j & 7)) << 2) | (e & 3)); }
 
+// 16-bit factors.  Chunk c is copied as it is stored (lane l: 8 rows 8 (l & 3) ..
+// of column 8 pass + (l >> 2), one 16-byte cp.async each) into staging buffer c & 1
+// (the two take the place of float32 chunk buffer 1), then widened by the same
+// lanes into float32 chunk buffer 0 in the swizzled layout of the tensor copies, so
+// that the arithmetic below is the float32 path's.  Columns m .. MP-1 become zeros.
+template <int DK, int DV, int MP, typename TS>
+SEED_DEV void issue_chunk16(int c, float* sA, const FastParams& p, long long unit, int m) {
+  constexpr int NCU = DK / 32, CHUNK = MP * 32;
+  const int lane = threadIdx.x & 31, q = lane & 3;
+  const bool isU = c < NCU;
+  const int D = isU ? DK : DV;
+  const int r0 = 32 * (isU ? c : c - NCU);
+  const TS* src = static_cast<const TS*>(isU ? p.U : p.V) + unit * (long long)m * D + r0;
+  TS* stg = reinterpret_cast<TS*>(sA + CHUNK) + (c & 1) * CHUNK;
+#pragma unroll
+  for (int pass = 0; pass < MP / 8; ++pass) {
+    const int j = pass * 8 + (lane >> 2);
+    if (j < m) cp_async16(stg + j * 32 + 8 * q, src + (long long)j * D + 8 * q);
+  }
+  cp_async_commit();
+}
+
+// Waits for chunk c (more: chunk c + 1 was issued after it) and widens it.
+template <int MP, typename TS>
+SEED_DEV void widen_chunk16(int c, float* sA, int m, bool more) {
+  constexpr int CHUNK = MP * 32;
+  if (more) cp_async_wait<1>();
+  else cp_async_wait<0>();
+  const int lane = threadIdx.x & 31, q = lane & 3;
+  const TS* stg = reinterpret_cast<const TS*>(sA + CHUNK) + (c & 1) * CHUNK;
+#pragma unroll
+  for (int pass = 0; pass < MP / 8; ++pass) {
+    const int j = pass * 8 + (lane >> 2);
+    float lo[4] = {0.f, 0.f, 0.f, 0.f}, hi[4] = {0.f, 0.f, 0.f, 0.f};
+    if (j < m) {
+      fac_ld<TS, 4>(stg + j * 32 + 8 * q, lo);
+      fac_ld<TS, 4>(stg + j * 32 + 8 * q + 4, hi);
+    }
+    st4(sA + j * 32 + (((2 * q) ^ (j & 7)) << 2), make_float4(lo[0], lo[1], lo[2], lo[3]));
+    st4(sA + j * 32 + (((2 * q + 1) ^ (j & 7)) << 2), make_float4(hi[0], hi[1], hi[2], hi[3]));
+  }
+  __syncwarp();
+}
+
+// The next chunk of the stream: float32 factors wait for its tensor copy (false on
+// timeout, after waiting for the copies in flight); 16-bit factors widen it and
+// issue chunk c + 2 into the staging buffer it leaves.  Returns the chunk's buffer
+// through buf.
+template <int DK, int DV, int MP, typename TS>
+SEED_DEV bool next_chunk(int c, uint32_t ph, float* sA, uint64_t* bar, const FastParams& p, long long unit,
+                         int m, const float*& buf) {
+  constexpr int NCH = (DK + DV) / 32, CHUNK = MP * 32;
+  if constexpr (std::is_same<TS, float>::value) {
+    const int bb = c & 1;
+    if (!__all_sync(kFull, mbar_wait_bounded(&bar[bb], ph, kWaitLimitNs))) {
+      mbar_wait_bounded(&bar[bb], ph, kWaitLimitNs);
+      if (c + 1 < NCH) mbar_wait_bounded(&bar[bb ^ 1], ph ^ (uint32_t)bb, kWaitLimitNs);
+      return false;
+    }
+    buf = sA + bb * CHUNK;
+  } else {
+    widen_chunk16<MP, TS>(c, sA, m, c + 1 < NCH);
+    if (c + 2 < NCH) issue_chunk16<DK, DV, MP, TS>(c + 2, sA, p, unit, m);
+    buf = sA;
+  }
+  return true;
+}
+
 // Tensor-core products in float32 accuracy: x = hi + lo with hi = tf32(x) and
 // lo = tf32(x - hi), and a b ~ hi_a hi_b + hi_a lo_b + lo_a hi_b (the dropped
 // lo_a lo_b is below 2^-21 of a b), each term one warp-level mma.sync m16n8k8 with
@@ -346,10 +414,11 @@ SEED_DEV void mma3_tf32(float (&d)[4], const uint32_t (&ah)[4], const uint32_t (
 // columns).  fold (KDA's U): entries weighted by P (true U = Diag(P) U).  Also
 // checks the column scale.  Returns false if a copy did not arrive in time (after
 // waiting for those in flight).
-template <bool KDA, int NCU, int NCH, int MP, int CHUNK, int LG>
+template <bool KDA, int DK, int DV, int MP, int LG, typename TS>
 SEED_DEV bool gram_stream(int c0, int c1, bool fold, float* sA, const CUtensorMap* tmU,
-                          const CUtensorMap* tmV, long long unit, int m, uint64_t* bar, const float* scl,
-                          float* Gs, float (&g)[MP], bool& bad) {
+                          const CUtensorMap* tmV, const FastParams& p, long long unit, int m, uint64_t* bar,
+                          const float* scl, float* Gs, float (&g)[MP], bool& bad) {
+  constexpr int NCU = DK / 32, NCH = (DK + DV) / 32, CHUNK = MP * 32;
   constexpr int NT = MP / 8, MT = MP / 16;
   const int lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
   float acc[MT][NT][4];
@@ -364,14 +433,8 @@ SEED_DEV bool gram_stream(int c0, int c1, bool fold, float* sA, const CUtensorMa
   for (int nt = 0; nt < NT; ++nt) mx[nt] = 0.f;
 #pragma unroll 1
   for (int c = c0; c < c1; ++c) {
-    const int bb = c & 1;
-    const uint32_t ph = (uint32_t)(c >> 1) & 1u;
-    if (!__all_sync(kFull, mbar_wait_bounded(&bar[bb], ph, kWaitLimitNs))) {
-      mbar_wait_bounded(&bar[bb], ph, kWaitLimitNs);
-      if (c + 1 < NCH) mbar_wait_bounded(&bar[bb ^ 1], (uint32_t)((c + 1) >> 1) & 1u, kWaitLimitNs);
-      return false;
-    }
-    const float* buf = sA + bb * CHUNK;
+    const float* buf;
+    if (!next_chunk<DK, DV, MP, TS>(c, (uint32_t)(c >> 1) & 1u, sA, bar, p, unit, m, buf)) return false;
     const int r0 = 32 * (c < NCU ? c : c - NCU);
 #pragma unroll 1
     for (int ks = 0; ks < 4; ++ks) {
@@ -397,7 +460,7 @@ SEED_DEV bool gram_stream(int c0, int c1, bool fold, float* sA, const CUtensorMa
       }
     }
     __syncwarp();   // every lane has read this chunk before the next copy overwrites it
-    if (c + 2 < NCH) issue_chunk<NCU, CHUNK>(c + 2, sA, tmU, tmV, unit, bar);
+    if (std::is_same<TS, float>::value && c + 2 < NCH) issue_chunk<NCU, CHUNK>(c + 2, sA, tmU, tmV, unit, bar);
   }
   // largest magnitude of column nt * 8 + gq, over the four lanes of the group
 #pragma unroll
@@ -455,7 +518,21 @@ struct FastLayout {
   static constexpr size_t bytes = FLOATS * sizeof(float) + (MP + 4) * sizeof(int) + 1024;
 };
 
-template <int FORM, int DK, int DV, int MP>
+// Chunks 0 and 1 of a stream.
+template <int DK, int DV, int MP, typename TS>
+SEED_DEV void start_stream(float* sA, const CUtensorMap* tmU, const CUtensorMap* tmV, const FastParams& p,
+                           long long unit, int m, uint64_t* bar) {
+  if constexpr (std::is_same<TS, float>::value) {
+    issue_chunk<DK / 32, MP * 32>(0, sA, tmU, tmV, unit, bar);
+    issue_chunk<DK / 32, MP * 32>(1, sA, tmU, tmV, unit, bar);
+  } else {
+    issue_chunk16<DK, DV, MP, TS>(0, sA, p, unit, m);
+    issue_chunk16<DK, DV, MP, TS>(1, sA, p, unit, m);
+  }
+}
+
+// The tensor maps describe float32 factors; with 16-bit factors they are unused.
+template <int FORM, int DK, int DV, int MP, typename TS>
 __global__ void __launch_bounds__(32)
     compress_fast_kernel(const FastParams p, const __grid_constant__ CUtensorMap tmU,
                          const __grid_constant__ CUtensorMap tmV) {
@@ -496,12 +573,11 @@ __global__ void __launch_bounds__(32)
   }
   for (int e = lane; e < p.slen; e += 32) scl[e] = p.scale[unit * p.slen + e];
   __syncwarp();
-  issue_chunk<NCU, CHUNK>(0, sA, &tmU, &tmV, unit, bar);
-  issue_chunk<NCU, CHUNK>(1, sA, &tmU, &tmV, unit, bar);
+  start_stream<DK, DV, MP, TS>(sA, &tmU, &tmV, p, unit, m, bar);
   bool bad = false;   // ill-conditioned or badly scaled: left for the Householder kernel
   float g[MP];
   // U: chunks 0 .. NCU-1, then its Cholesky factor (to its own region)
-  if (!gram_stream<KDA, NCU, NCH, MP, CHUNK, LG>(0, NCU, true, sA, &tmU, &tmV, unit, m, bar, scl, sLu, g, bad)) {
+  if (!gram_stream<KDA, DK, DV, MP, LG, TS>(0, NCU, true, sA, &tmU, &tmV, p, unit, m, bar, scl, sLu, g, bad)) {
     if (lane == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
     return;
   }
@@ -511,7 +587,7 @@ __global__ void __launch_bounds__(32)
     cholesky_rolled<MP, LG>(g, n, bad, sLu);
   }
   // V: chunks NCU .. NCH-1; L_v over the chunk buffers once the last one is read
-  if (!gram_stream<KDA, NCU, NCH, MP, CHUNK, LG>(NCU, NCH, false, sA, &tmU, &tmV, unit, m, bar, scl, sM, g, bad)) {
+  if (!gram_stream<KDA, DK, DV, MP, LG, TS>(NCU, NCH, false, sA, &tmU, &tmV, p, unit, m, bar, scl, sM, g, bad)) {
     if (lane == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
     return;
   }
@@ -715,24 +791,19 @@ __global__ void __launch_bounds__(32)
   //    holds them, so slots 0..R-1 can be overwritten in place.
   fence_proxy_async_smem();   // the chunk buffers were written with ordinary stores
   __syncwarp();
-  issue_chunk<NCU, CHUNK>(0, sA, &tmU, &tmV, unit, bar);
-  issue_chunk<NCU, CHUNK>(1, sA, &tmU, &tmV, unit, bar);
+  start_stream<DK, DV, MP, TS>(sA, &tmU, &tmV, p, unit, m, bar);
   bool nonfinite = false;
-  float* Uo = p.U + unit * (long long)m * DK;
-  float* Vo = p.V + unit * (long long)m * DV;
+  TS* Uo = static_cast<TS*>(p.U) + unit * (long long)m * DK;
+  TS* Vo = static_cast<TS*>(p.V) + unit * (long long)m * DV;
 #pragma unroll 1
   for (int c = 0; c < NCH; ++c) {
-    const int bb = c & 1;
-    const uint32_t ph = (uint32_t)(NCH / 2 + (c >> 1)) & 1u;
-    if (!__all_sync(kFull, mbar_wait_bounded(&bar[bb], ph, kWaitLimitNs))) {
+    const float* buf;
+    if (!next_chunk<DK, DV, MP, TS>(c, (uint32_t)(NCH / 2 + (c >> 1)) & 1u, sA, bar, p, unit, m, buf)) {
       if (lane == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
-      mbar_wait_bounded(&bar[bb], ph, kWaitLimitNs);
-      if (c + 1 < NCH) mbar_wait_bounded(&bar[bb ^ 1], (uint32_t)(NCH / 2 + ((c + 1) >> 1)) & 1u, kWaitLimitNs);
       return;   // the unit keeps R + W columns; the slots written so far hold partial results
     }
     const bool isU = c < NCU;
     const int r0 = 32 * (isU ? c : c - NCU);
-    const float* buf = sA + bb * CHUNK;
     const float* T = isU ? sTu : sTv;
     // out (32 rows x 16) = chunk (32 rows x MP) T (MP x 16): m16n8k8 tiles, rows
     // mt * 16 + .., output columns nt * 8 + ..; columns >= m are zero in both
@@ -766,8 +837,8 @@ __global__ void __launch_bounds__(32)
       }
     }
     __syncwarp();   // every lane has read this chunk before the next copy overwrites it
-    if (c + 2 < NCH) issue_chunk<NCU, CHUNK>(c + 2, sA, &tmU, &tmV, unit, bar);
-    float* out = (isU ? Uo : Vo) + r0;
+    if (std::is_same<TS, float>::value && c + 2 < NCH) issue_chunk<NCU, CHUNK>(c + 2, sA, &tmU, &tmV, unit, bar);
+    TS* out = (isU ? Uo : Vo) + r0;
     const int ld = isU ? DK : DV;
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt) {
@@ -782,8 +853,8 @@ __global__ void __launch_bounds__(32)
             const int q = nt * 8 + 2 * tq + e;
             if (q < p.R) {
               const float v = acc[mt][nt][2 * hh + e] * rowf;
-              nonfinite |= !isfinite(v);
-              out[(long long)q * ld + r] = v;
+              nonfinite |= !isfinite(fac_round<TS>(v));
+              out[(long long)q * ld + r] = fac_from_f<TS>(v);
             }
           }
         }
@@ -827,10 +898,10 @@ static bool make_panel_map(CUtensorMap* tm, const float* base, int D, int m, lon
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int FORM, int DK, int DV, int MP>
+template <int FORM, int DK, int DV, int MP, typename TS>
 static int launch_fast_t(const FastParams& p, int blocks, cudaStream_t st) {
   using Lay = FastLayout<FORM, DK, DV, MP>;
-  auto kern = compress_fast_kernel<FORM, DK, DV, MP>;
+  auto kern = compress_fast_kernel<FORM, DK, DV, MP, TS>;
   constexpr int kMaxDev = 64;
   static bool attr_set[kMaxDev] = {false};
   int dev = 0;
@@ -844,17 +915,31 @@ static int launch_fast_t(const FastParams& p, int blocks, cudaStream_t st) {
   const long long units = (long long)p.B * p.L * p.H;
   const int m = p.R + p.W;
   CUtensorMap tmU, tmV;
-  if (!make_panel_map(&tmU, p.U, DK, m, units, MP) || !make_panel_map(&tmV, p.V, DV, m, units, MP))
+  memset(&tmU, 0, sizeof(tmU));
+  memset(&tmV, 0, sizeof(tmV));
+  if (std::is_same<TS, float>::value &&
+      (!make_panel_map(&tmU, static_cast<const float*>(p.U), DK, m, units, MP) ||
+       !make_panel_map(&tmV, static_cast<const float*>(p.V), DV, m, units, MP)))
     return SEED_ERR_CUDA;
   kern<<<blocks, 32, Lay::bytes, st>>>(p, tmU, tmV);
   return cudaGetLastError() == cudaSuccess ? SEED_OK : SEED_ERR_CUDA;
 }
 
-template <int FORM, int DK, int DV>
-static int launch_fast_m(const FastParams& p, int blocks, cudaStream_t st) {
+template <int FORM, int DK, int DV, typename TS>
+static int launch_fast_mt(const FastParams& p, int blocks, cudaStream_t st) {
   const int m = p.R + p.W;
-  if (m <= 16) return launch_fast_t<FORM, DK, DV, 16>(p, blocks, st);
-  return launch_fast_t<FORM, DK, DV, 32>(p, blocks, st);
+  if (m <= 16) return launch_fast_t<FORM, DK, DV, 16, TS>(p, blocks, st);
+  return launch_fast_t<FORM, DK, DV, 32, TS>(p, blocks, st);
+}
+
+template <int FORM, int DK, int DV>
+static int launch_fast_m(const FastParams& p, int blocks, int factors, cudaStream_t st) {
+  switch (factors) {
+    case SEED_FACTORS_F32: return launch_fast_mt<FORM, DK, DV, float>(p, blocks, st);
+    case SEED_FACTORS_F16: return launch_fast_mt<FORM, DK, DV, __half>(p, blocks, st);
+    case SEED_FACTORS_BF16: return launch_fast_mt<FORM, DK, DV, __nv_bfloat16>(p, blocks, st);
+  }
+  return SEED_ERR_INVALID_ARG;
 }
 
 // R <= 16: the R new columns are accumulated in registers in one pass over the
@@ -872,10 +957,10 @@ int launch_compress_fast(const seed_dims& d, const seed_state& s, int layer, flo
   const int blocks = d.batch * d.heads * (layer < 0 ? d.layers : 1);
 #define SEED_FAST_DIMS(FORM)                                                                       \
   do {                                                                                             \
-    if (d.d_k == 128 && d.d_v == 128) return launch_fast_m<FORM, 128, 128>(p, blocks, st);          \
-    if (d.d_k == 128 && d.d_v == 64) return launch_fast_m<FORM, 128, 64>(p, blocks, st);            \
-    if (d.d_k == 64 && d.d_v == 128) return launch_fast_m<FORM, 64, 128>(p, blocks, st);            \
-    if (d.d_k == 64 && d.d_v == 64) return launch_fast_m<FORM, 64, 64>(p, blocks, st);              \
+    if (d.d_k == 128 && d.d_v == 128) return launch_fast_m<FORM, 128, 128>(p, blocks, d.factors, st);          \
+    if (d.d_k == 128 && d.d_v == 64) return launch_fast_m<FORM, 128, 64>(p, blocks, d.factors, st);            \
+    if (d.d_k == 64 && d.d_v == 128) return launch_fast_m<FORM, 64, 128>(p, blocks, d.factors, st);            \
+    if (d.d_k == 64 && d.d_v == 64) return launch_fast_m<FORM, 64, 64>(p, blocks, d.factors, st);              \
     return SEED_ERR_SHAPE;                                                                         \
   } while (0)
   switch (d.form) {

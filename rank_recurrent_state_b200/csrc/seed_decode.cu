@@ -42,9 +42,9 @@ SEED_DEV bool consumer_and(bool v) {
   return out != 0;
 }
 
-template <int FORM, int DK, int DV, int MAXC, int NS>
+template <int FORM, int DK, int DV, int MAXC, int NS, typename TS>
 __global__ void __launch_bounds__(kDecodeThreads) decode_step_kernel(const DecodeParams p) {
-  using Stage = DecodeStage<FORM, DK, DV, MAXC>;
+  using Stage = DecodeStage<FORM, DK, DV, MAXC, TS>;
   constexpr int NW = kConsumerWarps;
   constexpr int NT = NW * 32;
   constexpr int LK = DK / 4;            // lanes per U column (float4 each)
@@ -118,14 +118,16 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_step_kernel(const Decod
       const bool valid = c >= 0 && c < m;
       uint32_t bytes = 0;
       if (valid) {
-        bytes = (uint32_t)(c * (DK + DV) + 3 * DK + 2 * DV) * 4u;
+        bytes = (uint32_t)(c * (DK + DV) * sizeof(TS)) + (uint32_t)(3 * DK + 2 * DV) * 4u;
         bytes += KDA ? 2u * DK * 4u : (uint32_t)((c + 3) & ~3) * 4u;
       }
       mbar_arrive_expect_tx(&full[s], bytes);
       if (valid) {
         if (c > 0) {
-          bulk_g2s(S.U, p.U + unit * (long long)m * DK, (uint32_t)(c * DK * 4), &full[s]);
-          bulk_g2s(S.V, p.V + unit * (long long)m * DV, (uint32_t)(c * DV * 4), &full[s]);
+          bulk_g2s(S.U, static_cast<const TS*>(p.U) + unit * (long long)m * DK, (uint32_t)(c * DK * sizeof(TS)),
+                   &full[s]);
+          bulk_g2s(S.V, static_cast<const TS*>(p.V) + unit * (long long)m * DV, (uint32_t)(c * DV * sizeof(TS)),
+                   &full[s]);
         }
         bulk_g2s(S.a, p.a + unit * DK, DK * 4, &full[s]);
         bulk_g2s(S.k, p.k + (long long)u * DK, DK * 4, &full[s]);
@@ -177,7 +179,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_step_kernel(const Decod
 #pragma unroll
       for (int r = 0; r < CU; ++r) {
         const int j = gk + GK * r;
-        const float4 uc = j < c ? ld4(S.U + j * DK + 4 * lk) : zero4();
+        const float4 uc = j < c ? fac_ld4(S.U + j * DK + 4 * lk) : zero4();
         dv[r] = dot4(uc, qq);
         if constexpr (!M2) dv[CU + r] = dot4(uc, kk);
       }
@@ -247,7 +249,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_step_kernel(const Decod
         for (int r = 0; r < CV; ++r) {
           const int j = gv + GV * r;
           if (j < c) {
-            const float4 vc = ld4(S.V + j * DV + 4 * lv);
+            const float4 vc = fac_ld4(S.V + j * DV + 4 * lv);
             const float f = KDA ? 1.f : g * S.gam[j];
             if constexpr (!M2) yk = fma4(f * s_dk[j], vc, yk);
             yq = fma4(f * s_dq[j], vc, yq);
@@ -279,8 +281,8 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_step_kernel(const Decod
         else coef = be * omega;
         const float apq = (KDA ? aq : g * aq) + coef * kq;   // a+^T q
         bool bad = false;
-        float* Vnew = p.V + unit * (long long)m * DV + (long long)c * DV;
-        float* Unew = p.U + unit * (long long)m * DK + (long long)c * DK;
+        TS* Vnew = static_cast<TS*>(p.V) + unit * (long long)m * DV + (long long)c * DV;
+        TS* Unew = static_cast<TS*>(p.U) + unit * (long long)m * DK + (long long)c * DK;
         for (int e = tid; e < DV; e += NT) {
           float yke = 0.f, yqe = 0.f;
 #pragma unroll
@@ -291,8 +293,8 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_step_kernel(const Decod
           const float eps = S.v[e] - omega * S.vb[e];
           const float ncol = M2 ? be * eps : be * (eps - yke);
           const float oe = fmaf(S.vb[e], apq, yqe) + ncol * kq;
-          bad |= !(isfinite(ncol) && isfinite(oe));
-          Vnew[e] = ncol;
+          bad |= !(isfinite(fac_round<TS>(ncol)) && isfinite(oe));
+          Vnew[e] = fac_from_f<TS>(ncol);
           p.o[(long long)u * DV + e] = oe;
         }
         for (int e = tid; e < DK; e += NT) {
@@ -303,12 +305,13 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_step_kernel(const Decod
             const float pn = S.P[e] * S.al[e];
             anew = fmaf(S.al[e], ae, coef * ke);
             const float us = ke / pn;
-            bad |= !isfinite(us);
-            Unew[e] = us;
+            bad |= !isfinite(fac_round<TS>(us));
+            Unew[e] = fac_from_f<TS>(us);
             p.scale[unit * DK + e] = pn;
           } else {
             anew = fmaf(g, ae, coef * ke);
-            Unew[e] = ke;
+            bad |= !isfinite(fac_round<TS>(ke));
+            Unew[e] = fac_from_f<TS>(ke);
           }
           bad |= !isfinite(anew);
           p.a[unit * DK + e] = anew;
@@ -326,14 +329,14 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_step_kernel(const Decod
   }
 }
 
-template <int FORM, int DK, int DV, int MAXC>
+template <int FORM, int DK, int DV, int MAXC, typename TS>
 static int launch_one(const DecodeParams& p, cudaStream_t st) {
-  using Stage = DecodeStage<FORM, DK, DV, MAXC>;
+  using Stage = DecodeStage<FORM, DK, DV, MAXC, TS>;
   // stages: as many as fit in ~108 KB so that two CTAs share an SM, at least two
   constexpr int NS0 = (int)((108 * 1024) / sizeof(Stage));
   constexpr int NS = NS0 < 2 ? 2 : (NS0 > 6 ? 6 : NS0);
   const size_t smem = NS * sizeof(Stage) + 2 * NS * sizeof(uint64_t);
-  auto kern = decode_step_kernel<FORM, DK, DV, MAXC, NS>;
+  auto kern = decode_step_kernel<FORM, DK, DV, MAXC, NS, TS>;
   // per device: the shared-memory opt-in and the resident CTAs per SM
   constexpr int kMaxDev = 64;
   static int grid_per_sm[kMaxDev] = {0};
@@ -362,18 +365,28 @@ static int launch_one(const DecodeParams& p, cudaStream_t st) {
 
 // Up to 32 stored columns: one warp per unit (seed_decode_warp.cu); above, this
 // kernel with four consumer warps per unit.
-template <int FORM, int DK, int DV>
-static int launch_cols(const DecodeParams& p, cudaStream_t st) {
+template <int FORM, int DK, int DV, typename TS>
+static int launch_cols_t(const DecodeParams& p, cudaStream_t st) {
   const int maxc = p.R + p.W - 1;
-  if (maxc <= 32) return launch_decode_warp(p, FORM, DK, DV, st);
-  if (maxc <= 64) return launch_one<FORM, DK, DV, 64>(p, st);
-  return launch_one<FORM, DK, DV, 96>(p, st);
+  if (maxc <= 64) return launch_one<FORM, DK, DV, 64, TS>(p, st);
+  return launch_one<FORM, DK, DV, 96, TS>(p, st);
+}
+
+template <int FORM, int DK, int DV>
+static int launch_cols(const DecodeParams& p, int factors, cudaStream_t st) {
+  if (p.R + p.W - 1 <= 32) return launch_decode_warp(p, FORM, DK, DV, factors, st);
+  switch (factors) {
+    case SEED_FACTORS_F32: return launch_cols_t<FORM, DK, DV, float>(p, st);
+    case SEED_FACTORS_F16: return launch_cols_t<FORM, DK, DV, __half>(p, st);
+    case SEED_FACTORS_BF16: return launch_cols_t<FORM, DK, DV, __nv_bfloat16>(p, st);
+  }
+  return SEED_ERR_INVALID_ARG;
 }
 
 template <int FORM>
-static int launch_dims(const DecodeParams& p, int dk, int dv, cudaStream_t st) {
+static int launch_dims(const DecodeParams& p, int dk, int dv, int factors, cudaStream_t st) {
 #define SEED_DIMS_CASE(K, V) \
-  if (dk == K && dv == V) return launch_cols<FORM, K, V>(p, st);
+  if (dk == K && dv == V) return launch_cols<FORM, K, V>(p, factors, st);
   SEED_DIMS_CASE(16, 16)
   SEED_DIMS_CASE(32, 32)
   SEED_DIMS_CASE(64, 64)
@@ -390,9 +403,9 @@ int launch_decode_step(const seed_dims& d, const seed_state& s, int layer, const
   DecodeParams p{q, k, v, alpha, beta, o, s.a, s.U, s.V, s.scale, s.ncols, s.vbar, status,
                  d.batch, d.layers, d.heads, layer, d.R, d.W, scale_len(d)};
   switch (d.form) {
-    case SEED_GDN: return launch_dims<SEED_GDN>(p, d.d_k, d.d_v, st);
-    case SEED_KDA: return launch_dims<SEED_KDA>(p, d.d_k, d.d_v, st);
-    case SEED_MAMBA2: return launch_dims<SEED_MAMBA2>(p, d.d_k, d.d_v, st);
+    case SEED_GDN: return launch_dims<SEED_GDN>(p, d.d_k, d.d_v, d.factors, st);
+    case SEED_KDA: return launch_dims<SEED_KDA>(p, d.d_k, d.d_v, d.factors, st);
+    case SEED_MAMBA2: return launch_dims<SEED_MAMBA2>(p, d.d_k, d.d_v, d.factors, st);
   }
   return SEED_ERR_INVALID_ARG;
 }

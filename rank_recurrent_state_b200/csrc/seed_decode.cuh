@@ -14,8 +14,8 @@ struct DecodeParams {
   const float* beta;
   float* o;
   float* a;
-  float* U;
-  float* V;
+  void* U;   // element type: the kernel's factor type
+  void* V;
   float* scale;
   int32_t* ncols;
   const float* vbar;
@@ -23,13 +23,13 @@ struct DecodeParams {
   int B, L, H, layer, R, W, slen;
 };
 
-// One pipeline stage: everything a unit's step reads.
-template <int FORM, int DK, int DV, int MAXC>
+// One pipeline stage: everything a unit's step reads (U and V in their stored type).
+template <int FORM, int DK, int DV, int MAXC, typename TS>
 struct DecodeStage {
   static constexpr bool KDA = FORM == SEED_KDA;
   static constexpr int GPAD = (MAXC + 3) & ~3;
-  float U[MAXC * DK];
-  float V[MAXC * DV];
+  alignas(16) TS U[MAXC * DK];
+  alignas(16) TS V[MAXC * DV];
   float a[DK];
   float k[DK];
   float q[DK];
@@ -75,6 +75,6 @@ template <int NV>
 SEED_DEV constexpr int log2c() { return NV <= 1 ? 0 : 1 + log2c<NV / 2>(); }
 
 // The one-warp-per-unit decode kernel (seed_decode_warp.cu), for R + W - 1 <= 32.
-int launch_decode_warp(const DecodeParams& p, int form, int dk, int dv, cudaStream_t st);
+int launch_decode_warp(const DecodeParams& p, int form, int dk, int dv, int factors, cudaStream_t st);
 
 }  // namespace seed

@@ -114,27 +114,28 @@ SEED_DEV void load_vecs(const DecodeParams& p, int u, int c, UnitVecs<FORM, DK, 
 }
 
 // Lane 0: the bulk copies of the c stored columns of U and of V of unit u into the
-// stage (U at sU, V at sV), completing on bar.  A unit with an invalid column count
-// gets no copies (the wait still ends).
-template <int DK, int DV>
-SEED_DEV void issue_unit(const DecodeParams& p, float* sU, float* sV, uint64_t* bar, int u, int c, int m) {
+// stage (U at sU, V at sV, in their stored type TS), completing on bar.  A unit
+// with an invalid column count gets no copies (the wait still ends).  A column is
+// d_k (d_v) values of at least 2 bytes, d >= 16: every copy is a multiple of 16 bytes.
+template <int DK, int DV, typename TS>
+SEED_DEV void issue_unit(const DecodeParams& p, TS* sU, TS* sV, uint64_t* bar, int u, int c, int m) {
   const bool valid = c > 0 && c < m;
-  mbar_arrive_expect_tx(bar, valid ? (uint32_t)(c * (DK + DV)) * 4u : 0u);
+  mbar_arrive_expect_tx(bar, valid ? (uint32_t)(c * (DK + DV) * sizeof(TS)) : 0u);
   if (!valid) return;
   const long long unit = unit_index(p, u);
-  bulk_g2s(sU, p.U + unit * (long long)m * DK, (uint32_t)(c * DK * 4), bar);
-  bulk_g2s(sV, p.V + unit * (long long)m * DV, (uint32_t)(c * DV * 4), bar);
+  bulk_g2s(sU, static_cast<const TS*>(p.U) + unit * (long long)m * DK, (uint32_t)(c * DK * sizeof(TS)), bar);
+  bulk_g2s(sV, static_cast<const TS*>(p.V) + unit * (long long)m * DV, (uint32_t)(c * DV * sizeof(TS)), bar);
 }
 
 // Shared memory of one warp: the stage (U columns, then V columns, each sized for
 // the R + W - 1 columns a unit can hold before a step), the column coefficients and
 // the stage's mbarrier.
-__host__ __device__ constexpr size_t warp_stage_floats(int maxc, int dk, int dv) {
-  return (size_t)maxc * (dk + dv);
+__host__ __device__ constexpr size_t warp_stage_bytes(int maxc, int dk, int dv, int elem) {
+  return (size_t)maxc * (dk + dv) * elem;
 }
 constexpr int kCoefFloats = 2 * 32;
 
-template <int FORM, int DK, int DV, int MAXC>
+template <int FORM, int DK, int DV, int MAXC, typename TS>
 __global__ void __launch_bounds__(32) decode_warp_kernel(const DecodeParams p) {
   using Vecs = UnitVecs<FORM, DK, DV>;
   constexpr bool KDA = FORM == SEED_KDA;
@@ -144,9 +145,9 @@ __global__ void __launch_bounds__(32) decode_warp_kernel(const DecodeParams p) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const int m = p.R + p.W;
   const int maxc = m - 1;
-  float* sU = reinterpret_cast<float*>(smem_raw);
-  float* sV = sU + (size_t)maxc * DK;
-  float* s_f = sU + warp_stage_floats(maxc, DK, DV);   // [32][2] column coefficients (q, k)
+  TS* sU = reinterpret_cast<TS*>(smem_raw);
+  TS* sV = sU + (size_t)maxc * DK;
+  float* s_f = reinterpret_cast<float*>(smem_raw + warp_stage_bytes(maxc, DK, DV, sizeof(TS)));   // [32][2] (q, k)
   uint64_t* full = reinterpret_cast<uint64_t*>(s_f + kCoefFloats);
 
   const int lane = threadIdx.x;
@@ -163,7 +164,7 @@ __global__ void __launch_bounds__(32) decode_warp_kernel(const DecodeParams p) {
 
   // the first unit: its columns to the stage, its vectors to registers
   int c = p.ncols[unit_index(p, u0)];
-  if (lane == 0) issue_unit<DK, DV>(p, sU, sV, full, u0, c, m);
+  if (lane == 0) issue_unit<DK, DV, TS>(p, sU, sV, full, u0, c, m);
   Vecs cur, nxt;
   load_vecs<FORM, DK, DV>(p, u0, c, cur);
   int c_next = u0 + stride < n_units ? p.ncols[unit_index(p, u0 + stride)] : 0;
@@ -204,7 +205,7 @@ __global__ void __launch_bounds__(32) decode_warp_kernel(const DecodeParams p) {
           float ue[PK];
 #pragma unroll
           for (int e = 0; e < PK; ++e) ue[e] = 0.f;
-          if (j < c && kact) ldv<PK>(sU + j * DK + lane * PK, ue);
+          if (j < c && kact) fac_ld<TS, PK>(sU + j * DK + lane * PK, ue);
           dv[t] = dotv<PK>(ue, qq);
           if constexpr (!M2) dv[16 + t] = dotv<PK>(ue, kk);
         }
@@ -250,7 +251,7 @@ __global__ void __launch_bounds__(32) decode_warp_kernel(const DecodeParams p) {
           float ve[PV];
 #pragma unroll
           for (int e = 0; e < PV; ++e) ve[e] = 0.f;
-          if (vact) ldv<PV>(sV + j * DV + lane * PV, ve);
+          if (vact) fac_ld<TS, PV>(sV + j * DV + lane * PV, ve);
           const float2 f2 = *reinterpret_cast<const float2*>(s_f + 2 * j);   // (q, k) coefficients
 #pragma unroll
           for (int e = 0; e < PV; ++e) {
@@ -272,9 +273,9 @@ __global__ void __launch_bounds__(32) decode_warp_kernel(const DecodeParams p) {
             const float eps = cur.v[e] - omega * cur.vb[e];
             ncol[e] = M2 ? be * eps : be * (eps - yk[e]);
             oe[e] = fmaf(cur.vb[e], apq, yq[e]) + ncol[e] * kq;
-            bad |= !(isfinite(ncol[e]) && isfinite(oe[e]));
+            bad |= !(isfinite(fac_round<TS>(ncol[e])) && isfinite(oe[e]));
           }
-          stv<PV>(p.V + unit * (long long)m * DV + (long long)c * DV + lane * PV, ncol);
+          fac_st<TS, PV>(static_cast<TS*>(p.V) + unit * (long long)m * DV + (long long)c * DV + lane * PV, ncol);
           stv<PV>(p.o + (long long)u * DV + lane * PV, oe);
         }
         if (kact) {
@@ -285,14 +286,15 @@ __global__ void __launch_bounds__(32) decode_warp_kernel(const DecodeParams p) {
               pn[e] = cur.P[e] * cur.al[e];
               anew[e] = fmaf(cur.al[e], cur.a[e], coef * cur.k[e]);
               unew[e] = cur.k[e] / pn[e];
-              bad |= !isfinite(unew[e]);
+              bad |= !isfinite(fac_round<TS>(unew[e]));
             } else {
               anew[e] = fmaf(g, cur.a[e], coef * cur.k[e]);
               unew[e] = cur.k[e];
+              bad |= !isfinite(fac_round<TS>(unew[e]));
             }
             bad |= !isfinite(anew[e]);
           }
-          stv<PK>(p.U + unit * (long long)m * DK + (long long)c * DK + lane * PK, unew);
+          fac_st<TS, PK>(static_cast<TS*>(p.U) + unit * (long long)m * DK + (long long)c * DK + lane * PK, unew);
           stv<PK>(p.a + unit * DK + lane * PK, anew);
           if constexpr (KDA) stv<PK>(p.scale + unit * DK + lane * PK, pn);
         }
@@ -309,18 +311,18 @@ __global__ void __launch_bounds__(32) decode_warp_kernel(const DecodeParams p) {
     // every read of the stage (and of s_f) is above and complete (its values were
     // consumed); only bulk copies write the stage, so no proxy fence is needed
     __syncwarp();
-    if (lane == 0 && u_next < n_units) issue_unit<DK, DV>(p, sU, sV, full, u_next, c_next, m);
+    if (lane == 0 && u_next < n_units) issue_unit<DK, DV, TS>(p, sU, sV, full, u_next, c_next, m);
     cur = nxt;
     c = c_next;
     c_next = c_after;
   }
 }
 
-template <int FORM, int DK, int DV, int MAXC>
+template <int FORM, int DK, int DV, int MAXC, typename TS>
 static int launch_warp_t(const DecodeParams& p, cudaStream_t st) {
-  auto kern = decode_warp_kernel<FORM, DK, DV, MAXC>;
+  auto kern = decode_warp_kernel<FORM, DK, DV, MAXC, TS>;
   const int maxc = p.R + p.W - 1;
-  const size_t smem = warp_stage_floats(maxc, DK, DV) * sizeof(float) + kCoefFloats * sizeof(float) + 16;
+  const size_t smem = warp_stage_bytes(maxc, DK, DV, sizeof(TS)) + kCoefFloats * sizeof(float) + 16;
   // per device: the shared-memory opt-in (for the largest stage), and the resident
   // blocks per SM for each stage size
   constexpr int kMaxDev = 64;
@@ -330,7 +332,7 @@ static int launch_warp_t(const DecodeParams& p, cudaStream_t st) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev || maxc > MAXC) return SEED_ERR_CUDA;
   if (!attr_set[dev]) {
-    const size_t smax = warp_stage_floats(MAXC, DK, DV) * sizeof(float) + kCoefFloats * sizeof(float) + 16;
+    const size_t smax = warp_stage_bytes(MAXC, DK, DV, sizeof(TS)) + kCoefFloats * sizeof(float) + 16;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smax) != cudaSuccess)
       return SEED_ERR_CUDA;
     if (cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
@@ -349,26 +351,36 @@ static int launch_warp_t(const DecodeParams& p, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? SEED_OK : SEED_ERR_CUDA;
 }
 
-template <int FORM, int DK, int DV>
-static int launch_warp_dims(const DecodeParams& p, cudaStream_t st) {
+template <int FORM, int DK, int DV, typename TS>
+static int launch_warp_maxc(const DecodeParams& p, cudaStream_t st) {
   const int maxc = p.R + p.W - 1;
-  if (maxc <= 8) return launch_warp_t<FORM, DK, DV, 8>(p, st);
-  if (maxc <= 16) return launch_warp_t<FORM, DK, DV, 16>(p, st);
-  return launch_warp_t<FORM, DK, DV, 32>(p, st);
+  if (maxc <= 8) return launch_warp_t<FORM, DK, DV, 8, TS>(p, st);
+  if (maxc <= 16) return launch_warp_t<FORM, DK, DV, 16, TS>(p, st);
+  return launch_warp_t<FORM, DK, DV, 32, TS>(p, st);
+}
+
+template <int FORM, int DK, int DV>
+static int launch_warp_dims(const DecodeParams& p, int factors, cudaStream_t st) {
+  switch (factors) {
+    case SEED_FACTORS_F32: return launch_warp_maxc<FORM, DK, DV, float>(p, st);
+    case SEED_FACTORS_F16: return launch_warp_maxc<FORM, DK, DV, __half>(p, st);
+    case SEED_FACTORS_BF16: return launch_warp_maxc<FORM, DK, DV, __nv_bfloat16>(p, st);
+  }
+  return SEED_ERR_INVALID_ARG;
 }
 
 bool decode_warp_supported(const seed_dims& d) { return d.R + d.W - 1 <= 32; }
 
-int launch_decode_warp(const DecodeParams& p, int form, int dk, int dv, cudaStream_t st) {
-#define SEED_WARP_DIMS(FORM)                                                     \
-  do {                                                                           \
-    if (dk == 16 && dv == 16) return launch_warp_dims<FORM, 16, 16>(p, st);      \
-    if (dk == 32 && dv == 32) return launch_warp_dims<FORM, 32, 32>(p, st);      \
-    if (dk == 64 && dv == 64) return launch_warp_dims<FORM, 64, 64>(p, st);      \
-    if (dk == 128 && dv == 128) return launch_warp_dims<FORM, 128, 128>(p, st);  \
-    if (dk == 128 && dv == 64) return launch_warp_dims<FORM, 128, 64>(p, st);    \
-    if (dk == 64 && dv == 128) return launch_warp_dims<FORM, 64, 128>(p, st);    \
-    return SEED_ERR_SHAPE;                                                       \
+int launch_decode_warp(const DecodeParams& p, int form, int dk, int dv, int factors, cudaStream_t st) {
+#define SEED_WARP_DIMS(FORM)                                                              \
+  do {                                                                                    \
+    if (dk == 16 && dv == 16) return launch_warp_dims<FORM, 16, 16>(p, factors, st);      \
+    if (dk == 32 && dv == 32) return launch_warp_dims<FORM, 32, 32>(p, factors, st);      \
+    if (dk == 64 && dv == 64) return launch_warp_dims<FORM, 64, 64>(p, factors, st);      \
+    if (dk == 128 && dv == 128) return launch_warp_dims<FORM, 128, 128>(p, factors, st);  \
+    if (dk == 128 && dv == 64) return launch_warp_dims<FORM, 128, 64>(p, factors, st);    \
+    if (dk == 64 && dv == 128) return launch_warp_dims<FORM, 64, 128>(p, factors, st);    \
+    return SEED_ERR_SHAPE;                                                                \
   } while (0)
   switch (form) {
     case SEED_GDN: SEED_WARP_DIMS(SEED_GDN);

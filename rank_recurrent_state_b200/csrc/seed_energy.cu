@@ -21,15 +21,15 @@ namespace seed {
 
 struct EnergyParams {
   const float* a;
-  const float* U;
-  const float* V;
+  const void* U;   // element type: the kernel's factor type
+  const void* V;
   const float* scale;
   const int32_t* ncols;
   const float* vbar;
   const int32_t* units;
   float* out;
   uint32_t* status;
-  int B, L, H, layer, R, W, form, slen;
+  int B, L, H, layer, R, W, form, slen, factors;
 };
 
 constexpr int kEnergyThreads = 128;
@@ -47,7 +47,7 @@ SEED_DEV float block_sum(float v, float* red) {
   return t;
 }
 
-template <int DK, int DV>
+template <int DK, int DV, typename TS>
 __global__ void __launch_bounds__(kEnergyThreads) energy_kernel(const EnergyParams p) {
   constexpr int NT = kEnergyThreads, LU = DK + 1, LV = DV + 1;
   extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -76,11 +76,11 @@ __global__ void __launch_bounds__(kEnergyThreads) energy_kernel(const EnergyPara
   for (int idx = threadIdx.x; idx < c * DK; idx += NT) {
     const int j = idx / DK, i = idx - j * DK;
     const float sc = kda ? p.scale[unit * DK + i] : p.scale[unit * p.slen + j];
-    sU[j * LU + i] = sc * p.U[unit * (long long)m * DK + idx];
+    sU[j * LU + i] = sc * fac_to_f(static_cast<const TS*>(p.U)[unit * (long long)m * DK + idx]);
   }
   for (int idx = threadIdx.x; idx < c * DV; idx += NT) {
     const int j = idx / DV, i = idx - j * DV;
-    sV[j * LV + i] = p.V[unit * (long long)m * DV + idx];
+    sV[j * LV + i] = fac_to_f(static_cast<const TS*>(p.V)[unit * (long long)m * DV + idx]);
   }
   for (int i = threadIdx.x; i < DK; i += NT) s_a[i] = p.a[unit * DK + i];
   for (int i = threadIdx.x; i < DV; i += NT) s_vb[i] = p.vbar[((long long)l * p.H + h) * DV + i];
@@ -125,20 +125,30 @@ __global__ void __launch_bounds__(kEnergyThreads) energy_kernel(const EnergyPara
   }
 }
 
-template <int DK, int DV>
-static int launch_energy_t(const EnergyParams& p, int blocks, cudaStream_t st) {
+template <int DK, int DV, typename TS>
+static int launch_energy_tt(const EnergyParams& p, int blocks, cudaStream_t st) {
   const size_t smem = ((size_t)(p.R + p.W) * (DK + 1 + DV + 1) + DK + DV) * sizeof(float);
-  auto kern = energy_kernel<DK, DV>;
+  auto kern = energy_kernel<DK, DV, TS>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SEED_ERR_CUDA;
   kern<<<blocks, kEnergyThreads, smem, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? SEED_OK : SEED_ERR_CUDA;
 }
 
+template <int DK, int DV>
+static int launch_energy_t(const EnergyParams& p, int blocks, cudaStream_t st) {
+  switch (p.factors) {
+    case SEED_FACTORS_F32: return launch_energy_tt<DK, DV, float>(p, blocks, st);
+    case SEED_FACTORS_F16: return launch_energy_tt<DK, DV, __half>(p, blocks, st);
+    case SEED_FACTORS_BF16: return launch_energy_tt<DK, DV, __nv_bfloat16>(p, blocks, st);
+  }
+  return SEED_ERR_INVALID_ARG;
+}
+
 int launch_state_energy(const seed_dims& d, const seed_state& s, int layer, const int32_t* units,
                         int n_units, float* out, uint32_t* status, cudaStream_t st) {
   EnergyParams p{s.a, s.U, s.V, s.scale, s.ncols, s.vbar, units, out, status,
-                 d.batch, d.layers, d.heads, layer, d.R, d.W, d.form, scale_len(d)};
+                 d.batch, d.layers, d.heads, layer, d.R, d.W, d.form, scale_len(d), d.factors};
   if (d.d_k == 16 && d.d_v == 16) return launch_energy_t<16, 16>(p, n_units, st);
   if (d.d_k == 32 && d.d_v == 32) return launch_energy_t<32, 32>(p, n_units, st);
   if (d.d_k == 64 && d.d_v == 64) return launch_energy_t<64, 64>(p, n_units, st);

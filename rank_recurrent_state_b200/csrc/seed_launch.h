@@ -2,6 +2,8 @@
 // Arguments are validated by seed_abi.cu before any of these is called.
 #pragma once
 
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -14,6 +16,20 @@ namespace seed {
 // R + W rounded up to a multiple of 4 (column scales, 16-byte aligned per unit).
 inline int scale_len(const seed_dims& d) {
   return d.form == SEED_KDA ? d.d_k : ((d.R + d.W + 3) & ~3);
+}
+
+// Bytes of one element of U and V.
+inline int factor_bytes(const seed_dims& d) { return d.factors == SEED_FACTORS_F32 ? 4 : 2; }
+
+// f(T{}) with T the element type of U and V (float, __half or __nv_bfloat16).
+template <typename F>
+int with_factor_type(const seed_dims& d, F&& f) {
+  switch (d.factors) {
+    case SEED_FACTORS_F32: return f(float{});
+    case SEED_FACTORS_F16: return f(__half{});
+    case SEED_FACTORS_BF16: return f(__nv_bfloat16{});
+  }
+  return SEED_ERR_INVALID_ARG;
 }
 
 bool decode_dims_supported(int dk, int dv);

@@ -42,6 +42,15 @@ SEED_DEV void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar
       : "memory");
 }
 
+// Ampere-style asynchronous 16-byte copy global -> shared (no mbarrier): groups
+// are committed in order and waited for by count; each thread waits for its own.
+SEED_DEV void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+SEED_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+SEED_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 // Tiled 3-D tensor copy global -> shared through a tensor map (no multicast),
 // completing on `bar`; coordinates innermost first.  The innermost coordinate x
 // times the element size must be a multiple of 16 bytes.

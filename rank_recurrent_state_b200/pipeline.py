@@ -21,9 +21,10 @@ class DeviceRun:
     """One workload resident on the device: v̄, the stored state and a workspace."""
 
     def __init__(self, cfg, batch: int | None = None, b0: int = 0, device: str = "cuda",
-                 n_prefill: int | None = None, keep_dense: bool = False, ragged: bool = False):
+                 n_prefill: int | None = None, keep_dense: bool = False, ragged: bool = False,
+                 factors: int = S.SEED_FACTORS_F32):
         self.cfg = cfg
-        self.dims = S.Dims.from_config(cfg, batch)
+        self.dims = S.Dims.from_config(cfg, batch, factors)
         self.key = S.synth_key(cfg, b0)
         self.device = device
         d = self.dims
@@ -73,7 +74,7 @@ class DeviceRun:
             nb = int((self.phase > j).sum())
             if nb == 0:
                 break
-            dj = S.Dims(d.form, nb, d.layers, d.heads, d.d_k, d.d_v, d.R, d.W)
+            dj = S.Dims(d.form, nb, d.layers, d.heads, d.d_k, d.d_v, d.R, d.W, d.factors)
             bj = {k: (None if x is None else x[:nb]) for k, x in buf.items()}
             for l in range(d.layers):
                 S.seed_synth_token_inputs(dj, self.key, S.SEED_PHASE_LEADIN, j, l, self.vbar,

@@ -1,6 +1,8 @@
 """Algorithmic byte accounting of the decode step (host logic for measurement).
 
-Per head-step (one unit, one decode step, c columns held before the step), fp32:
+Per head-step (one unit, one decode step, c columns held before the step), fp32
+(with 16-bit factors, fb = 2 bytes per U and V value instead of 4; the sink, the
+scales and the dense state stay fp32):
 
   lazy (the layout libseed uses)
     GDN, Mamba-2  4 [ d_k + (d_k + d_v + 1) c + d_k + d_k + d_v + (c + 1) ]
@@ -26,18 +28,21 @@ from __future__ import annotations
 FORM_KDA = 1
 
 
-def lazy_bytes(form: int, d_k: int, d_v: int, c: float) -> float:
+def lazy_bytes(form: int, d_k: int, d_v: int, c: float, fb: int = 4) -> float:
+    """a read and written (4 d_k each), the c stored columns of U and V read and one
+    new pair written (fb bytes a value), and the decay state read and written."""
+    factors = fb * ((d_k + d_v) * c + d_k + d_v)
     if form == FORM_KDA:
-        return 4.0 * (d_k + (d_k + d_v) * c + d_k + d_k + d_v + 2 * d_k)
-    return 4.0 * (d_k + (d_k + d_v + 1) * c + d_k + d_k + d_v + (c + 1))
+        return factors + 4.0 * (2 * d_k + 2 * d_k)
+    return factors + 4.0 * (2 * d_k + c + (c + 1))
 
 
-def explicit_bytes(d_k: int, d_v: int, c: float) -> float:
-    return 4.0 * (d_k + (d_k + d_v) * c + d_k + d_k * c + d_k + d_v)
+def explicit_bytes(d_k: int, d_v: int, c: float, fb: int = 4) -> float:
+    return fb * ((d_k + d_v) * c + d_k * c + d_k + d_v) + 4.0 * 2 * d_k
 
 
-def table2_bytes(d_k: int, d_v: int, R: int, W: int) -> float:
-    return 2 * 4.0 * (d_k + (d_k + d_v) * (R + W / 2))
+def table2_bytes(d_k: int, d_v: int, R: int, W: int, fb: int = 4) -> float:
+    return 2 * (4.0 * d_k + fb * (d_k + d_v) * (R + W / 2))
 
 
 def dense_bytes(d_k: int, d_v: int) -> float:

@@ -20,6 +20,10 @@ SEED_GDN, SEED_KDA, SEED_MAMBA2 = 0, 1, 2
 SEED_ALL_LAYERS = -1
 SEED_PHASE_PREFILL, SEED_PHASE_DECODE, SEED_PHASE_LEADIN = 0, 1, 2
 SEED_MAX_COLS = 96
+SEED_FACTORS_F32, SEED_FACTORS_F16, SEED_FACTORS_BF16 = 0, 1, 2
+FACTOR_DTYPES = {SEED_FACTORS_F32: torch.float32, SEED_FACTORS_F16: torch.float16,
+                 SEED_FACTORS_BF16: torch.bfloat16}
+FACTOR_NAMES = {"f32": SEED_FACTORS_F32, "f16": SEED_FACTORS_F16, "bf16": SEED_FACTORS_BF16}
 
 FLAG_FULL = 0x1
 FLAG_NONFINITE = 0x2
@@ -48,6 +52,7 @@ class Dims:
     d_v: int
     R: int
     W: int
+    factors: int = SEED_FACTORS_F32   # element type of U and V
 
     @property
     def m(self) -> int:
@@ -59,12 +64,16 @@ class Dims:
 
     def c(self) -> _lib.seed_dims:
         return _lib.seed_dims(self.form, self.batch, self.layers, self.heads, self.d_k, self.d_v,
-                              self.R, self.W)
+                              self.R, self.W, self.factors)
+
+    @property
+    def factor_dtype(self) -> torch.dtype:
+        return FACTOR_DTYPES[self.factors]
 
     @staticmethod
-    def from_config(cfg, batch: int | None = None) -> "Dims":
+    def from_config(cfg, batch: int | None = None, factors: int = SEED_FACTORS_F32) -> "Dims":
         return Dims(cfg.form, cfg.batch if batch is None else batch, cfg.layers, cfg.heads,
-                    cfg.d_k, cfg.d_v, cfg.R, cfg.W)
+                    cfg.d_k, cfg.d_v, cfg.R, cfg.W, factors)
 
 
 def _ptr(t) -> int | None:
@@ -94,8 +103,8 @@ def _check(fn: str, rc: int) -> None:
 class State:
     """Device tensors of the stored state (layouts as in seed.h)."""
     a: torch.Tensor          # [B][L][H][d_k]
-    U: torch.Tensor          # [B][L][H][R+W][d_k]
-    V: torch.Tensor          # [B][L][H][R+W][d_v]
+    U: torch.Tensor          # [B][L][H][R+W][d_k], element type dims.factor_dtype
+    V: torch.Tensor          # [B][L][H][R+W][d_v], same
     scale: torch.Tensor      # [B][L][H][ceil4(R+W)] (GDN, Mamba-2) or [B][L][H][d_k] (KDA)
     ncols: torch.Tensor      # [B][L][H] int32
     vbar: torch.Tensor       # [L][H][d_v]
@@ -110,9 +119,10 @@ class State:
         B, L, H = dims.batch, dims.layers, dims.heads
         slen = dims.d_k if dims.form == SEED_KDA else (dims.m + 3) // 4 * 4
         f32 = dict(dtype=torch.float32, device=dev)
+        fac = dict(dtype=FACTOR_DTYPES[dims.factors], device=dev)
         return State(a=torch.zeros(B, L, H, dims.d_k, **f32),
-                     U=torch.zeros(B, L, H, dims.m, dims.d_k, **f32),
-                     V=torch.zeros(B, L, H, dims.m, dims.d_v, **f32),
+                     U=torch.zeros(B, L, H, dims.m, dims.d_k, **fac),
+                     V=torch.zeros(B, L, H, dims.m, dims.d_v, **fac),
                      scale=torch.ones(B, L, H, slen, **f32),
                      ncols=torch.zeros(B, L, H, dtype=torch.int32, device=dev),
                      vbar=vbar)

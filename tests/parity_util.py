@@ -28,14 +28,15 @@ def ensure_lib():
     assert torch.cuda.is_available(), "GPU tests need CUDA"
 
 
-def run_device(cfg, sample_units, n_prefill, n_decode, batch=None):
+def run_device(cfg, sample_units, n_prefill, n_decode, batch=None, factors=0):
     """Run prefill, conversion and n_decode steps of every unit of (cfg, batch) on the
-    device; return the trajectories of the sampled global units as numpy arrays."""
+    device; return the trajectories of the sampled global units as numpy arrays.
+    factors: storage format of U and V (seed_factors)."""
     import torch
     from rank_recurrent_state_b200 import seed as S
     from rank_recurrent_state_b200.pipeline import DeviceRun
 
-    run = DeviceRun(cfg, batch=batch, n_prefill=n_prefill)
+    run = DeviceRun(cfg, batch=batch, n_prefill=n_prefill, factors=factors)
     d = run.dims
     run.prefill_and_convert()
     su = np.asarray(sample_units, dtype=np.int64)

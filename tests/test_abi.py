@@ -80,6 +80,8 @@ def test_scale_len_and_workspace(lib):
 @pytest.mark.parametrize("dims,code", [
     (None, -1),
     (_dims(form=3), -1),
+    (_dims(factors=3), -1),                     # no such factor format
+    (_dims(factors=-1), -1),
     (_dims(batch=0), -1),
     (_dims(R=0), -1),
     (_dims(d_k=48), -2),
