@@ -60,6 +60,9 @@ def parse_args(argv=None):
                          "back only after its old copy has decayed)")
     ap.add_argument("--factors", default="f32", choices=["f32", "f16", "bf16"],
                     help="storage format of the factors U and V (arithmetic stays f32)")
+    ap.add_argument("--fused", action="store_true",
+                    help="compress inside the decode launch of the step that fills R + W "
+                         "(seed_decode_step_compress) instead of a separate compression launch")
     ap.add_argument("--ragged", action="store_true",
                     help="ragged compression schedules: requests joined at different times, a "
                          "compression launch after every step compresses the units that are due")
@@ -230,7 +233,7 @@ def cpu_oracle_rate(cfg, seconds: float, rank_seed: int = 0) -> dict:
             "affinity_cores": len(os.sched_getaffinity(0))}
 
 
-def config_obj(cfg, batch, world, prefill, ragged=False, factors="f32"):
+def config_obj(cfg, batch, world, prefill, ragged=False, factors="f32", fused=False):
     schedule = ("ragged: request b joined W-1-floor(bW/B) steps before the others; a compression "
                 "launch after every step compresses the units that are due" if ragged else
                 "lockstep: every unit compresses after steps W, 2W, ...")
@@ -241,6 +244,8 @@ def config_obj(cfg, batch, world, prefill, ragged=False, factors="f32"):
             "batch_per_gpu": batch, "global_batch": batch * world, "prefill_tokens": prefill,
             "parallelism": f"dp{world} (requests sharded, no collective)",
             "schedule": schedule,
+            "compression": ("fused into the decode launch of the step that fills R + W" if fused
+                            else "a separate launch over all units after the step that fills R + W"),
             "factors": factors + (" (U and V stored in 16 bits, rounded to nearest when written)"
                                   if factors != "f32" else ""),
             "l2": "inputs and state larger than L2 (no flush needed)"}
@@ -362,8 +367,17 @@ def run_ours(args, world, rank, local):
 
     def one_step(s, ev=None):
         t = s % P
+        fuse = args.fused and (args.ragged or run.c + 1 == d.m)
         for l in range(L):
             qq, kk, vv, aa, bb = inputs(t, l)
+            if fuse:
+                if ev is not None:
+                    ev["fus"].append((torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)))
+                    ev["fus"][-1][0].record(stream)
+                S.seed_decode_step_compress(d, run.state, l, qq, kk, vv, aa, bb, o[l], run.ws, stream=stream)
+                if ev is not None:
+                    ev["fus"][-1][1].record(stream)
+                continue
             if ev is not None:
                 ev["dec"].append((torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
                                   roofline.mean_columns(d.R, d.W) if args.ragged else run.c))
@@ -372,7 +386,9 @@ def run_ours(args, world, rank, local):
             if ev is not None:
                 ev["dec"][-1][1].record(stream)
         run.c += 1
-        if run.c == d.m or args.ragged:
+        if fuse:
+            run.c = d.R if run.c == d.m else run.c
+        elif run.c == d.m or args.ragged:
             if ev is not None:
                 ev["cmp"].append((torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)))
                 ev["cmp"][-1][0].record(stream)
@@ -386,7 +402,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     flags_warm = S.seed_get_status(run.ws)
 
-    ev = {"dec": [], "cmp": []}
+    ev = {"dec": [], "cmp": [], "fus": []}
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     visible = [x for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
     gpu_index = int(visible[local]) if len(visible) > local and visible[local].isdigit() else local
@@ -408,7 +424,8 @@ def run_ours(args, world, rank, local):
     dec_ms = [a.elapsed_time(b) for a, b, _ in ev["dec"]]
     dec_bytes = [BH * roofline.lazy_bytes(d.form, d.d_k, d.d_v, c, fb) for _, _, c in ev["dec"]]
     cmp_ms = [a.elapsed_time(b) for a, b in ev["cmp"]]
-    dec_gbs = sum(dec_bytes) / (sum(dec_ms) / 1e3) / 1e9
+    # (with --fused --ragged every launch is a fused one: no plain decode launch to time)
+    dec_gbs = sum(dec_bytes) / (sum(dec_ms) / 1e3) / 1e9 if dec_ms else None
     peak, peak_kind = measured_peak_hbm()
     cbar = roofline.mean_columns(d.R, d.W)
 
@@ -417,14 +434,16 @@ def run_ours(args, world, rank, local):
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded Philox4x32-10 inputs and prefill, generated on the device)",
-        "config": config_obj(cfg, B, world, prefill, args.ragged, args.factors),
+        "config": config_obj(cfg, B, world, prefill, args.ragged, args.factors, args.fused),
         "roofline": {"bound": "hbm", "kernel": decode_kernel_name(d), "achieved": dec_gbs, "peak": peak,
-                     "unit": "GB/s", "frac": dec_gbs / peak, "peak_source": f"{peak_kind} copy bandwidth",
-                     "frac_of_nominal_8TBs": dec_gbs / NOMINAL_HBM_GBS,
+                     "unit": "GB/s", "frac": dec_gbs / peak if dec_ms else None,
+                     "peak_source": f"{peak_kind} copy bandwidth",
+                     "frac_of_nominal_8TBs": dec_gbs / NOMINAL_HBM_GBS if dec_ms else None,
                      "traffic": decode_traffic(d, BH, cbar),
                      "algorithmic_bytes_per_head_step_mean": roofline.lazy_bytes(d.form, d.d_k, d.d_v, cbar, fb),
-                     "avg_launch_us": 1e3 * sum(dec_ms) / len(dec_ms), "launches": len(dec_ms)},
-        "decode_only": {"head_steps_per_s": len(dec_ms) * BH * world / (sum(dec_ms) / 1e3),
+                     "avg_launch_us": 1e3 * sum(dec_ms) / len(dec_ms) if dec_ms else None,
+                     "launches": len(dec_ms)},
+        "decode_only": {"head_steps_per_s": len(dec_ms) * BH * world / (sum(dec_ms) / 1e3) if dec_ms else None,
                         "GBps": dec_gbs},
         "compress": {"launches": len(cmp_ms), "ms_per_launch": (sum(cmp_ms) / len(cmp_ms)) if cmp_ms else None,
                      "ns_per_head_step_amortized": 1e6 * sum(cmp_ms) / (args.steps * units) if cmp_ms else 0.0,
@@ -433,10 +452,17 @@ def run_ours(args, world, rank, local):
                                             if diag["compress_units"] else None),
                      "cholqr_units": diag["cholqr_units"], "householder_units": diag["householder_units"],
                      **compress_rate(d, diag, cmp_ms, clk.summary())},
-        "gpu_launches": len(dec_ms) + len(cmp_ms),
+        "gpu_launches": len(dec_ms) + len(cmp_ms) + len(ev["fus"]),
         "status_flags": flags | flags_warm,
         "setup_s": t_setup,
     }
+    if ev["fus"]:
+        fus_ms = [a.elapsed_time(b) for a, b in ev["fus"]]
+        line["fused"] = {"launches": len(fus_ms), "ms_per_launch": sum(fus_ms) / len(fus_ms),
+                         "share_of_step": sum(fus_ms) / elapsed_ms,
+                         "note": "decode step of one layer with the compression of its due units "
+                                 "(seed_decode_step_compress); the Householder launch for declined "
+                                 "units is included"}
     clocks = clk.summary()
     line["clocks"] = clocks
 
@@ -504,6 +530,7 @@ def run_ours(args, world, rank, local):
         n = 0
         for s in range(args.e2e_steps):
             t = s % Ph
+            fuse = args.fused and (args.ragged or run.c + 1 == d.m)
             for l in range(L):
                 bi = n % nb
                 bq, bk, bv, ba, bb = bufs[bi]
@@ -517,8 +544,8 @@ def run_ours(args, world, rank, local):
                 stream.wait_event(ev_in[bi])
                 if s > 0:
                     stream.wait_event(ev_out[l])   # last step's o of this layer is out
-                S.seed_decode_step(d, run.state, l, bq, bk, bv, ba if kda else ba[:BH], bb[:BH], o[l],
-                                   run.ws, stream)
+                step_fn = S.seed_decode_step_compress if fuse else S.seed_decode_step
+                step_fn(d, run.state, l, bq, bk, bv, ba if kda else ba[:BH], bb[:BH], o[l], run.ws, stream=stream)
                 ev_free[bi].record(stream)
                 ev_dec[l].record(stream)
                 with torch.cuda.stream(s_out):
@@ -527,8 +554,9 @@ def run_ours(args, world, rank, local):
                     ev_out[l].record(s_out)
                 n += 1
             run.c += 1
-            if run.c == d.m:
-                S.seed_compress(d, run.state, S.SEED_ALL_LAYERS, run.ws, stream=stream)
+            if run.c == d.m or args.ragged:   # ragged: some request is due after every step
+                if not fuse:
+                    S.seed_compress(d, run.state, S.SEED_ALL_LAYERS, run.ws, stream=stream)
                 run.c = d.R
         stream.wait_stream(s_out)
         stream.wait_stream(s_in)

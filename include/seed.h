@@ -189,6 +189,23 @@ int seed_decode_step(const seed_dims* dims, const seed_state* state, int32_t lay
 int seed_compress(const seed_dims* dims, const seed_state* state, int32_t layer,
                   float* sigma_out, void* ws, size_t ws_bytes, void* stream);
 
+/* One decode step of one layer (as seed_decode_step) fused with the compression of
+ * the units it brings to R + W columns (as seed_compress on that layer): call it
+ * instead of seed_decode_step for the step after which a compression is due (every
+ * step with ragged per-request schedules); no separate seed_compress is needed.
+ * Where R + W <= 32, R <= 16 and d_k, d_v are in {64, 128}, one launch does both:
+ * the warp that stepped a unit compresses it right away (SEED figures & tables,
+ * Figure 1(b): the step, then every W steps the compression), its columns read
+ * again from L2 instead of HBM; units that launch's Cholesky-QR path declines are
+ * compressed by the Householder path in a second launch over the layer.  Other
+ * shapes: a decode launch and a compression launch.  Results, their storage and
+ * the errors as with seed_decode_step followed by seed_compress(layer).
+ *   sigma_out  optional: [B * H][R] singular values kept (rows of compressed units)  */
+int seed_decode_step_compress(const seed_dims* dims, const seed_state* state, int32_t layer,
+                              const float* q, const float* k, const float* v, const float* alpha,
+                              const float* beta, float* o, float* sigma_out, void* ws,
+                              size_t ws_bytes, void* stream);
+
 /* Dense state S = a vbar^T + U V^T (true U, scales applied) of units of `layer`
  * (or all layers).  units: optional list of unit indices within the scope
  * (b * H + h for one layer, the global unit index for all layers); NULL = every

@@ -44,6 +44,9 @@ SIGNATURES = {
                                         c_void_p, c_size_t, c_void_p]),
     "seed_compress": (ctypes.c_int, [ctypes.POINTER(seed_dims), ctypes.POINTER(seed_state), c_int32,
                                      c_void_p, c_void_p, c_size_t, c_void_p]),
+    "seed_decode_step_compress": (ctypes.c_int, [ctypes.POINTER(seed_dims), ctypes.POINTER(seed_state), c_int32,
+                                                 c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                                 c_void_p, c_void_p, c_size_t, c_void_p]),
     "seed_state_to_dense": (ctypes.c_int, [ctypes.POINTER(seed_dims), ctypes.POINTER(seed_state), c_int32,
                                            c_void_p, c_int32, c_void_p, c_void_p, c_size_t, c_void_p]),
     "seed_state_energy": (ctypes.c_int, [ctypes.POINTER(seed_dims), ctypes.POINTER(seed_state), c_int32,

@@ -396,6 +396,11 @@ int launch_compress(const seed_dims& d, const seed_state& s, int layer, float* s
     const int rc = launch_compress_fast(d, s, layer, sigma_out, status, st);
     if (rc != SEED_OK) return rc;
   }
+  return launch_compress_householder(d, s, layer, sigma_out, status, st);
+}
+
+int launch_compress_householder(const seed_dims& d, const seed_state& s, int layer, float* sigma_out,
+                                uint32_t* status, cudaStream_t st) {
   CompressParams p{s.U, s.V, s.scale, s.ncols, sigma_out, status,
                    d.batch, d.layers, d.heads, layer, d.R, d.W, scale_len(d)};
   const int blocks = d.batch * d.heads * (layer < 0 ? d.layers : 1);

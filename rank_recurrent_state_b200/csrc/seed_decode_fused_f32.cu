@@ -1,0 +1,10 @@
+// seed_decode_fused_f32.cu -- the fused decode-and-compress kernels for float factors.
+#include "seed_decode_fused.cuh"
+
+namespace seed {
+
+int launch_fused_f32(const seed_dims& d, const DecodeParams& p, const FastParams& fp, cudaStream_t st) {
+  return launch_fused_typed<float>(d, p, fp, st);
+}
+
+}  // namespace seed

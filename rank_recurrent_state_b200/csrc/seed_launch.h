@@ -45,6 +45,17 @@ int launch_compress_fast(const seed_dims& d, const seed_state& s, int layer, flo
 int launch_compress(const seed_dims& d, const seed_state& s, int layer, float* sigma_out,
                     uint32_t* status, cudaStream_t st);
 
+// The Householder compression alone (the units still holding R + W columns).
+int launch_compress_householder(const seed_dims& d, const seed_state& s, int layer, float* sigma_out,
+                                uint32_t* status, cudaStream_t st);
+
+// The decode step of one layer with the compression of the units it brings to
+// R + W columns (seed_decode_fused.cu).
+bool decode_compress_fused_supported(const seed_dims& d);
+int launch_decode_compress(const seed_dims& d, const seed_state& s, int layer, const float* q, const float* k,
+                           const float* v, const float* alpha, const float* beta, float* o, float* sigma_out,
+                           uint32_t* status, cudaStream_t st);
+
 int launch_init_from_dense(const seed_dims& d, const seed_state& s, int layer, const float* S,
                            float* sigma_out, uint32_t* status, cudaStream_t st);
 

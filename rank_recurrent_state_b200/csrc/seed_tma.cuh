@@ -21,6 +21,8 @@ SEED_DEV void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.clus
 // async-proxy (bulk copy) accesses, e.g. before a copy overwrites a buffer that was
 // just written with ordinary stores.
 SEED_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// Orders this thread's ordinary global writes before later async-proxy (TMA) reads.
+SEED_DEV void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
 SEED_DEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),

@@ -4,7 +4,9 @@ prefill (synthetic, dense) -> seed_state_init_from_dense -> per step and layer:
 seed_synth_token_inputs + seed_decode_step, and seed_compress after the step that
 fills R + W columns ("every W steps", decode steps counted from 1).  With ragged
 schedules the requests joined at different times (a lead-in of up to W - 1 steps)
-and seed_compress runs after every step, compressing the units that are due.
+and seed_compress runs after every step, compressing the units that are due.  With
+fused=True the step after which a compression is due (every step when ragged) is
+seed_decode_step_compress, which compresses the due units inside the decode launch.
 
 Every step of the path runs in libseed's kernels; this module only allocates
 tensors, orders the calls and tracks the (uniform) column count on the host.
@@ -22,7 +24,7 @@ class DeviceRun:
 
     def __init__(self, cfg, batch: int | None = None, b0: int = 0, device: str = "cuda",
                  n_prefill: int | None = None, keep_dense: bool = False, ragged: bool = False,
-                 factors: int = S.SEED_FACTORS_F32):
+                 factors: int = S.SEED_FACTORS_F32, fused: bool = False):
         self.cfg = cfg
         self.dims = S.Dims.from_config(cfg, batch, factors)
         self.key = S.synth_key(cfg, b0)
@@ -42,6 +44,7 @@ class DeviceRun:
         # others, phi_b = W - 1 - floor(b W / B) for the workload's B requests, so the
         # requests still in their lead-in at lead-in step j are a prefix of the batch
         self.ragged = ragged
+        self.fused = fused
         gb = torch.arange(b0, b0 + self.dims.batch)
         self.phase = (cfg.W - 1 - (gb * cfg.W) // cfg.batch).clamp(min=0) if ragged else torch.zeros_like(gb)
 
@@ -92,10 +95,22 @@ class DeviceRun:
         """One decode step of every layer (inputs generated on the device), then the
         compression if it is due.  Returns True when a compression ran."""
         d = self.dims
+        fuse = self.fused and (self.ragged or self.c + 1 == d.m)
+        sig_l = None
+        if fuse and sigma is not None:
+            sig_l = torch.empty(d.batch * d.heads, d.R, dtype=torch.float32, device=self.device)
         for l in range(d.layers):
             self.gen_inputs(self.t, l, buf)
-            S.seed_decode_step(d, self.state, l, buf["q"], buf["k"], buf["v"], buf["alpha"],
-                               buf["beta"], buf["o"], self.ws)
+            if fuse:
+                if sig_l is not None:   # keep the rows of units this step does not compress
+                    sig_l.copy_(sigma.view(d.batch, d.layers, d.heads, d.R)[:, l].reshape(-1, d.R))
+                S.seed_decode_step_compress(d, self.state, l, buf["q"], buf["k"], buf["v"], buf["alpha"],
+                                            buf["beta"], buf["o"], self.ws, sigma_out=sig_l)
+                if sig_l is not None:
+                    sigma.view(d.batch, d.layers, d.heads, d.R)[:, l] = sig_l.view(d.batch, d.heads, d.R)
+            else:
+                S.seed_decode_step(d, self.state, l, buf["q"], buf["k"], buf["v"], buf["alpha"],
+                                   buf["beta"], buf["o"], self.ws)
             if dense and self.dense is not None:
                 S.seed_dense_step(d, self.dense, l, buf["q"], buf["k"], buf["v"], buf["alpha"],
                                   buf["beta"], buf["o_dense"], self.ws)
@@ -104,10 +119,12 @@ class DeviceRun:
         self.c += 1
         self.t += 1
         if self.ragged:   # some request is due after every step: only its units compress
-            S.seed_compress(d, self.state, S.SEED_ALL_LAYERS, self.ws, sigma_out=sigma)
+            if not fuse:
+                S.seed_compress(d, self.state, S.SEED_ALL_LAYERS, self.ws, sigma_out=sigma)
             return True
         if self.c == d.m:
-            S.seed_compress(d, self.state, S.SEED_ALL_LAYERS, self.ws, sigma_out=sigma)
+            if not fuse:
+                S.seed_compress(d, self.state, S.SEED_ALL_LAYERS, self.ws, sigma_out=sigma)
             self.c = d.R
             return True
         return False

@@ -184,6 +184,16 @@ def seed_decode_step_noalloc(dims: Dims, state: State, layer: int, q, k, v, alph
         _ptr(o), _ptr(status_out), _stream(stream)))
 
 
+def seed_decode_step_compress(dims: Dims, state: State, layer: int, q, k, v, alpha, beta, o,
+                              ws: Workspace, sigma_out: torch.Tensor | None = None, stream=None) -> None:
+    """seed_decode_step fused with the compression of the units the step brings to
+    R + W columns; sigma_out [B * H][R] (rows of compressed units written)."""
+    d, s = dims.c(), state.c()
+    _check("seed_decode_step_compress", _lib.load().seed_decode_step_compress(
+        ctypes.byref(d), ctypes.byref(s), layer, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+        _ptr(o), _ptr(sigma_out), ws.ptr, ws.nbytes, _stream(stream)))
+
+
 def seed_noalloc_workspace_bytes() -> int:
     return int(_lib.load().seed_noalloc_workspace_bytes())
 

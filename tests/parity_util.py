@@ -28,15 +28,16 @@ def ensure_lib():
     assert torch.cuda.is_available(), "GPU tests need CUDA"
 
 
-def run_device(cfg, sample_units, n_prefill, n_decode, batch=None, factors=0):
+def run_device(cfg, sample_units, n_prefill, n_decode, batch=None, factors=0, fused=False):
     """Run prefill, conversion and n_decode steps of every unit of (cfg, batch) on the
     device; return the trajectories of the sampled global units as numpy arrays.
-    factors: storage format of U and V (seed_factors)."""
+    factors: storage format of U and V (seed_factors); fused: compress inside the
+    decode launch of the step that fills R + W (seed_decode_step_compress)."""
     import torch
     from rank_recurrent_state_b200 import seed as S
     from rank_recurrent_state_b200.pipeline import DeviceRun
 
-    run = DeviceRun(cfg, batch=batch, n_prefill=n_prefill, factors=factors)
+    run = DeviceRun(cfg, batch=batch, n_prefill=n_prefill, factors=factors, fused=fused)
     d = run.dims
     run.prefill_and_convert()
     su = np.asarray(sample_units, dtype=np.int64)
@@ -66,7 +67,7 @@ def run_device(cfg, sample_units, n_prefill, n_decode, batch=None, factors=0):
                 b=b, l=l, h=h)
 
 
-def run_device_ragged(cfg, sample_units, n_prefill, n_decode, batch=None):
+def run_device_ragged(cfg, sample_units, n_prefill, n_decode, batch=None, fused=False):
     """Like run_device, with ragged compression schedules: requests joined the batch at
     different times (DeviceRun's lead-in) and every step ends with a compression of the
     units that are due.  Returns the trajectories of the sampled units plus, per unit,
@@ -75,7 +76,7 @@ def run_device_ragged(cfg, sample_units, n_prefill, n_decode, batch=None):
     from rank_recurrent_state_b200 import seed as S
     from rank_recurrent_state_b200.pipeline import DeviceRun
 
-    run = DeviceRun(cfg, batch=batch, n_prefill=n_prefill, ragged=True)
+    run = DeviceRun(cfg, batch=batch, n_prefill=n_prefill, ragged=True, fused=fused)
     d = run.dims
     run.prefill_and_convert()
     su = np.asarray(sample_units, dtype=np.int64)

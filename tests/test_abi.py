@@ -129,6 +129,20 @@ def test_other_entry_points_validate(lib):
     assert lib.seed_synth_dense_prefill(ctypes.byref(d), bad_key, 4, 0, A, A, None) == -1
 
 
+def test_fused_decode_compress_validates(lib):
+    d, s = _dims(), _state()
+    call = lambda layer=0, q=A, sig=None, wsb=256: lib.seed_decode_step_compress(  # noqa: E731
+        ctypes.byref(d), ctypes.byref(s), layer, q, A, A, A, A, A, sig, A, wsb, None)
+    assert call(layer=-1) == -1                  # one layer per call
+    assert call(layer=3) == -1
+    assert call(q=MIS) == -3
+    assert call(sig=MIS) == -3
+    assert call(wsb=8) == -5
+    bad = _dims(factors=7)
+    assert lib.seed_decode_step_compress(ctypes.byref(bad), ctypes.byref(s), 0, A, A, A, A, A, A, None, A, 256,
+                                         None) == -1
+
+
 def test_noalloc_decode_step_validates_before_touching_the_device(lib):
     d, s = _dims(), _state()
     assert lib.seed_noalloc_workspace_bytes() >= lib.seed_workspace_bytes(ctypes.byref(d))
