@@ -39,8 +39,12 @@ NOMINAL_HBM_GBS = 8000.0
 # (dram__bytes_read.sum + dram__bytes_write.sum; profiles/decode_warp_kernel_gdn_stack_2layers.md):
 # a full per-layer launch (256 requests x 48 heads) at c = 19 stored columns.  Set to None
 # whenever the decode kernel changes until it is measured again.
-NCU_DECODE_TRAFFIC = {"kernel": "decode_warp_kernel", "form": 0, "d_k": 128, "d_v": 128, "R": 16,
-                      "W": 16, "units": 12288, "c": 19, "bytes": 266.031e6 + 19.914e6}
+NCU_DECODE_TRAFFIC = [
+    {"kernel": "decode_warp_kernel", "form": 0, "d_k": 128, "d_v": 128, "R": 16, "W": 16, "factors": 0,
+     "units": 12288, "c": 19, "bytes": 266.032e6 + 20.088e6},
+    {"kernel": "decode_warp_kernel", "form": 0, "d_k": 128, "d_v": 128, "R": 16, "W": 16, "factors": 1,
+     "units": 12288, "c": 19, "bytes": 146.493e6 + 10.716e6},
+]
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -286,11 +290,14 @@ def decode_traffic(d, units, cbar):
     column count to this launch's by the state + input/output bytes; None when the
     capture does not match this kernel and shape."""
     from rank_recurrent_state_b200 import roofline
-    t = NCU_DECODE_TRAFFIC
-    if t is None or decode_kernel_name(d) != t["kernel"] or (d.form, d.d_k, d.d_v, d.R, d.W, d.factors) != (
-            t["form"], t["d_k"], t["d_v"], t["R"], t["W"], t.get("factors", 0)):
+    key = (decode_kernel_name(d), d.form, d.d_k, d.d_v, d.R, d.W, d.factors)
+    match = [t for t in NCU_DECODE_TRAFFIC
+             if (t["kernel"], t["form"], t["d_k"], t["d_v"], t["R"], t["W"], t["factors"]) == key]
+    if not match:
         return None
-    per = lambda c: roofline.lazy_bytes(d.form, d.d_k, d.d_v, c) + roofline.io_bytes(d.form, d.d_k, d.d_v)  # noqa: E731
+    t = match[0]
+    fb = 4 if d.factors == 0 else 2
+    per = lambda c: roofline.lazy_bytes(d.form, d.d_k, d.d_v, c, fb) + roofline.io_bytes(d.form, d.d_k, d.d_v)  # noqa: E731
     return t["bytes"] / t["units"] * units * per(cbar) / per(t["c"])
 
 

@@ -16,8 +16,10 @@
 
 namespace seed {
 
+// At most 168 registers a thread (12 warps per SM where shared memory allows, as
+// the compression wants); the body fits without spills.
 template <int FORM, int DK, int DV, int MAXC, typename TS, int MP>
-__global__ void __launch_bounds__(32)
+__global__ void __launch_bounds__(32, 12)
     decode_compress_warp_kernel(const DecodeParams p, const FastParams fp, const __grid_constant__ CUtensorMap tmU,
                                 const __grid_constant__ CUtensorMap tmV) {
   decode_warp_run<FORM, DK, DV, MAXC, TS, true, MP>(p, &fp, &tmU, &tmV);
