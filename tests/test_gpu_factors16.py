@@ -341,3 +341,31 @@ def test_trajectory_drift_matches_float32_factors(factors):
     # the sink a is never rounded: it follows its own float32 recurrence, and the
     # 16-bit content enters it only through omega, which does not involve U and V
     assert rel_fro(dev16["a"], dev32["a"]) <= TOL
+
+
+@pytest.mark.parametrize("factors", [F16, BF16], ids=["f16", "bf16"])
+def test_value_beyond_the_format_range_is_flagged(factors):
+    """A new V column beyond fp16's largest finite value (65504) is stored as +-inf
+    and raises SEED_FLAG_NONFINITE; bf16 has float32's range and stores it finite."""
+    import torch
+    from rank_recurrent_state_b200 import seed as S
+    rng = np.random.default_rng(5000 + factors)
+    n, dk, dv, R, W, c = 8, 128, 128, 16, 16, 20
+    host = _stored_state(FORM_GDN, n, dk, dv, R, W, c, rng, factors)
+    vbar = np.zeros(dv)
+    vbar[0] = 1.0
+    d, st, ws = _upload(FORM_GDN, n, dk, dv, R, W, factors, host, c, vbar)
+    inp = _step_inputs(FORM_GDN, n, dk, dv, vbar, rng)
+    inp["v"][:, 5] = 1e5          # orthogonal to vbar: lands in the new V column
+    inp["beta"][:] = 1.0
+    dev = {key: torch.from_numpy(val).cuda() for key, val in inp.items()}
+    o = torch.empty(n, dv, device="cuda")
+    S.seed_decode_step(d, st, 0, dev["q"], dev["k"], dev["v"], dev["alpha"], dev["beta"], o, ws)
+    flags = S.seed_get_status(ws)
+    col = st.V.reshape(n, R + W, dv)[:, c, 5].double().cpu().numpy()
+    if factors == F16:
+        assert flags & S.FLAG_NONFINITE
+        assert np.all(np.isinf(col))
+    else:
+        assert flags == 0
+        assert np.all(np.isfinite(col)) and np.all(np.abs(col) > 5e4)

@@ -21,14 +21,14 @@ def _lib():
     ensure_lib()
 
 
-def _twin_runs(cid, batch):
+def _twin_runs(cid, batch, factors=0):
     """Two device runs on one seeded workload: prefill + conversion, then the second
     run's state is made a bit-identical copy of the first's."""
     from rank_recurrent_state_b200.pipeline import DeviceRun
     cfg = configs.config(cid)
-    a = DeviceRun(cfg, batch=batch, n_prefill=24)
+    a = DeviceRun(cfg, batch=batch, n_prefill=24, factors=factors)
     a.prefill_and_convert()
-    b = DeviceRun(cfg, batch=batch, n_prefill=24)
+    b = DeviceRun(cfg, batch=batch, n_prefill=24, factors=factors)
     b.prefill_and_convert()
     b.state.load_state_dict(a.state.state_dict())
     return a, b
@@ -40,11 +40,11 @@ def _assert_same_state(sa, sb):
         assert torch.equal(getattr(sa, name), getattr(sb, name)), name
 
 
-@pytest.mark.parametrize("cid", [0, 2, 3, 4])
-def test_two_calls_in_a_row_match_the_workspace_entry_point(cid):
+@pytest.mark.parametrize("cid,factors", [(0, 0), (2, 0), (3, 0), (4, 0), (2, 1), (4, 2)])
+def test_two_calls_in_a_row_match_the_workspace_entry_point(cid, factors):
     import torch
     from rank_recurrent_state_b200 import seed as S
-    a, b = _twin_runs(cid, batch=4)
+    a, b = _twin_runs(cid, batch=4, factors=factors)
     d = a.dims
     status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
     for t in range(2):
