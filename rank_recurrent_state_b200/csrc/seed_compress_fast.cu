@@ -4,14 +4,28 @@
 
 namespace seed {
 
-// One warp per block and per unit of the scope.
+// One warp per block and per unit of the scope.  The kernel has no static shared
+// memory, so its dynamic shared memory starts the block's window, which is
+// allocated without alignment slack (more blocks per SM); a block that finds it
+// off a 1 KB boundary leaves its unit to the Householder kernel (counted with the
+// units the fast path declines) rather than misplace the swizzled buffers.
 template <int FORM, int DK, int DV, int MP, typename TS>
 __global__ void __launch_bounds__(32)
     compress_fast_kernel(const FastParams p, const __grid_constant__ CUtensorMap tmU,
                          const __grid_constant__ CUtensorMap tmV) {
+  using Lay = FastLayout<FORM, DK, DV, MP>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  float* sA = reinterpret_cast<float*>(smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023));
-  __shared__ __align__(8) uint64_t bar[2];
+  if (smem_addr(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) {
+      const int per = p.layer < 0 ? p.L * p.H : p.H;
+      const int b = blockIdx.x / per, rest = blockIdx.x - b * per;
+      const long long unit = p.layer < 0 ? (long long)blockIdx.x : ((long long)b * p.L + p.layer) * p.H + rest;
+      if (p.ncols[unit] == p.R + p.W) atomicAdd(p.status + 6, 1u);
+    }
+    return;
+  }
+  float* sA = reinterpret_cast<float*>(smem_raw);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem_raw + Lay::BAR_OFF);
   if (threadIdx.x == 0) {
     mbar_init(&bar[0], 1);
     mbar_init(&bar[1], 1);

@@ -507,23 +507,27 @@ SEED_DEV bool gram_stream(int c0, int c1, bool fold, float* sA, const CUtensorMa
 
 // Shared memory.  Region A first holds two 32-row chunk buffers through which the
 // panels stream (U chunks, then V chunks); after the V Gram it holds L_v, then M
-// in place of it, the selected left vectors X and Gram-Schmidt scratch, and at the
-// end the chunks of the panels again.  L_u has its own region, used from the U Gram
-// until the small right factors T_u and T_v replace it.
+// in place of it and the selected left vectors X, and at the end the chunks of the
+// panels again.  L_u has its own region, used from the U Gram until the small
+// right factors T_u and T_v replace it; the two chunk barriers come last.  Region A
+// must start on a 1 KB boundary (the 128-byte swizzle of the tensor copies).
 template <int FORM, int DK, int DV, int MP>
 struct FastLayout {
   static constexpr int CHUNK = MP * 32;                         // one swizzled chunk (MP x 128 B)
   static constexpr int LG = MP + 4, LX = MP + 1;
   static constexpr int SL = (FORM == SEED_KDA ? DK : MP);
-  static constexpr int OFF_M = 0, OFF_X = MP * LG, OFF_P = OFF_X + kFastMaxR * LX;
-  static constexpr int A_CH = 2 * CHUNK, A_B = OFF_P + kFastMaxR * LX;
-  static constexpr int A = ((A_CH > A_B ? A_CH : A_B) + 255) & ~255;   // keeps L_u 1 KB aligned
+  static constexpr int OFF_M = 0, OFF_X = MP * LG;
+  static constexpr int A_CH = 2 * CHUNK, A_B = OFF_X + kFastMaxR * LX;
+  static constexpr int A = ((A_CH > A_B ? A_CH : A_B) + 3) & ~3;
   static constexpr int LU = A;                                  // L_u (MP x LG), then T_u | T_v
   static constexpr int LU_N = (MP * LG > 2 * MP * kFastMaxR ? MP * LG : 2 * MP * kFastMaxR);
   static constexpr int SMALL = LU + LU_N;                       // nu nv du dv nrm, scl
   static constexpr int FLOATS = SMALL + 5 * MP + SL;
-  // + 1 KB: the dynamic shared memory is re-aligned to the 1 KB the swizzle needs
-  static constexpr size_t bytes = FLOATS * sizeof(float) + (MP + 4) * sizeof(int) + 1024;
+  static constexpr size_t BAR_OFF = FLOATS * sizeof(float) + (MP + 4) * sizeof(int);   // 8-byte aligned
+  static constexpr size_t bytes = BAR_OFF + 2 * sizeof(uint64_t);
+  // a block whose dynamic shared memory may start anywhere re-aligns region A
+  static constexpr size_t bytes_aligned = bytes + 1024;
+  static_assert(BAR_OFF % 8 == 0, "barrier alignment");
 };
 
 // Chunks 0 and 1 of a stream.
@@ -554,7 +558,6 @@ SEED_DEV bool compress_fast_unit(const FastParams& p, const CUtensorMap& tmU, co
   constexpr int NCU = DK / 32, NCV = DV / 32, NCH = NCU + NCV;
   float* sM = sA + Lay::OFF_M;       // L_v, then M (column-major), then T_u | T_v
   float* sX = sA + Lay::OFF_X;       // R x LX
-  float* sP = sA + Lay::OFF_P;       // R x LX scratch
   float* sLu = sA + Lay::LU;
   float* nu = sA + Lay::SMALL;
   float* nv = nu + MP;
@@ -689,7 +692,7 @@ SEED_DEV bool compress_fast_unit(const FastParams& p, const CUtensorMap& tmU, co
   //     the total) are left unrotated, so they need not be orthogonal to the
   //     others; when every selected sigma is above 1e-4 sigma_max none of them is
   //     such a column and the x_r are orthonormal as they are.  Otherwise they are
-  //     orthonormalised in descending order (classical Gram-Schmidt, two passes;
+  //     orthonormalised in descending order (modified Gram-Schmidt, two passes;
   //     lane = row), so that the result below is exactly the projection of U V^T on
   //     their span; a vector that loses more than half its norm to the earlier ones
   //     adds no new direction and is dropped.
@@ -707,17 +710,13 @@ SEED_DEV bool compress_fast_unit(const FastParams& p, const CUtensorMap& tmU, co
       const int j = sel[r];
       const float sj = nrm[j];
       float x = (lane < MP && sj > szero) ? sM[j * LG + lane] / sj : 0.f;
+#pragma unroll 1
       for (int pass = 0; pass < 2; ++pass) {
-        for (int k = 0; k < r; ++k)
-          if (lane < MP) sP[k * LX + lane] = x * sX[k * LX + lane];
-        __syncwarp();
-        float dk = 0.f;
-        if (lane < r)
-          for (int i = 0; i < MP; ++i) dk += sP[lane * LX + i];
-        __syncwarp();
-        for (int k = 0; k < r; ++k) {
-          const float d = __shfl_sync(kFull, dk, k);
-          if (lane < MP) x = fmaf(-d, sX[k * LX + lane], x);
+#pragma unroll 1
+        for (int k = 0; k < r; ++k) {   // r is the same in every lane
+          const float xk = lane < MP ? sX[k * LX + lane] : 0.f;
+          const float d = group_sum<32>(x * xk);
+          x = fmaf(-d, xk, x);
         }
       }
       const float nx = sqrtf(group_sum<32>(x * x));

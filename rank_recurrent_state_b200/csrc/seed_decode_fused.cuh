@@ -30,7 +30,7 @@ __global__ void __launch_bounds__(32, 12)
 template <int FORM, int DK, int DV, int MP, typename TS>
 static size_t fused_smem(int maxc) {
   const size_t dec = warp_stage_bytes(maxc, DK, DV, sizeof(TS)) + kCoefFloats * sizeof(float) + 16;
-  const size_t cmp = FastLayout<FORM, DK, DV, MP>::bytes;
+  const size_t cmp = FastLayout<FORM, DK, DV, MP>::bytes_aligned;
   return dec > cmp ? dec : cmp;
 }
 
