@@ -521,9 +521,9 @@ struct FastLayout {
   static constexpr int A = ((A_CH > A_B ? A_CH : A_B) + 3) & ~3;
   static constexpr int LU = A;                                  // L_u (MP x LG), then T_u | T_v
   static constexpr int LU_N = (MP * LG > 2 * MP * kFastMaxR ? MP * LG : 2 * MP * kFastMaxR);
-  static constexpr int SMALL = LU + LU_N;                       // nu nv du dv nrm, scl
-  static constexpr int FLOATS = SMALL + 5 * MP + SL;
-  static constexpr size_t BAR_OFF = FLOATS * sizeof(float) + (MP + 4) * sizeof(int);   // 8-byte aligned
+  static constexpr int SMALL = LU + LU_N;
+  static constexpr int FLOATS = SMALL + 4 * MP + SL;           // nu nv du nrm, scl
+  static constexpr size_t BAR_OFF = FLOATS * sizeof(float) + kFastMaxR * sizeof(int);   // 8-byte aligned
   static constexpr size_t bytes = BAR_OFF + 2 * sizeof(uint64_t);
   // a block whose dynamic shared memory may start anywhere re-aligns region A
   static constexpr size_t bytes_aligned = bytes + 1024;
@@ -562,8 +562,7 @@ SEED_DEV bool compress_fast_unit(const FastParams& p, const CUtensorMap& tmU, co
   float* nu = sA + Lay::SMALL;
   float* nv = nu + MP;
   float* du = nv + MP;
-  float* dvv = du + MP;
-  float* nrm = dvv + MP;
+  float* nrm = du + MP;
   float* scl = nrm + MP;
   int* sel = reinterpret_cast<int*>(scl + Lay::SL);
 
@@ -612,16 +611,15 @@ SEED_DEV bool compress_fast_unit(const FastParams& p, const CUtensorMap& tmU, co
     return true;
   }
 
-  // D_u, D_v: true column norms (GDN / Mamba-2: with the lazy scale gamma_j); the
-  // core is formed with w_k = D_u D_v / max(D_u D_v) so that its entries are of
-  // order one, and its singular values are scaled back by wmax
+  // D_u, D_v: true column norms (GDN / Mamba-2: with the lazy scale gamma_j; D_v is
+  // nv); the core is formed with w_k = D_u D_v / max(D_u D_v) so that its entries
+  // are of order one, and its singular values are scaled back by wmax
   float wl = 0.f;
   if (lane < MP) {
     const float gj = (KDA || lane >= m) ? 1.f : scl[lane];
-    const float a = nu[lane] * gj, bv = nv[lane];
+    const float a = nu[lane] * gj;
     du[lane] = a;
-    dvv[lane] = bv;
-    wl = a * bv;
+    wl = a * nv[lane];
   }
   const float wmax = warp_max(wl);
   const float winv = wmax > 0.f ? 1.f / wmax : 0.f;
@@ -636,7 +634,7 @@ SEED_DEV bool compress_fast_unit(const FastParams& p, const CUtensorMap& tmU, co
     for (int i = 0; i < MP; ++i) acc[i] = 0.f;
 #pragma unroll 2
     for (int k = 0; k < MP; ++k) {
-      const float cf = sM[k * LG + j] * (du[k] * dvv[k] * winv);
+      const float cf = sM[k * LG + j] * (du[k] * nv[k] * winv);
 #pragma unroll
       for (int i4 = 0; i4 < MP; i4 += 4) {
         const float4 l = ld4(sLu + k * LG + i4);
