@@ -23,6 +23,9 @@
 //      its own rows, no reduction;
 //   4. the sink update, the new column pair and the read-out, written straight
 //      from registers.
+// With 16-bit factors (fp16, bf16) the stage holds the stored 16-bit columns (half
+// the space, so more warps per SM), widened to float32 as they are read; the new
+// pair is rounded to nearest as it is stored.
 #pragma once
 
 #include "seed_common.cuh"
