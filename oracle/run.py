@@ -8,7 +8,7 @@ Per unit (request b, layer l, head h), following SEED figures & tables
      appends one column pair,
   4. after the step that brings the column count to R + W, the factors are
      compressed back to rank R (``compress.truncate_qr_core``): with decode steps
-     counted from 1 this is after steps W, 2W, 3W, ... ("every W steps"); a
+     counted from 1 this is after steps W, 2W, 3W, ... (every W steps); a
      request that joined j steps earlier (ragged schedules) is j steps ahead.
 An open-loop dense shadow S_t^exact runs the dense recurrence on the same inputs
 from the uncompressed prefill state, for Lemma 1 and Corollary 4 checks.

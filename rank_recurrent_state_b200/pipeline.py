@@ -2,7 +2,7 @@
 
 prefill (synthetic, dense) -> seed_state_init_from_dense -> per step and layer:
 seed_synth_token_inputs + seed_decode_step, and seed_compress after the step that
-fills R + W columns ("every W steps", decode steps counted from 1).  With ragged
+fills R + W columns (every W steps, decode steps counted from 1).  With ragged
 schedules the requests joined at different times (a lead-in of up to W - 1 steps)
 and seed_compress runs after every step, compressing the units that are due.  With
 fused=True the step after which a compression is due (every step when ragged) is
