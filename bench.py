@@ -282,7 +282,7 @@ def run_reference(args, world, rank):
 # ------------------------------------------------------------------ GPU arm
 
 def decode_kernel_name(d):
-    return "decode_warp_kernel" if d.R + d.W - 1 <= 32 else "decode_step_kernel"
+    return "decode_warp_kernel" if d.R + d.W - 1 <= 64 else "decode_step_kernel"
 
 
 def decode_traffic(d, units, cbar):

@@ -13,7 +13,7 @@ template <int FORM, int DK, int DV, int MAXC, typename TS>
 static int launch_warp_t(const DecodeParams& p, cudaStream_t st) {
   auto kern = decode_warp_kernel<FORM, DK, DV, MAXC, TS>;
   const int maxc = p.R + p.W - 1;
-  const size_t smem = warp_stage_bytes(maxc, DK, DV, sizeof(TS)) + kCoefFloats * sizeof(float) + 16;
+  const size_t smem = warp_stage_bytes(maxc, DK, DV, sizeof(TS)) + coef_floats(MAXC) * sizeof(float) + 16;
   // per device: the shared-memory opt-in (for the largest stage), and the resident
   // blocks per SM for each stage size
   constexpr int kMaxDev = 64;
@@ -23,7 +23,7 @@ static int launch_warp_t(const DecodeParams& p, cudaStream_t st) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev || maxc > MAXC) return SEED_ERR_CUDA;
   if (!attr_set[dev]) {
-    const size_t smax = warp_stage_bytes(MAXC, DK, DV, sizeof(TS)) + kCoefFloats * sizeof(float) + 16;
+    const size_t smax = warp_stage_bytes(MAXC, DK, DV, sizeof(TS)) + coef_floats(MAXC) * sizeof(float) + 16;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smax) != cudaSuccess)
       return SEED_ERR_CUDA;
     if (cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
@@ -47,7 +47,9 @@ static int launch_warp_maxc(const DecodeParams& p, cudaStream_t st) {
   const int maxc = p.R + p.W - 1;
   if (maxc <= 8) return launch_warp_t<FORM, DK, DV, 8, TS>(p, st);
   if (maxc <= 16) return launch_warp_t<FORM, DK, DV, 16, TS>(p, st);
-  return launch_warp_t<FORM, DK, DV, 32, TS>(p, st);
+  if (maxc <= 32) return launch_warp_t<FORM, DK, DV, 32, TS>(p, st);
+  if (maxc <= 48) return launch_warp_t<FORM, DK, DV, 48, TS>(p, st);
+  return launch_warp_t<FORM, DK, DV, 64, TS>(p, st);
 }
 
 template <int FORM, int DK, int DV>
@@ -60,7 +62,7 @@ static int launch_warp_dims(const DecodeParams& p, int factors, cudaStream_t st)
   return SEED_ERR_INVALID_ARG;
 }
 
-bool decode_warp_supported(const seed_dims& d) { return d.R + d.W - 1 <= 32; }
+bool decode_warp_supported(const seed_dims& d) { return d.R + d.W - 1 <= 64; }
 
 int launch_decode_warp(const DecodeParams& p, int form, int dk, int dv, int factors, cudaStream_t st) {
 #define SEED_WARP_DIMS(FORM)                                                              \

@@ -1,10 +1,10 @@
-// seed_decode_warp.cuh -- the decode step with one warp per unit, for R + W <= 33.
+// seed_decode_warp.cuh -- the decode step with one warp per unit, for R + W <= 65.
 //
 // "Shallow Encoding Emits Deep Memories", SEED summary (picx.dev), "Exact Update
 // (Lemma 2)" with the sink recurrence of Lemma 1, and the read-out o = S+^T q;
 // the arithmetic is that of seed_decode.cu, organised differently.
 //
-// With at most 32 stored columns a unit is small enough for one warp, and a warp
+// With at most 64 stored columns a unit is small enough for one warp, and a warp
 // that owns a unit needs no block-level synchronisation at all.  Every warp of a
 // persistent grid (one warp per block) owns one shared-memory stage sized for the
 // R + W - 1 columns a unit holds at most before a step; lane 0 fills it with two
@@ -140,6 +140,8 @@ __host__ __device__ constexpr size_t warp_stage_bytes(int maxc, int dk, int dv, 
   return (size_t)maxc * (dk + dv) * elem;
 }
 constexpr int kCoefFloats = 2 * 32;
+// The column coefficients of a stage of up to MAXC columns: a (q, k) pair each.
+__host__ __device__ constexpr int coef_floats(int maxc) { return 2 * (maxc > 32 ? maxc : 32); }
 
 // The body of both kernels below.  FUSE: after the step of a unit that brings it to
 // R + W columns, the same warp compresses it in place (compress_fast_unit, panel
@@ -231,7 +233,9 @@ SEED_DEV void decode_warp_run(const DecodeParams& p, const FastParams* fp, const
         const float tot = warp_xreduce<32>(dv);
         const int j = c0 + (M2 ? lane : (lane & 15));
         if (j < c) {
-          const float f = KDA ? 1.f : g * (c0 == 0 ? cur.gam_lo : cur.gam_hi);
+          // gamma_j: from registers for j < 32, from HBM (cached) above
+          const float gj = c0 >= 32 ? p.scale[unit * p.slen + j] : (c0 == 0 ? cur.gam_lo : cur.gam_hi);
+          const float f = KDA ? 1.f : g * gj;
           s_f[2 * j + (M2 ? 0 : (lane >> 4))] = f * tot;
         }
       }
@@ -321,7 +325,8 @@ SEED_DEV void decode_warp_run(const DecodeParams& p, const FastParams* fp, const
           // gamma_j of column j = lane: gam_lo for lanes < 16 (and every lane for
           // Mamba-2), gam_hi above; the new column's scale is 1
           const float gl = (M2 || lane < 16) ? cur.gam_lo : cur.gam_hi;
-          for (int j = lane; j <= c; j += 32) p.scale[unit * p.slen + j] = j < c ? g * gl : 1.f;
+          for (int j = lane; j <= c; j += 32)
+            p.scale[unit * p.slen + j] = j < c ? g * (j < 32 ? gl : p.scale[unit * p.slen + j]) : 1.f;
         }
         if (lane == 0) p.ncols[unit] = c + 1;
         if (__any_sync(0xffffffffu, bad) && lane == 0) raise_flag(p.status, SEED_FLAG_NONFINITE);

@@ -108,7 +108,7 @@ def test_mamba2_reduced():
     _parity(cfg, sample, 200, 2 * cfg.W + 3, batch=1)
 
 
-@pytest.mark.parametrize("R,W", [(8, 8), (16, 16), (32, 64), (8, 64)])
+@pytest.mark.parametrize("R,W", [(8, 8), (16, 16), (16, 32), (32, 32), (32, 64), (8, 64)])
 def test_kda_sweep_reduced(R, W):
     """KDA 128x128 with per-channel decay over the R, W sweep (one request, sampled heads)."""
     cfg = config(4, R=R, W=W)
