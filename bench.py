@@ -204,7 +204,7 @@ def cpu_oracle_rate(cfg, seconds: float, rank_seed: int = 0) -> dict:
     except Exception:   # pragma: no cover - reporting only
         threads = 1
     rng = np.random.default_rng(1234 + rank_seed)
-    n = 96
+    n = min(96, cfg.units)   # the sample, or every unit of a small workload
     u = rng.choice(cfg.units, size=n, replace=False)
     b, rem = np.divmod(u, cfg.layers * cfg.heads)
     l, h = np.divmod(rem, cfg.heads)

@@ -62,3 +62,24 @@ def test_reference_arm_prints_only_on_rank0(capsys):
     args = bench.parse_args(["--impl", "reference", "--cpu-seconds", "0.01", "--config", "0"])
     assert bench.run_reference(args, world=2, rank=1) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_line_carries_the_contract_keys(capsys):
+    """Rank 0 of the reference arm prints one JSON line with the keys of the bench
+    contract (the oracle timed on the host cores, a bounded sample)."""
+    import json
+
+    import bench
+    args = bench.parse_args(["--impl", "reference", "--cpu-seconds", "0.2", "--config", "0"])
+    assert bench.run_reference(args, world=1, rank=0) == 0
+    lines = [x for x in capsys.readouterr().out.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
+    assert "workload" in d["config"]
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert d["e2e"]["value"] == d["value"] and d["e2e"]["h2d_bytes_per_step"] == 0
