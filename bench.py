@@ -35,10 +35,11 @@ if ROOT not in sys.path:
 METRIC = "decode head-steps/s and achieved HBM GB/s (% of B200 peak) at R=16,W=16"
 UNIT = "head-steps/s"
 NOMINAL_HBM_GBS = 8000.0
-# DRAM bytes (read + write) of one decode launch of the GDN stack shape, measured by ncu
-# (dram__bytes_read.sum + dram__bytes_write.sum; profiles/decode_warp_kernel_gdn_stack_2layers.md):
-# a full per-layer launch (256 requests x 48 heads) at c = 19 stored columns.  Set to None
-# whenever the decode kernel changes until it is measured again.
+# DRAM bytes (read + write) of one decode launch, measured by ncu (dram__bytes_read.sum +
+# dram__bytes_write.sum; profiles/decode_warp_kernel_*gdn_stack_2layers.md) for a full
+# per-layer launch of the GDN stack shape (256 requests x 48 heads) at c = 19 stored
+# columns, per factor format.  Set an entry to None whenever that kernel changes, until
+# it is measured again.
 NCU_DECODE_TRAFFIC = [
     {"kernel": "decode_warp_kernel", "form": 0, "d_k": 128, "d_v": 128, "R": 16, "W": 16, "factors": 0,
      "units": 12288, "c": 19, "bytes": 266.032e6 + 20.088e6},
@@ -291,7 +292,7 @@ def decode_traffic(d, units, cbar):
     capture does not match this kernel and shape."""
     from rank_recurrent_state_b200 import roofline
     key = (decode_kernel_name(d), d.form, d.d_k, d.d_v, d.R, d.W, d.factors)
-    match = [t for t in NCU_DECODE_TRAFFIC
+    match = [t for t in (NCU_DECODE_TRAFFIC or [])
              if (t["kernel"], t["form"], t["d_k"], t["d_v"], t["R"], t["W"], t["factors"]) == key]
     if not match:
         return None

@@ -233,8 +233,9 @@ SEED_DEV void decode_warp_run(const DecodeParams& p, const FastParams* fp, const
         const float tot = warp_xreduce<32>(dv);
         const int j = c0 + (M2 ? lane : (lane & 15));
         if (j < c) {
-          // gamma_j: from registers for j < 32, from HBM (cached) above
-          const float gj = c0 >= 32 ? p.scale[unit * p.slen + j] : (c0 == 0 ? cur.gam_lo : cur.gam_hi);
+          // gamma_j: from registers for j < 32, from HBM (cached) above (stages of more
+          // than 32 columns only)
+          const float gj = (MAXC > 32 && c0 >= 32) ? p.scale[unit * p.slen + j] : (c0 == 0 ? cur.gam_lo : cur.gam_hi);
           const float f = KDA ? 1.f : g * gj;
           s_f[2 * j + (M2 ? 0 : (lane >> 4))] = f * tot;
         }
@@ -326,7 +327,7 @@ SEED_DEV void decode_warp_run(const DecodeParams& p, const FastParams* fp, const
           // Mamba-2), gam_hi above; the new column's scale is 1
           const float gl = (M2 || lane < 16) ? cur.gam_lo : cur.gam_hi;
           for (int j = lane; j <= c; j += 32)
-            p.scale[unit * p.slen + j] = j < c ? g * (j < 32 ? gl : p.scale[unit * p.slen + j]) : 1.f;
+            p.scale[unit * p.slen + j] = j < c ? g * ((MAXC > 32 && j >= 32) ? p.scale[unit * p.slen + j] : gl) : 1.f;
         }
         if (lane == 0) p.ncols[unit] = c + 1;
         if (__any_sync(0xffffffffu, bad) && lane == 0) raise_flag(p.status, SEED_FLAG_NONFINITE);
