@@ -3,9 +3,9 @@
 What it computes: the best rank-R approximation of the content U V^T, the only
 approximation of the method.  SEED summary (picx.dev), "Open-Loop Error Bound
 (Corollary 4)" (the compression error that the bound integrates), and SEED
-figures & tables (thelatestinai.com), Figure 1(b) ("every W steps, the factors
-are compressed back to rank R") and Table 1.  The sink a v̄^T is never touched
-("the sink is kept exactly": SEED commentary (sungsoo.github.io), "2. Exact
+figures & tables (thelatestinai.com), Figure 1(b) (the factors return to rank R
+once every W steps) and Table 1.  The sink a v̄^T is never touched: it is carried
+exactly, outside the truncation (SEED commentary (sungsoo.github.io), "2. Exact
 factored update").
 
 Two functions:
