@@ -388,3 +388,21 @@ def test_byte_account_reproduces_table2(golden_dir):
         rs = bytes_model.resident_bytes(bytes_model.shallow_state_bytes(heads, dk, dv, R, W // 2), T, int(cache))
         assert round(ro / 1e6) == res_o
         assert round(rs / 1e6) == res_s
+
+
+# ------------------------------------------------------------------- small helpers
+
+def test_rel_gap_and_numerical_rank_closed_forms():
+    """The gap at the truncation point and the numerical-rank rule on spectra whose
+    answers are written out: s = (4, 3, 3, 1) has gap (4-3)/4 at R = 1, none at R = 2
+    (a tie) and no s_{R+1} at R = 4; singular values at or below max(d) eps s_1 count
+    as zero, larger ones keep their square roots."""
+    from oracle import compress as oc
+    s = np.array([[4.0, 3.0, 3.0, 1.0]])
+    assert oc.rel_gap(s, 1)[0] == 0.25
+    assert oc.rel_gap(s, 2)[0] == 0.0
+    assert oc.rel_gap(s, 3)[0] == 0.5
+    assert oc.rel_gap(s, 4)[0] == 1.0
+    assert oc.tail_norm(s, 2)[0] == np.sqrt(10.0)
+    sq = oc.numerical_sqrt_sigma(np.array([[4.0, 1e-3, 1e-20, 0.0]]), (16, 16))
+    np.testing.assert_array_equal(sq, [[2.0, np.sqrt(1e-3), 0.0, 0.0]])
