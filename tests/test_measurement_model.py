@@ -4,9 +4,10 @@ the bench's config object.
 
 The float32 byte counts per head-step follow the accounting of Table 17 on the
 SEED figures & tables page (GDN stack at the mean column count R + (W - 1) / 2:
-26,304 B with lazy decay, 38,144 B with U rewritten, 50,176 B in the Table 2
-convention, 131,072 B dense; KDA 27,136 B; the Mamba-2 stack 20,032 B); the 16-bit
-counts follow from the same terms with two bytes per stored U and V value.
+26,304 B with lazy decay, 38,144 B with U rewritten; 50,176 B in the Table 2
+convention, every state read and written at R + W / 2; 131,072 B dense; KDA
+27,136 B; the Mamba-2 stack 20,032 B); the 16-bit counts follow from the same
+terms with two bytes per stored U and V value.
 """
 
 import pytest
