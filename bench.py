@@ -302,6 +302,21 @@ def decode_traffic(d, units, cbar):
     return t["bytes"] / t["units"] * units * per(cbar) / per(t["c"])
 
 
+def compress_kernel_launches(d) -> int:
+    """Kernels one seed_compress call launches: the fast (Cholesky-QR) kernel where the
+    shape allows it, then the Householder scan over the units still due."""
+    fast = d.R + d.W <= 32 and d.R <= 16 and d.d_k in (64, 128) and d.d_v in (64, 128)
+    return 2 if fast else 1
+
+
+def fused_kernel_launches(d) -> int:
+    """Kernels one seed_decode_step_compress call launches: the fused kernel and the
+    Householder scan, or a decode launch and a compression."""
+    if d.R + d.W - 1 <= 32 and compress_kernel_launches(d) == 2:
+        return 2
+    return 1 + compress_kernel_launches(d)
+
+
 def compress_rate(d, diag, cmp_ms, clk):
     """FP32 rate of the compression launches (the FLOP model of roofline.compress_flops,
     with the measured mean Jacobi sweeps) and its fraction of the CUDA-core FP32 peak
@@ -460,7 +475,8 @@ def run_ours(args, world, rank, local):
                                             if diag["compress_units"] else None),
                      "cholqr_units": diag["cholqr_units"], "householder_units": diag["householder_units"],
                      **compress_rate(d, diag, cmp_ms, clk.summary())},
-        "gpu_launches": len(dec_ms) + len(cmp_ms) + len(ev["fus"]),
+        "gpu_launches": (len(dec_ms) + len(cmp_ms) * compress_kernel_launches(d)
+                         + len(ev["fus"]) * fused_kernel_launches(d)),
         "status_flags": flags | flags_warm,
         "setup_s": t_setup,
     }

@@ -70,3 +70,15 @@ def test_config_object_names_the_workload():
     assert c["workload"].startswith("gdn-stack") and c["layers"] == 36 and c["heads"] == 48
     assert c["global_batch"] == 256 and c["factors"].startswith("f16") and "fused" in c["compression"]
     assert "L2" in c["l2"]
+
+
+def test_kernel_launch_counts():
+    import bench
+    from rank_recurrent_state_b200.seed import Dims
+    gdn = Dims(0, 256, 36, 48, 128, 128, 16, 16)
+    m2 = Dims(2, 256, 40, 64, 128, 64, 8, 32)          # R + W = 40: Householder only
+    tiny = Dims(0, 1, 1, 2, 16, 16, 4, 4)               # d = 16: Householder only
+    assert bench.compress_kernel_launches(gdn) == 2
+    assert bench.compress_kernel_launches(m2) == 1 and bench.compress_kernel_launches(tiny) == 1
+    assert bench.fused_kernel_launches(gdn) == 2
+    assert bench.fused_kernel_launches(m2) == 2 and bench.fused_kernel_launches(tiny) == 2
