@@ -149,3 +149,40 @@ def test_noalloc_decode_step_validates_before_touching_the_device(lib):
     assert lib.seed_decode_step_noalloc(None, ctypes.byref(s), 0, A, A, A, A, A, A, None, None) == -1
     assert lib.seed_decode_step_noalloc(ctypes.byref(d), ctypes.byref(s), 0, A, A, A, A, A, A,
                                         0x10002, None) == -3
+
+
+def test_headers_compile_as_c_and_link(lib, tmp_path):
+    """A plain C99 program includes both headers, links against libseed.so and calls
+    entry points whose argument checks run on the host (no device needed)."""
+    import shutil
+    import subprocess
+    from rank_recurrent_state_b200 import build as b
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include "seed.h"
+#include "seed_synth.h"
+int main(void) {
+  seed_dims d = {SEED_GDN, 2, 3, 4, 128, 128, 16, 16, SEED_FACTORS_F16};
+  seed_state s = {0};
+  if (seed_scale_len(&d) != 32) return 1;
+  if (seed_workspace_bytes(&d) < 4) return 2;
+  if (seed_decode_step(&d, &s, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0) != SEED_ERR_INVALID_ARG) return 3;
+  d.factors = 9;
+  if (seed_scale_len(&d) != -1) return 4;
+  printf("%s\n", seed_status_string(SEED_ERR_SHAPE));
+  return 0;
+}
+""")
+    exe = tmp_path / "abi"
+    libdir = os.path.dirname(b.LIB)
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
+                        "-o", str(exe), "-L", libdir, "-lseed", f"-Wl,-rpath,{libdir}"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, (r.returncode, r.stderr)
+    assert r.stdout.strip()
