@@ -99,6 +99,24 @@ def _check(fn: str, rc: int) -> None:
         raise SeedError(fn, rc)
 
 
+def _check_state(dims: "Dims", state: "State") -> None:
+    """The C ABI sees only pointers: check here that the state's tensors have the
+    element types and sizes the dims describe (U and V in the factor format)."""
+    B, L, H, m = dims.batch, dims.layers, dims.heads, dims.m
+    slen = dims.d_k if dims.form == SEED_KDA else (m + 3) // 4 * 4
+    want = {"a": (torch.float32, B * L * H * dims.d_k),
+            "U": (FACTOR_DTYPES[dims.factors], B * L * H * m * dims.d_k),
+            "V": (FACTOR_DTYPES[dims.factors], B * L * H * m * dims.d_v),
+            "scale": (torch.float32, B * L * H * slen),
+            "ncols": (torch.int32, B * L * H),
+            "vbar": (torch.float32, L * H * dims.d_v)}
+    for name, (dtype, n) in want.items():
+        t = getattr(state, name)
+        if t.dtype != dtype or t.numel() < n:
+            raise ValueError(f"state.{name}: expected {dtype} with at least {n} elements, got {t.dtype} "
+                             f"with {t.numel()}")
+
+
 @dataclass
 class State:
     """Device tensors of the stored state (layouts as in seed.h)."""
@@ -160,6 +178,7 @@ def seed_workspace_bytes(dims: Dims) -> int:
 
 def seed_state_init_from_dense(dims: Dims, state: State, layer: int, S_dense: torch.Tensor,
                                ws: Workspace, sigma_out: torch.Tensor | None = None, stream=None) -> None:
+    _check_state(dims, state)
     d, s = dims.c(), state.c()
     _check("seed_state_init_from_dense", _lib.load().seed_state_init_from_dense(
         ctypes.byref(d), ctypes.byref(s), layer, _ptr(S_dense), _ptr(sigma_out), ws.ptr, ws.nbytes,
@@ -168,6 +187,7 @@ def seed_state_init_from_dense(dims: Dims, state: State, layer: int, S_dense: to
 
 def seed_decode_step(dims: Dims, state: State, layer: int, q, k, v, alpha, beta, o,
                      ws: Workspace, stream=None) -> None:
+    _check_state(dims, state)
     d, s = dims.c(), state.c()
     _check("seed_decode_step", _lib.load().seed_decode_step(
         ctypes.byref(d), ctypes.byref(s), layer, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
@@ -178,6 +198,7 @@ def seed_decode_step_noalloc(dims: Dims, state: State, layer: int, q, k, v, alph
                              status_out: torch.Tensor | None = None, stream=None) -> None:
     """seed_decode_step with the library's own fixed device workspace; status_out, if
     given, is a device int32/uint32 tensor of one element that receives the flags."""
+    _check_state(dims, state)
     d, s = dims.c(), state.c()
     _check("seed_decode_step_noalloc", _lib.load().seed_decode_step_noalloc(
         ctypes.byref(d), ctypes.byref(s), layer, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
@@ -188,6 +209,7 @@ def seed_decode_step_compress(dims: Dims, state: State, layer: int, q, k, v, alp
                               ws: Workspace, sigma_out: torch.Tensor | None = None, stream=None) -> None:
     """seed_decode_step fused with the compression of the units the step brings to
     R + W columns; sigma_out [B * H][R] (rows of compressed units written)."""
+    _check_state(dims, state)
     d, s = dims.c(), state.c()
     _check("seed_decode_step_compress", _lib.load().seed_decode_step_compress(
         ctypes.byref(d), ctypes.byref(s), layer, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
@@ -200,6 +222,7 @@ def seed_noalloc_workspace_bytes() -> int:
 
 def seed_compress(dims: Dims, state: State, layer: int, ws: Workspace,
                   sigma_out: torch.Tensor | None = None, stream=None) -> None:
+    _check_state(dims, state)
     d, s = dims.c(), state.c()
     _check("seed_compress", _lib.load().seed_compress(
         ctypes.byref(d), ctypes.byref(s), layer, _ptr(sigma_out), ws.ptr, ws.nbytes, _stream(stream)))
@@ -207,6 +230,7 @@ def seed_compress(dims: Dims, state: State, layer: int, ws: Workspace,
 
 def seed_state_to_dense(dims: Dims, state: State, layer: int, S_out: torch.Tensor, ws: Workspace,
                         units: torch.Tensor | None = None, stream=None) -> None:
+    _check_state(dims, state)
     d, s = dims.c(), state.c()
     n = 0 if units is None else int(units.numel())
     _check("seed_state_to_dense", _lib.load().seed_state_to_dense(
@@ -217,6 +241,7 @@ def seed_state_to_dense(dims: Dims, state: State, layer: int, S_out: torch.Tenso
 def seed_state_energy(dims: Dims, state: State, layer: int, out: torch.Tensor, ws: Workspace,
                       units: torch.Tensor | None = None, stream=None) -> None:
     """out [n][4]: sink energy, content energy, cross term, total (see seed.h)."""
+    _check_state(dims, state)
     d, s = dims.c(), state.c()
     n = 0 if units is None else int(units.numel())
     _check("seed_state_energy", _lib.load().seed_state_energy(

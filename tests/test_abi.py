@@ -186,3 +186,21 @@ int main(void) {
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0, (r.returncode, r.stderr)
     assert r.stdout.strip()
+
+
+def test_binding_checks_state_types_before_calling():
+    """The binding rejects a state whose factor tensors do not have the dims' element
+    type (the C ABI cannot see it) before anything reaches the library."""
+    import torch
+    from rank_recurrent_state_b200 import seed as S
+    d = S.Dims(S.SEED_GDN, 2, 1, 2, 64, 64, 8, 8, S.SEED_FACTORS_F16)
+    vbar = torch.ones(1, 2, 64)
+    st = S.State.allocate(d, vbar, device="cpu")
+    assert st.U.dtype == torch.float16 and st.V.dtype == torch.float16
+    S._check_state(d, st)                                   # matches: no error
+    st32 = S.State.allocate(S.Dims(S.SEED_GDN, 2, 1, 2, 64, 64, 8, 8), vbar, device="cpu")
+    with pytest.raises(ValueError, match="state.U"):
+        S.seed_compress(d, st32, S.SEED_ALL_LAYERS, None)
+    small = S.State.allocate(S.Dims(S.SEED_GDN, 1, 1, 2, 64, 64, 8, 8, S.SEED_FACTORS_F16), vbar, device="cpu")
+    with pytest.raises(ValueError, match="state.a"):
+        S.seed_decode_step(d, small, 0, None, None, None, None, None, None, None)
