@@ -92,3 +92,46 @@ def test_wrong_sign_of_the_cross_energy(monkeypatch):
         return e
     monkeypatch.setattr(diagnostics, "energies", planted)
     _fails(diag_pins.test_parts_add_up_to_the_energy_of_the_reconstructed_state)
+
+
+def test_core_without_the_transpose_in_the_qr_route(monkeypatch):
+    def planted(U, V, R):
+        Qu, Ru = np.linalg.qr(U)
+        Qv, Rv = np.linalg.qr(V)
+        M = Ru @ Rv                                              # R_u R_v instead of R_u R_v^T
+        X, s, Yt = np.linalg.svd(M, full_matrices=False)
+        sq = np.sqrt(s[:, :R])
+        return Qu @ X[:, :, :R] * sq[:, None, :], Qv @ np.swapaxes(Yt[:, :R, :], 1, 2) * sq[:, None, :], s
+    monkeypatch.setattr(compress, "truncate_qr_core", planted)
+    _fails(pins.test_qr_core_route_equals_product_svd)
+
+
+def test_sink_projection_without_the_norm(monkeypatch):
+    def planted(S, vbar):
+        return np.einsum("nij,nj->ni", S, vbar)                  # S vbar, not S vbar / |vbar|^2
+    monkeypatch.setattr(factored, "sink_coefficient", planted)
+    import oracle.convert as oconv
+    monkeypatch.setattr(oconv, "sink_coefficient", planted)
+    _fails(pins.test_conversion_recovers_a_known_sink_and_content)
+
+
+def test_mamba2_with_the_erase_left_on(monkeypatch):
+    real = factored.step
+
+    def planted(form, a, U, V, vbar, q, k, v, alpha, beta):
+        if form == pins.FORM_MAMBA2:                             # GDN's update with Delta as beta
+            return real(pins.FORM_GDN, a, U, V, vbar, q, k, v, alpha, beta)
+        return real(form, a, U, V, vbar, q, k, v, alpha, beta)
+    monkeypatch.setattr(factored, "step", planted)
+    _fails(pins.test_mamba2_is_the_general_update_with_erase_off)
+
+
+def test_kda_decay_applied_after_the_erase(monkeypatch):
+    def planted(S, k, v, alpha, beta):
+        b = np.asarray(beta, dtype=np.float64)[:, None, None]
+        kS = np.einsum("ni,nij->nj", k, S)
+        E = S - b * np.einsum("ni,nj->nij", k, kS)
+        return alpha[:, :, None] * E + b * np.einsum("ni,nj->nij", k, v)   # Diag(alpha) (I - b k k^T) S
+    monkeypatch.setattr(recurrences, "kda_step", planted)
+    _fails(pins.test_kda_closed_form_and_gdn_special_case)
+
