@@ -204,3 +204,21 @@ def test_binding_checks_state_types_before_calling():
     small = S.State.allocate(S.Dims(S.SEED_GDN, 1, 1, 2, 64, 64, 8, 8, S.SEED_FACTORS_F16), vbar, device="cpu")
     with pytest.raises(ValueError, match="state.a"):
         S.seed_decode_step(d, small, 0, None, None, None, None, None, None, None)
+
+
+def test_oracle_and_product_path_share_no_code():
+    """The package never imports the oracle, the oracle never imports the package or
+    loads the library; the one module both use is the seeded input generator."""
+    import ast
+    pkg = os.path.join(ROOT, "rank_recurrent_state_b200")
+    for path in glob.glob(os.path.join(pkg, "*.py")):
+        tree = ast.parse(open(path).read())
+        for node in ast.walk(tree):
+            names = ([a.name for a in node.names] if isinstance(node, ast.Import)
+                     else [node.module or ""] if isinstance(node, ast.ImportFrom) else [])
+            assert not any(n.split(".")[0] == "oracle" for n in names), path
+    for path in glob.glob(os.path.join(ROOT, "rank_recurrent_state_b200", "csrc", "*")):
+        assert "oracle" not in open(path).read().lower(), path
+    for path in glob.glob(os.path.join(ROOT, "oracle", "*.py")):
+        text = open(path).read()
+        assert "rank_recurrent_state_b200" not in text and "libseed" not in text, path
