@@ -222,3 +222,10 @@ def test_oracle_and_product_path_share_no_code():
     for path in glob.glob(os.path.join(ROOT, "oracle", "*.py")):
         text = open(path).read()
         assert "rank_recurrent_state_b200" not in text and "libseed" not in text, path
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    """Without libseed.so the binding raises; there is no CPU path to fall back to."""
+    monkeypatch.setattr(_lib, "_LIB", None)
+    with pytest.raises(ImportError, match="no CPU fallback"):
+        _lib.load(str(tmp_path / "libseed.so"))
