@@ -91,3 +91,38 @@ def test_transposed_warp_reduction_lane_mapping(nv):
     totals = vals.sum(axis=0)
     for lane in range(32):
         assert out[lane] == totals[(lane >> sh) & (nv - 1)]
+
+
+def _swz(j, e):
+    """Offset of element e of column j in a swizzled float32 chunk (the kernels' swz)."""
+    return j * 32 + ((((e >> 2) ^ (j & 7)) << 2) | (e & 3))
+
+
+@pytest.mark.parametrize("mp,m", [(16, 9), (16, 16), (32, 24), (32, 32)])
+def test_16bit_chunk_widening_lands_in_the_swizzled_layout(mp, m):
+    """issue_chunk16 / widen_chunk16: lane l copies rows 8 (l & 3) .. of column
+    8 pass + (l >> 2) and widens them into two float4 slots; together the lanes must
+    write every (column, row) of the chunk exactly once, at swz(column, row), with
+    zeros for the columns past m, and read only staging slots they filled."""
+    chunk = np.full(mp * 32, np.nan)
+    written = np.zeros(mp * 32, dtype=int)
+    staged = set()
+    for lane in range(32):
+        q = lane & 3
+        for p in range(mp // 8):
+            j = p * 8 + (lane >> 2)
+            if j < m:
+                staged.add((lane, j))                      # the cp.async of this lane
+            for half in range(2):                          # rows 8q .. 8q+3, 8q+4 .. 8q+7
+                base = j * 32 + (((2 * q + half) ^ (j & 7)) << 2)
+                for t in range(4):
+                    e = 8 * q + 4 * half + t
+                    assert base + t == _swz(j, e)
+                    chunk[base + t] = (1000 * j + e) if j < m else 0.0
+                    written[base + t] += 1
+                if j < m:
+                    assert (lane, j) in staged             # reads its own staging slot
+    assert np.all(written == 1)
+    for j in range(mp):
+        for e in range(32):
+            assert chunk[_swz(j, e)] == ((1000 * j + e) if j < m else 0.0)
