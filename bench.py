@@ -72,8 +72,11 @@ def parse_args(argv=None):
                     help="ragged compression schedules: requests joined at different times, a "
                          "compression launch after every step compresses the units that are due")
     ap.add_argument("--dense-steps", type=int, default=8)
-    ap.add_argument("--e2e-steps", type=int, default=8)
+    ap.add_argument("--e2e-steps", type=int, default=None,
+                    help="end-to-end steps (default: one compression window, W)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--reference-units", type=int, default=384,
+                    help="units of the workload the reference arm (the fp64 oracle) steps")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
@@ -257,7 +260,16 @@ def config_obj(cfg, batch, world, prefill, ragged=False, factors="f32", fused=Fa
 
 
 def run_reference(args, world, rank):
-    from workloads import config
+    """The reference arm: the fp64 oracle, as it stands, on the host cores.  Each of
+    the W warm-up and K timed steps is one decode step (and the compression when it
+    is due) of a fixed seeded sample of the workload's units; value = K x sample /
+    the timed seconds.  Rank 0 alone runs it."""
+    import numpy as np
+
+    from oracle import compress as ocomp
+    from oracle import convert as oconv
+    from oracle import factored, recurrences
+    from workloads import config, philox
     cfg = config(args.config)
     if args.batch:
         cfg = cfg.replace(batch=args.batch)
@@ -265,17 +277,60 @@ def run_reference(args, world, rank):
         cfg = cfg.replace(layers=args.layers)
     if rank != 0:
         return 0
-    per = max(1.0, args.cpu_seconds)
-    res = cpu_oracle_rate(cfg, per)
-    line = {"metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:   # pragma: no cover - reporting only
+        threads = 1
+    n = min(args.reference_units, cfg.units)
+    rng = np.random.default_rng(1234)
+    u = rng.choice(cfg.units, size=n, replace=False)
+    b, rem = np.divmod(u, cfg.layers * cfg.heads)
+    l, h = np.divmod(rem, cfg.heads)
+    n_pre = 256
+    S0 = recurrences.dense_prefill(cfg, b, l, h, n_pre)
+    vb = philox.vbar(cfg, l, h).astype(np.float64)
+    a, U, V, _ = oconv.convert(S0, vb, cfg.R)
+    c = cfg.R
+    P = max(args.input_steps, 1)
+    inputs = {}
+
+    def step(t):
+        nonlocal a, U, V, c
+        if t % P not in inputs:
+            inputs[t % P] = recurrences.f64(philox.token_inputs(cfg, b, l, h, t % P, philox.PHASE_DECODE))
+        inp = inputs[t % P]
+        a, U, V, _o = factored.step(cfg.form, a, U, V, vb, inp["q"], inp["k"], inp["v"],
+                                    inp["alpha"], inp["beta"])
+        c += 1
+        if c == cfg.R + cfg.W:
+            U, V, _s = ocomp.truncate_qr_core(U, V, cfg.R)
+            c = cfg.R
+
+    for t in range(min(P, args.warmup + args.steps)):   # input generation, outside the timing
+        if t not in inputs:
+            inputs[t] = recurrences.f64(philox.token_inputs(cfg, b, l, h, t, philox.PHASE_DECODE))
+    for t in range(args.warmup):
+        step(t)
+    t0 = time.perf_counter()
+    for t in range(args.steps):
+        step(args.warmup + t)
+    dt = time.perf_counter() - t0
+    value = args.steps * n / dt
+    prefill = cfg.n_prefill if args.prefill is None else args.prefill
+    sample = (f"{n} seeded units of the workload (of {cfg.units}), each step one fp64 NumPy decode step of "
+              f"all of them plus the compression when due; {args.steps} timed steps after {args.warmup} "
+              f"warm-up steps, {dt:.2f} s; the sample's state comes from a {n_pre}-token oracle prefill "
+              f"and conversion (untimed), inputs pre-generated")
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded Philox4x32-10 inputs)", "impl": "reference",
-            "config": config_obj(cfg, cfg.batch, world, 256),
-            "cpu_baseline": res,
-            "e2e": {"value": res["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
-                    "d2h_bytes_per_step": 0}}
-    line["ms_per_step"] = cfg.units / res["value"] * 1e3
+            "config": config_obj(cfg, cfg.batch, world, prefill),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": int(threads), "kind": "oracle",
+                             "sample": sample, "affinity_cores": len(os.sched_getaffinity(0))},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "note": "ms_per_step is the measured time of one step of the sample, not of the whole workload"}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -331,6 +386,208 @@ def compress_rate(d, diag, cmp_ms, clk):
     peak = roofline.fp32_peak_tflops(mhz)
     return {"flops_per_unit": flops / d.units, "tflops": tflops, "fp32_peak_tflops": peak,
             "frac_fp32_peak": tflops / peak}
+
+
+def steady_state(dec, cmp_ms, R, W, layers):
+    """Steady-state step time from the run's own per-launch CUDA-event times.
+
+    In lockstep every unit holds c = R, R + 1, ..., R + W - 1 columns before the
+    W steps of one compression window, and one compression closes the window, so
+    a step costs on average
+
+        t_step = ( sum_c layers * t_dec(c) + t_cmp ) / W
+
+    with t_dec(c) the mean decode-launch time at column count c and t_cmp the mean
+    compression time.  Column counts the timed window did not reach take the
+    least-squares line through the measured ones (the launch moves bytes linear
+    in c).  dec: list of (ms, c).  Returns a dict (ms per step, the per-c means)."""
+    import numpy as np
+    by_c = {}
+    for ms, c in dec:
+        by_c.setdefault(int(round(c)), []).append(ms)
+    cs = np.array(sorted(by_c), dtype=np.float64)
+    means = np.array([sum(by_c[int(c)]) / len(by_c[int(c)]) for c in cs])
+    if cs.size >= 2:
+        slope, icpt = np.polyfit(cs, means, 1)
+    else:
+        slope, icpt = 0.0, float(means[0])
+    window_cs = range(R, R + W)
+    t_dec = {c: (sum(by_c[c]) / len(by_c[c]) if c in by_c else icpt + slope * c) for c in window_cs}
+    t_cmp = sum(cmp_ms) / len(cmp_ms) if cmp_ms else 0.0
+    dec_window = layers * sum(t_dec.values())
+    return {"ms_per_step": (dec_window + t_cmp) / W, "decode_ms_per_launch_mean": sum(t_dec.values()) / W,
+            "compress_ms": t_cmp, "decode_share": dec_window / (dec_window + t_cmp),
+            "column_counts_measured": int(cs.size), "column_counts_in_window": W}
+
+
+def gpu_numa_affinity(local: int):
+    """CPUs local to this rank's GPU (NVML), or None when NVML cannot tell."""
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            visible = [x for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
+            idx = int(visible[local]) if len(visible) > local and visible[local].isdigit() else local
+            h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            n = (os.cpu_count() + 63) // 64
+            masks = pynvml.nvmlDeviceGetCpuAffinity(h, n)
+        finally:
+            pynvml.nvmlShutdown()
+    except Exception:   # pragma: no cover - reporting only
+        return None
+    cpus = {64 * i + b for i, m in enumerate(masks) for b in range(64) if (int(m) >> b) & 1}
+    cpus &= os.sched_getaffinity(0)
+    return cpus or None
+
+
+def run_e2e(args, run, d, L, BH, q, k, v, alpha, beta, o, kda, stream, dev, world, local, units, step_ms, s_next):
+    """The same metric through the public API with host buffers: every step copies its
+    inputs from pinned host memory to the device and each layer's o back, inside the
+    timed region.  Timed over whole compression windows that start right after a
+    compression (steady state); also measures the host link alone in the same run."""
+    import torch
+
+    from rank_recurrent_state_b200 import seed as S
+    # pinned buffers on the GPU's NUMA node: allocate them from a thread bound to the
+    # CPUs local to the GPU (pages are placed on the allocating thread's node)
+    aff = gpu_numa_affinity(local)
+    old_aff = os.sched_getaffinity(0)
+    if aff:
+        os.sched_setaffinity(0, aff)
+    try:
+        Ph = 2
+        hq = torch.empty(Ph, L, BH, d.d_k, dtype=torch.float32, pin_memory=True)
+        hk = torch.empty_like(hq, pin_memory=True)
+        hv = torch.empty(Ph, L, BH, d.d_v, dtype=torch.float32, pin_memory=True)
+        ha = torch.empty(Ph, *alpha.shape[1:], dtype=torch.float32, pin_memory=True)
+        hb = torch.empty(Ph, *beta.shape[1:], dtype=torch.float32, pin_memory=True)
+        ho = torch.empty(L, BH, d.d_v, dtype=torch.float32, pin_memory=True)
+    finally:
+        if aff:
+            os.sched_setaffinity(0, old_aff)
+    for t in range(Ph):
+        hq[t].copy_(q[t]); hk[t].copy_(k[t]); hv[t].copy_(v[t]); ha[t].copy_(alpha[t]); hb[t].copy_(beta[t])
+    # inputs copied in on their own stream into two alternating device buffers, each
+    # layer's o copied out on a third stream as soon as it is written, so that the
+    # transfers (host memory and PCIe bound) overlap the decode launches
+    nb = 2
+    bufs = [(torch.empty_like(q[0, 0]), torch.empty_like(k[0, 0]), torch.empty_like(v[0, 0]),
+             torch.empty_like(alpha[0, 0]), torch.empty_like(beta[0, 0])) for _ in range(nb)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(nb)]
+    ev_free = [torch.cuda.Event() for _ in range(nb)]
+    ev_dec = [torch.cuda.Event() for _ in range(L)]
+    ev_out = [torch.cuda.Event() for _ in range(L)]
+    h2d = L * sum(x.numel() for x in bufs[0]) * 4   # as copied
+    d2h = o.numel() * 4
+
+    # the host link alone: one step's inputs in (all layers, one copy per tensor), the
+    # outputs out, then both at once (PCIe is full duplex)
+    def timed(fn, reps=3):
+        best = None
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1)
+            best = ms if best is None else min(best, ms)
+        return best
+
+    def h2d_all():
+        q[1].copy_(hq[0], non_blocking=True); k[1].copy_(hk[0], non_blocking=True)
+        v[1].copy_(hv[0], non_blocking=True); alpha[1].copy_(ha[0], non_blocking=True)
+        beta[1].copy_(hb[0], non_blocking=True)
+
+    def d2h_all():
+        ho.copy_(o, non_blocking=True)
+
+    def both():
+        s_in.wait_stream(stream)
+        with torch.cuda.stream(s_in):
+            h2d_all()
+        d2h_all()
+        stream.wait_stream(s_in)
+
+    h2d_bytes_all = (hq[0].numel() + hk[0].numel() + hv[0].numel() + ha[0].numel() + hb[0].numel()) * 4
+    t_h2d, t_d2h, t_both = timed(h2d_all), timed(d2h_all), timed(both)
+    link = {"h2d_GBps": h2d_bytes_all / (t_h2d / 1e3) / 1e9, "d2h_GBps": d2h / (t_d2h / 1e3) / 1e9,
+            "duplex_ms_per_step": t_both, "pinned_on_gpu_numa_node": bool(aff),
+            "gpu_local_cpus": len(aff) if aff else None}
+    # restore the pool's step-1 inputs overwritten by the link test
+    for l in range(L):
+        al = alpha[1, l] if kda else alpha[1, l, :BH]
+        S.seed_synth_token_inputs(d, run.key, S.SEED_PHASE_DECODE, 1, l, run.vbar, q[1, l], k[1, l],
+                                  v[1, l], al, beta[1, l, :BH])
+    bound_ms = max(t_both, step_ms)   # copies overlapped with the device work at best
+
+    # align to the start of a window (the step after a compression), untimed
+    while run.c != d.R and not args.ragged:
+        for l in range(L):
+            S.seed_decode_step(d, run.state, l, q[0, l], k[0, l], v[0, l],
+                               alpha[0, l] if kda else alpha[0, l, :BH], beta[0, l, :BH], o[l], run.ws, stream)
+        run.c += 1
+        if run.c == d.m:
+            S.seed_compress(d, run.state, S.SEED_ALL_LAYERS, run.ws, stream=stream)
+            run.c = d.R
+    n_steps = args.e2e_steps if args.e2e_steps else d.W
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    s_in.wait_stream(stream)
+    s_out.wait_stream(stream)
+    n = 0
+    for s in range(n_steps):
+        t = s % Ph
+        fuse = args.fused and (args.ragged or run.c + 1 == d.m)
+        for l in range(L):
+            bi = n % nb
+            bq, bk, bv, ba, bb = bufs[bi]
+            with torch.cuda.stream(s_in):
+                if n >= nb:
+                    s_in.wait_event(ev_free[bi])
+                bq.copy_(hq[t, l], non_blocking=True); bk.copy_(hk[t, l], non_blocking=True)
+                bv.copy_(hv[t, l], non_blocking=True); ba.copy_(ha[t, l], non_blocking=True)
+                bb.copy_(hb[t, l], non_blocking=True)
+                ev_in[bi].record(s_in)
+            stream.wait_event(ev_in[bi])
+            if s > 0:
+                stream.wait_event(ev_out[l])   # last step's o of this layer is out
+            step_fn = S.seed_decode_step_compress if fuse else S.seed_decode_step
+            step_fn(d, run.state, l, bq, bk, bv, ba if kda else ba[:BH], bb[:BH], o[l], run.ws, stream=stream)
+            ev_free[bi].record(stream)
+            ev_dec[l].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_dec[l])
+                ho[l].copy_(o[l], non_blocking=True)
+                ev_out[l].record(s_out)
+            n += 1
+        run.c += 1
+        if run.c == d.m or args.ragged:   # ragged: some request is due after every step
+            if not fuse:
+                S.seed_compress(d, run.state, S.SEED_ALL_LAYERS, run.ws, stream=stream)
+            run.c = d.R
+    stream.wait_stream(s_out)
+    stream.wait_stream(s_in)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    per_step = e2e_ms / n_steps
+    return {"value": n_steps * units * world / (e2e_ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_steps,
+            "ms_per_step": per_step,
+            "h2d_GBps_achieved": h2d / (per_step / 1e3) / 1e9, "d2h_GBps_achieved": d2h / (per_step / 1e3) / 1e9,
+            "host_link": link,
+            "host_link_bound_value": units * world / (bound_ms / 1e3),
+            "frac_of_host_link_bound": (units * world / (per_step / 1e3)) / (units * world / (bound_ms / 1e3)),
+            "note": "pinned host buffers; every step copies its inputs in and its o out (copies on their own "
+                    "streams, overlapping the decode launches); timed over whole compression windows "
+                    "starting right after a compression; host_link_bound_value = units / max(device "
+                    "step, one step's input and output copies run alone and together)"}
 
 
 def run_ours(args, world, rank, local):
@@ -441,49 +698,107 @@ def run_ours(args, world, rank, local):
     elapsed_ms = max_over_ranks(start.elapsed_time(end), world, dev)
     flags = S.seed_get_status(run.ws)
     diag = S.seed_get_diagnostics(run.ws)
+    s_next = args.warmup + args.steps
 
     units = d.units
-    value = args.steps * units * world / (elapsed_ms / 1e3)
-    dec_ms = [a.elapsed_time(b) for a, b, _ in ev["dec"]]
-    dec_bytes = [BH * roofline.lazy_bytes(d.form, d.d_k, d.d_v, c, fb) for _, _, c in ev["dec"]]
+    dec_pairs = [(a.elapsed_time(b), c) for a, b, c in ev["dec"]]
     cmp_ms = [a.elapsed_time(b) for a, b in ev["cmp"]]
-    # (with --fused --ragged every launch is a fused one: no plain decode launch to time)
-    dec_gbs = sum(dec_bytes) / (sum(dec_ms) / 1e3) / 1e9 if dec_ms else None
+    fus_ms = [a.elapsed_time(b) for a, b in ev["fus"]]
+    extra_cmp = False
+    if not args.ragged and not cmp_ms and not fus_ms and d.m - d.R > 0:
+        # the timed window held no compression (fewer steps than W): time the next
+        # one, after the timed region, so that the steady state below has its cost
+        while True:
+            due = run.c + 1 == d.m
+            ev2 = {"dec": [], "cmp": [], "fus": []}
+            one_step(s_next, ev2)
+            s_next += 1
+            if due:
+                cmp_ms = [a.elapsed_time(b) for a, b in ev2["cmp"]]
+                fus_ms = [a.elapsed_time(b) for a, b in ev2["fus"]]
+                extra_cmp = True
+                break
+        torch.cuda.synchronize()
+        diag2 = S.seed_get_diagnostics(run.ws)
+        for key in diag:
+            diag[key] += diag2[key]
+        flags |= S.seed_get_status(run.ws)
+    raw_value = args.steps * units * world / (elapsed_ms / 1e3)
+    # steady state of one compression window (lockstep), from the per-launch times
+    if args.ragged:
+        steady = None   # every step holds every column count and compresses 1/W of the units
+        step_ms = elapsed_ms / args.steps
+    elif args.fused:
+        # the fused launches replace the decode launches of the window's last step and
+        # the compression: window = decode at c = R .. R + W - 2, then the fused launches
+        steady = steady_state(dec_pairs, [], d.R, d.W - 1, L)
+        t_fus = sum(fus_ms) / len(fus_ms) if fus_ms else 0.0
+        step_ms = (steady["ms_per_step"] * (d.W - 1) + L * t_fus) / d.W
+        steady["ms_per_step"] = step_ms
+        steady["fused_ms_per_launch"] = t_fus
+    else:
+        steady = steady_state(dec_pairs, cmp_ms, d.R, d.W, L)
+        step_ms = steady["ms_per_step"]
+    value = units * world / (step_ms / 1e3)
+    step_ms = max_over_ranks(step_ms, world, dev)
+    value = units * world / (step_ms / 1e3)
+    dec_ms = [ms for ms, _ in dec_pairs]
+    if steady is not None and dec_ms:
+        dec_launch_ms = steady["decode_ms_per_launch_mean"]
+    else:
+        dec_launch_ms = sum(dec_ms) / len(dec_ms) if dec_ms else None
     peak, peak_kind = measured_peak_hbm()
     cbar = roofline.mean_columns(d.R, d.W)
+    if steady is not None and args.fused:
+        cbar = roofline.mean_columns(d.R, d.W - 1)
+    # algorithmic bytes of the mean launch of a window (the byte model is linear in c)
+    dec_bytes = BH * roofline.lazy_bytes(d.form, d.d_k, d.d_v, cbar, fb)
+    dec_gbs = dec_bytes / (dec_launch_ms / 1e3) / 1e9 if dec_launch_ms else None
+    t_cmp = sum(cmp_ms) / len(cmp_ms) if cmp_ms else None
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded Philox4x32-10 inputs and prefill, generated on the device)",
         "config": config_obj(cfg, B, world, prefill, args.ragged, args.factors, args.fused),
+        "steady_state": (None if steady is None else dict(
+            steady, how="value = units / t_step with t_step = (sum over the window's column counts "
+                        "c = R .. R+W-1 of layers x t_decode(c) + t_compress) / W, every t the mean "
+                        "CUDA-event time of those launches in the timed region"
+                        + ("; the compression was timed right after the timed region (fewer timed "
+                           "steps than W)" if extra_cmp else ""))),
+        "window": {"ms_per_step": elapsed_ms / args.steps, "value": raw_value,
+                   "compressions": len(cmp_ms) + len(fus_ms) // max(L, 1) if not extra_cmp else 0,
+                   "note": "the K timed steps as they fell, K x units / (max over ranks of the "
+                           "event time between the barriers)"},
         "roofline": {"bound": "hbm", "kernel": decode_kernel_name(d), "achieved": dec_gbs, "peak": peak,
-                     "unit": "GB/s", "frac": dec_gbs / peak if dec_ms else None,
+                     "unit": "GB/s", "frac": dec_gbs / peak if dec_gbs else None,
                      "peak_source": f"{peak_kind} copy bandwidth",
-                     "frac_of_nominal_8TBs": dec_gbs / NOMINAL_HBM_GBS if dec_ms else None,
+                     "frac_of_nominal_8TBs": dec_gbs / NOMINAL_HBM_GBS if dec_gbs else None,
                      "traffic": decode_traffic(d, BH, cbar),
                      "algorithmic_bytes_per_head_step_mean": roofline.lazy_bytes(d.form, d.d_k, d.d_v, cbar, fb),
-                     "avg_launch_us": 1e3 * sum(dec_ms) / len(dec_ms) if dec_ms else None,
+                     "algorithmic_bytes_per_launch": dec_bytes,
+                     "avg_launch_us": 1e3 * dec_launch_ms if dec_launch_ms else None,
                      "launches": len(dec_ms)},
-        "decode_only": {"head_steps_per_s": len(dec_ms) * BH * world / (sum(dec_ms) / 1e3) if dec_ms else None,
+        "decode_only": {"head_steps_per_s": BH * world / (dec_launch_ms / 1e3) if dec_launch_ms else None,
                         "GBps": dec_gbs},
-        "compress": {"launches": len(cmp_ms), "ms_per_launch": (sum(cmp_ms) / len(cmp_ms)) if cmp_ms else None,
-                     "ns_per_head_step_amortized": 1e6 * sum(cmp_ms) / (args.steps * units) if cmp_ms else 0.0,
-                     "share_of_step": sum(cmp_ms) / elapsed_ms,
+        "compress": {"launches": len(cmp_ms), "ms_per_launch": t_cmp,
+                     "ns_per_head_step_amortized": (1e6 * t_cmp / (d.W * units) if t_cmp and not args.ragged
+                                                    else 1e6 * sum(cmp_ms) / (args.steps * units)),
+                     "share_of_step": ((t_cmp / d.W) / step_ms if t_cmp and not args.ragged
+                                       else sum(cmp_ms) / elapsed_ms),
                      "jacobi_sweeps_mean": (diag["compress_sweeps"] / diag["compress_units"]
                                             if diag["compress_units"] else None),
                      "cholqr_units": diag["cholqr_units"], "householder_units": diag["householder_units"],
                      **compress_rate(d, diag, cmp_ms, clk.summary())},
-        "gpu_launches": (len(dec_ms) + len(cmp_ms) * compress_kernel_launches(d)
-                         + len(ev["fus"]) * fused_kernel_launches(d)),
+        "gpu_launches": (len(dec_ms) + (len(cmp_ms) if not extra_cmp else 0) * compress_kernel_launches(d)
+                         + (len(fus_ms) if not extra_cmp else 0) * fused_kernel_launches(d)),
         "status_flags": flags | flags_warm,
         "setup_s": t_setup,
     }
-    if ev["fus"]:
-        fus_ms = [a.elapsed_time(b) for a, b in ev["fus"]]
+    if fus_ms:
         line["fused"] = {"launches": len(fus_ms), "ms_per_launch": sum(fus_ms) / len(fus_ms),
-                         "share_of_step": sum(fus_ms) / elapsed_ms,
                          "note": "decode step of one layer with the compression of its due units "
                                  "(seed_decode_step_compress); the Householder launch for declined "
                                  "units is included"}
@@ -523,75 +838,8 @@ def run_ours(args, world, rank, local):
 
     # ---- end to end: host inputs in pinned memory, copies inside the timed region
     if not args.no_e2e:
-        Ph = 2
-        hq = torch.empty(Ph, L, BH, d.d_k, dtype=torch.float32, pin_memory=True)
-        hk = torch.empty_like(hq, pin_memory=True)
-        hv = torch.empty(Ph, L, BH, d.d_v, dtype=torch.float32, pin_memory=True)
-        ha = torch.empty(Ph, *alpha.shape[1:], dtype=torch.float32, pin_memory=True)
-        hb = torch.empty(Ph, *beta.shape[1:], dtype=torch.float32, pin_memory=True)
-        for t in range(Ph):
-            hq[t].copy_(q[t]); hk[t].copy_(k[t]); hv[t].copy_(v[t]); ha[t].copy_(alpha[t]); hb[t].copy_(beta[t])
-        ho = torch.empty(L, BH, d.d_v, dtype=torch.float32, pin_memory=True)
-        # inputs copied in on their own stream into two alternating device buffers, each
-        # layer's o copied out on a third stream as soon as it is written, so that the
-        # transfers (host memory and PCIe bound) overlap the decode launches
-        nb = 2
-        bufs = [(torch.empty_like(q[0, 0]), torch.empty_like(k[0, 0]), torch.empty_like(v[0, 0]),
-                 torch.empty_like(alpha[0, 0]), torch.empty_like(beta[0, 0])) for _ in range(nb)]
-        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        ev_in = [torch.cuda.Event() for _ in range(nb)]
-        ev_free = [torch.cuda.Event() for _ in range(nb)]
-        ev_dec = [torch.cuda.Event() for _ in range(L)]
-        ev_out = [torch.cuda.Event() for _ in range(L)]
-        h2d = L * sum(x.numel() for x in bufs[0]) * 4   # as copied
-        d2h = o.numel() * 4
-        torch.cuda.synchronize()
-        barrier(world, dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        s_in.wait_stream(stream)
-        s_out.wait_stream(stream)
-        n = 0
-        for s in range(args.e2e_steps):
-            t = s % Ph
-            fuse = args.fused and (args.ragged or run.c + 1 == d.m)
-            for l in range(L):
-                bi = n % nb
-                bq, bk, bv, ba, bb = bufs[bi]
-                with torch.cuda.stream(s_in):
-                    if n >= nb:
-                        s_in.wait_event(ev_free[bi])
-                    bq.copy_(hq[t, l], non_blocking=True); bk.copy_(hk[t, l], non_blocking=True)
-                    bv.copy_(hv[t, l], non_blocking=True); ba.copy_(ha[t, l], non_blocking=True)
-                    bb.copy_(hb[t, l], non_blocking=True)
-                    ev_in[bi].record(s_in)
-                stream.wait_event(ev_in[bi])
-                if s > 0:
-                    stream.wait_event(ev_out[l])   # last step's o of this layer is out
-                step_fn = S.seed_decode_step_compress if fuse else S.seed_decode_step
-                step_fn(d, run.state, l, bq, bk, bv, ba if kda else ba[:BH], bb[:BH], o[l], run.ws, stream=stream)
-                ev_free[bi].record(stream)
-                ev_dec[l].record(stream)
-                with torch.cuda.stream(s_out):
-                    s_out.wait_event(ev_dec[l])
-                    ho[l].copy_(o[l], non_blocking=True)
-                    ev_out[l].record(s_out)
-                n += 1
-            run.c += 1
-            if run.c == d.m or args.ragged:   # ragged: some request is due after every step
-                if not fuse:
-                    S.seed_compress(d, run.state, S.SEED_ALL_LAYERS, run.ws, stream=stream)
-                run.c = d.R
-        stream.wait_stream(s_out)
-        stream.wait_stream(s_in)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        barrier(world, dev)
-        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-        line["e2e"] = {"value": args.e2e_steps * units * world / (e2e_ms / 1e3), "unit": UNIT,
-                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                       "note": "pinned host buffers; every step copies its inputs in and its o out "
-                               "(copies on their own streams, overlapping the decode launches)"}
+        line["e2e"] = run_e2e(args, run, d, L, BH, q, k, v, alpha, beta, o, kda, stream, dev, world, local,
+                              units, step_ms, s_next)
         line["status_flags"] |= S.seed_get_status(run.ws)
 
     if rank == 0 and world == 1 and not args.no_cpu:

@@ -70,8 +70,10 @@ typedef enum {
 #define SEED_FLAG_BADINDEX 0x20u  /* seed_state_to_dense met a unit index outside the scope;
                                      that output slab was not written                      */
 #define SEED_FLAG_TIMEOUT 0x40u   /* a bounded wait for a bulk copy gave up (1 s); the unit
-                                     being worked on was left unchanged or, in a
-                                     compression, partly written                          */
+                                     being worked on was left unchanged, except that a
+                                     compression that had already written part of its
+                                     result sets the unit's column count to -1 (later
+                                     calls flag it SEED_FLAG_BADCOLS and skip it)          */
 
 /* Supported shapes: (d_k, d_v) equal and in {16, 32, 64, 128}, or (128, 64), or
  * (64, 128); R >= 1, W >= 1, R + W <= SEED_MAX_COLS and R + W <= min(d_k, d_v).
@@ -249,6 +251,18 @@ int seed_get_status(void* ws, void* stream, uint32_t* flags);
  * Returns SEED_OK or SEED_ERR_CUDA.                                                 */
 int seed_get_diagnostics(void* ws, void* stream, uint32_t* counters);
 
+/* Test hook for the bounded waits (no counterpart in the pages).  With enable != 0,
+ * every later call on this workspace that waits for bulk copies with a bounded wait
+ * -- seed_decode_step's and seed_decode_step_compress's decode warps, and
+ * seed_compress's Cholesky-QR blocks with float32 factors -- withholds its first
+ * copy and gives up on it at once: the warp raises SEED_FLAG_TIMEOUT, waits (at
+ * most 1 s) in vain for the withheld bytes with no copy in flight, and stops, so
+ * the units it had not finished are left unchanged (a decode warp fails on its
+ * first unit, before touching any unit; a compression block's unit goes to the
+ * Householder path as usual).  enable = 0 turns it off; seed_workspace_init clears
+ * it.  The workspace word lies past the status word and the counters.              */
+int seed_debug_wait_fault(void* ws, size_t ws_bytes, int32_t enable, void* stream);
+
 /* Static description of a seed_status code. */
 const char* seed_status_string(int status);
 
@@ -269,6 +283,10 @@ const char* seed_status_string(int status);
  * shape does).  Nothing is enqueued when an argument is rejected.
  * The first call on each device looks up the array's address and may load the
  * module onto the device: make it before any stream capture on that device.
+ * The address is kept per device together with the id of the context it was
+ * looked up in; after a device reset (cudaDeviceReset, or the primary context
+ * released and created again) the next call sees a new context and looks the
+ * address up again, so that call too should come before any stream capture.
  * All calls on a device share the one array: calls that can run at the same time
  * (other streams, other host threads) race on the status word; serialise them,
  * or use seed_decode_step with a workspace each.                                  */

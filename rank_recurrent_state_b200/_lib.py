@@ -57,6 +57,7 @@ SIGNATURES = {
     "seed_get_status": (ctypes.c_int, [c_void_p, c_void_p, ctypes.POINTER(c_uint32)]),
     "seed_get_diagnostics": (ctypes.c_int, [c_void_p, c_void_p, ctypes.POINTER(c_uint32)]),
     "seed_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "seed_debug_wait_fault": (ctypes.c_int, [c_void_p, c_size_t, c_int32, c_void_p]),
     "seed_synth_vbar": (ctypes.c_int, [ctypes.POINTER(seed_dims), seed_synth_key, c_void_p, c_void_p]),
     "seed_synth_token_inputs": (ctypes.c_int, [ctypes.POINTER(seed_dims), seed_synth_key, c_int32, c_int32,
                                                c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,

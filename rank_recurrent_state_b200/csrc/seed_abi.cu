@@ -227,6 +227,14 @@ int seed_get_diagnostics(void* ws, void* stream, uint32_t* counters) {
   return SEED_OK;
 }
 
+int seed_debug_wait_fault(void* ws, size_t ws_bytes, int32_t enable, void* stream) {
+  SEED_TRY(check_ws(ws, ws_bytes));
+  uint32_t* word = status_word(ws) + seed::kWsWaitFaultWordHost;
+  return cudaMemsetAsync(word, enable ? 1 : 0, sizeof(uint32_t), as_stream(stream)) == cudaSuccess
+             ? SEED_OK
+             : SEED_ERR_CUDA;
+}
+
 const char* seed_status_string(int status) {
   switch (status) {
     case SEED_OK: return "ok";

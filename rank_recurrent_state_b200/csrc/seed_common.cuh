@@ -10,6 +10,7 @@
 #include <type_traits>
 
 #include "../../include/seed.h"
+#include "seed_launch.h"
 
 #define SEED_DEV __device__ __forceinline__
 
@@ -19,6 +20,17 @@ constexpr int kWarp = 32;
 
 // ------------------------------------------------------------------ status word
 SEED_DEV void raise_flag(uint32_t* status, uint32_t flag) { atomicOr(status, flag); }
+
+// Workspace word (32-bit index from the status word) that, when nonzero, makes the
+// kernels with bounded copy waits fail their first wait on purpose: each warp
+// (decode) or block (fast compression) withholds its first bulk copy and gives up
+// on it at once.  No copy is then in flight when the wait fails.  Set only by
+// seed_debug_wait_fault, for the tests of the timeout path.
+constexpr int kWsWaitFaultWord = 8;
+static_assert(kWsWaitFaultWord == kWsWaitFaultWordHost, "one workspace layout");
+SEED_DEV bool wait_fault_injected(const uint32_t* status) {
+  return *reinterpret_cast<const volatile uint32_t*>(status + kWsWaitFaultWord) != 0u;
+}
 
 // ------------------------------------------------------------------ vector helpers
 SEED_DEV float4 ld_stream4(const float* p) { return __ldcs(reinterpret_cast<const float4*>(p)); }

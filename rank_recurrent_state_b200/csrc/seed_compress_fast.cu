@@ -36,20 +36,6 @@ __global__ void __launch_bounds__(32)
   compress_fast_unit<FORM, DK, DV, MP, TS>(p, tmU, tmV, blockIdx.x, sA, bar, uses);
 }
 
-static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess || !ptr)
-      return nullptr;
-    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
 // A factor array [units][m][D] as a 3-D float tensor {D, m, units}; boxes of 32 rows
 // of MP columns of one unit, 128-byte swizzle, zero fill outside (columns >= m).
 bool make_panel_map(CUtensorMap* tm, const float* base, int D, int m, long long units, int MP) {
@@ -68,16 +54,9 @@ template <int FORM, int DK, int DV, int MP, typename TS>
 static int launch_fast_t(const FastParams& p, int blocks, cudaStream_t st) {
   using Lay = FastLayout<FORM, DK, DV, MP>;
   auto kern = compress_fast_kernel<FORM, DK, DV, MP, TS>;
-  constexpr int kMaxDev = 64;
-  static bool attr_set[kMaxDev] = {false};
+  static LaunchCache cache;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return SEED_ERR_CUDA;
-  if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::bytes) !=
-        cudaSuccess)
-      return SEED_ERR_CUDA;
-    attr_set[dev] = true;
-  }
+  if (const int rc = cache.prepare(reinterpret_cast<const void*>(kern), Lay::bytes, &dev)) return rc;
   const long long units = (long long)p.B * p.L * p.H;
   const int m = p.R + p.W;
   CUtensorMap tmU, tmV;

@@ -302,15 +302,16 @@ SEED_DEV int jacobi_regs(float* sM, bool& conv) {
 // bar[c & 1].  Columns m .. MP-1 lie outside the tensor and arrive as zeros.  In
 // shared memory column j is a 128-byte row whose 16-byte pieces are permuted by
 // the 128-byte swizzle: piece f sits at f ^ (j & 7).
+// withhold: announce the bytes but issue no copy (the injected wait fault).
 template <int NCU, int CHUNK>
 SEED_DEV void issue_chunk(int c, float* sA, const CUtensorMap* tmU, const CUtensorMap* tmV, long long unit,
-                          uint64_t* bar) {
+                          uint64_t* bar, bool withhold = false) {
   const int bb = c & 1;
   const bool isU = c < NCU;
   const int r0 = 32 * (isU ? c : c - NCU);
   if ((threadIdx.x & 31) == 0) {
     mbar_arrive_expect_tx(&bar[bb], (uint32_t)(CHUNK * 4));
-    tma_load_3d(sA + bb * CHUNK, isU ? tmU : tmV, r0, 0, (int)unit, &bar[bb]);
+    if (!withhold) tma_load_3d(sA + bb * CHUNK, isU ? tmU : tmV, r0, 0, (int)unit, &bar[bb]);
   }
 }
 
@@ -368,12 +369,12 @@ SEED_DEV void widen_chunk16(int c, float* sA, int m, bool more) {
 // through buf.
 template <int DK, int DV, int MP, typename TS>
 SEED_DEV bool next_chunk(int c, uint32_t (&uses)[2], float* sA, uint64_t* bar, const FastParams& p,
-                         long long unit, int m, const float*& buf) {
+                         long long unit, int m, const float*& buf, uint64_t limit = kWaitLimitNs) {
   constexpr int NCH = (DK + DV) / 32, CHUNK = MP * 32;
   if constexpr (std::is_same<TS, float>::value) {
     const int bb = c & 1;
     const uint32_t ph = uses[bb] & 1u;
-    if (!__all_sync(kFull, mbar_wait_bounded(&bar[bb], ph, kWaitLimitNs))) {
+    if (!__all_sync(kFull, mbar_wait_bounded(&bar[bb], ph, limit))) {
       mbar_wait_bounded(&bar[bb], ph, kWaitLimitNs);
       if (c + 1 < NCH) mbar_wait_bounded(&bar[bb ^ 1], uses[bb ^ 1] & 1u, kWaitLimitNs);
       return false;
@@ -425,7 +426,8 @@ SEED_DEV void mma3_tf32(float (&d)[4], const uint32_t (&ah)[4], const uint32_t (
 template <bool KDA, int DK, int DV, int MP, int LG, typename TS>
 SEED_DEV bool gram_stream(int c0, int c1, bool fold, float* sA, const CUtensorMap* tmU,
                           const CUtensorMap* tmV, const FastParams& p, long long unit, int m, uint64_t* bar,
-                          uint32_t (&uses)[2], const float* scl, float* Gs, float (&g)[MP], bool& bad) {
+                          uint32_t (&uses)[2], const float* scl, float* Gs, float (&g)[MP], bool& bad,
+                          bool fault = false) {
   constexpr int NCU = DK / 32, NCH = (DK + DV) / 32, CHUNK = MP * 32;
   constexpr int NT = MP / 8, MT = MP / 16;
   const int lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
@@ -442,7 +444,9 @@ SEED_DEV bool gram_stream(int c0, int c1, bool fold, float* sA, const CUtensorMa
 #pragma unroll 1
   for (int c = c0; c < c1; ++c) {
     const float* buf;
-    if (!next_chunk<DK, DV, MP, TS>(c, uses, sA, bar, p, unit, m, buf)) return false;
+    if (!next_chunk<DK, DV, MP, TS>(c, uses, sA, bar, p, unit, m, buf,
+                                    (fault && c == c0) ? 0ull : kWaitLimitNs))
+      return false;
     const int r0 = 32 * (c < NCU ? c : c - NCU);
 #pragma unroll 1
     for (int ks = 0; ks < 4; ++ks) {
@@ -533,9 +537,9 @@ struct FastLayout {
 // Chunks 0 and 1 of a stream.
 template <int DK, int DV, int MP, typename TS>
 SEED_DEV void start_stream(float* sA, const CUtensorMap* tmU, const CUtensorMap* tmV, const FastParams& p,
-                           long long unit, int m, uint64_t* bar) {
+                           long long unit, int m, uint64_t* bar, bool withhold = false) {
   if constexpr (std::is_same<TS, float>::value) {
-    issue_chunk<DK / 32, MP * 32>(0, sA, tmU, tmV, unit, bar);
+    issue_chunk<DK / 32, MP * 32>(0, sA, tmU, tmV, unit, bar, withhold);
     issue_chunk<DK / 32, MP * 32>(1, sA, tmU, tmV, unit, bar);
   } else {
     issue_chunk16<DK, DV, MP, TS>(0, sA, p, unit, m);
@@ -580,12 +584,16 @@ SEED_DEV bool compress_fast_unit(const FastParams& p, const CUtensorMap& tmU, co
   __syncwarp();
   for (int e = lane; e < p.slen; e += 32) scl[e] = p.scale[unit * p.slen + e];
   __syncwarp();
-  start_stream<DK, DV, MP, TS>(sA, &tmU, &tmV, p, unit, m, bar);
+  // the injected wait fault (float32 factors: the only ones copied with mbarriers)
+  const bool fault = std::is_same<TS, float>::value && wait_fault_injected(p.status);
+  start_stream<DK, DV, MP, TS>(sA, &tmU, &tmV, p, unit, m, bar, fault);
   bool bad = false;   // ill-conditioned or badly scaled: left for the Householder kernel
   float g[MP];
-  // U: chunks 0 .. NCU-1, then its Cholesky factor (to its own region)
+  // U: chunks 0 .. NCU-1, then its Cholesky factor (to its own region); a copy that
+  // does not arrive here leaves the unit untouched at R + W columns, for the
+  // Householder kernel
   if (!gram_stream<KDA, DK, DV, MP, LG, TS>(0, NCU, true, sA, &tmU, &tmV, p, unit, m, bar, uses, scl, sLu, g,
-                                            bad)) {
+                                            bad, fault)) {
     if (lane == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
     return false;
   }
@@ -803,8 +811,15 @@ SEED_DEV bool compress_fast_unit(const FastParams& p, const CUtensorMap& tmU, co
   for (int c = 0; c < NCH; ++c) {
     const float* buf;
     if (!next_chunk<DK, DV, MP, TS>(c, uses, sA, bar, p, unit, m, buf)) {
-      if (lane == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
-      return false;   // the unit keeps R + W columns; the slots written so far hold partial results
+      // slots of the chunks before c already hold results: the unit no longer
+      // represents its state, so it is marked invalid (column count -1) instead of
+      // being left at R + W for the Householder kernel, which would compress the
+      // mixture; later calls flag it with SEED_FLAG_BADCOLS and leave it alone
+      if (lane == 0) {
+        if (c > 0) p.ncols[unit] = -1;
+        raise_flag(p.status, SEED_FLAG_TIMEOUT);
+      }
+      return false;
     }
     const bool isU = c < NCU;
     const int r0 = 32 * (isU ? c : c - NCU);

@@ -338,26 +338,20 @@ static int launch_one(const DecodeParams& p, cudaStream_t st) {
   const size_t smem = NS * sizeof(Stage) + 2 * NS * sizeof(uint64_t);
   auto kern = decode_step_kernel<FORM, DK, DV, MAXC, NS, TS>;
   // per device: the shared-memory opt-in and the resident CTAs per SM
-  constexpr int kMaxDev = 64;
-  static int grid_per_sm[kMaxDev] = {0};
-  static int sm_count[kMaxDev] = {0};
+  static LaunchCache cache;
+  static std::atomic<int> grid_per_sm[kMaxDev];
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return SEED_ERR_CUDA;
-  if (grid_per_sm[dev] == 0) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
+  if (const int rc = cache.prepare(reinterpret_cast<const void*>(kern), smem, &dev)) return rc;
+  int per_sm = grid_per_sm[dev].load(std::memory_order_relaxed);
+  if (per_sm == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kDecodeThreads, smem) != cudaSuccess)
       return SEED_ERR_CUDA;
-    int n = 0, sms = 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return SEED_ERR_CUDA;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kDecodeThreads, smem) !=
-        cudaSuccess)
-      return SEED_ERR_CUDA;
-    sm_count[dev] = sms;
-    grid_per_sm[dev] = n > 0 ? n : 1;
+    per_sm = n > 0 ? n : 1;
+    grid_per_sm[dev].store(per_sm, std::memory_order_relaxed);
   }
   const int units = p.B * p.H;
-  int grid = grid_per_sm[dev] * sm_count[dev];
+  int grid = per_sm * cache.sm_count[dev].load(std::memory_order_relaxed);
   if (grid > units) grid = units;
   kern<<<grid, kDecodeThreads, smem, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? SEED_OK : SEED_ERR_CUDA;

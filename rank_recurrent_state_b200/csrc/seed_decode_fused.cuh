@@ -39,24 +39,18 @@ static int launch_fused_t(const DecodeParams& p, const FastParams& fp, cudaStrea
   auto kern = decode_compress_warp_kernel<FORM, DK, DV, MAXC, TS, MP>;
   const int m = p.R + p.W, maxc = m - 1;
   const size_t smem = fused_smem<FORM, DK, DV, MP, TS>(maxc);
-  constexpr int kMaxDev = 64;
-  static bool attr_set[kMaxDev] = {false};
-  static int sm_count[kMaxDev] = {0};
-  static int grid_per_sm[kMaxDev][MAXC + 1] = {};
+  static LaunchCache cache;
+  static std::atomic<int> grid_per_sm[kMaxDev][MAXC + 1];
+  if (maxc > MAXC) return SEED_ERR_CUDA;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev || maxc > MAXC) return SEED_ERR_CUDA;
-  if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)fused_smem<FORM, DK, DV, MP, TS>(MAXC)) != cudaSuccess)
-      return SEED_ERR_CUDA;
-    if (cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return SEED_ERR_CUDA;
-    attr_set[dev] = true;
-  }
-  if (grid_per_sm[dev][maxc] == 0) {
+  if (const int rc = cache.prepare(reinterpret_cast<const void*>(kern), fused_smem<FORM, DK, DV, MP, TS>(MAXC), &dev))
+    return rc;
+  int per_sm = grid_per_sm[dev][maxc].load(std::memory_order_relaxed);
+  if (per_sm == 0) {
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 32, smem) != cudaSuccess) return SEED_ERR_CUDA;
-    grid_per_sm[dev][maxc] = n > 0 ? n : 1;
+    per_sm = n > 0 ? n : 1;
+    grid_per_sm[dev][maxc].store(per_sm, std::memory_order_relaxed);
   }
   CUtensorMap tmU, tmV;
   memset(&tmU, 0, sizeof(tmU));
@@ -67,7 +61,7 @@ static int launch_fused_t(const DecodeParams& p, const FastParams& fp, cudaStrea
        !make_panel_map(&tmV, static_cast<const float*>(p.V), DV, m, all_units, MP)))
     return SEED_ERR_CUDA;
   const int units = p.B * p.H;
-  int grid = grid_per_sm[dev][maxc] * sm_count[dev];
+  int grid = per_sm * cache.sm_count[dev].load(std::memory_order_relaxed);
   if (grid > units) grid = units;
   kern<<<grid, 32, smem, st>>>(p, fp, tmU, tmV);
   return cudaGetLastError() == cudaSuccess ? SEED_OK : SEED_ERR_CUDA;

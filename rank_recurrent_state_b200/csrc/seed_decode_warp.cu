@@ -16,27 +16,21 @@ static int launch_warp_t(const DecodeParams& p, cudaStream_t st) {
   const size_t smem = warp_stage_bytes(maxc, DK, DV, sizeof(TS)) + coef_floats(MAXC) * sizeof(float) + 16;
   // per device: the shared-memory opt-in (for the largest stage), and the resident
   // blocks per SM for each stage size
-  constexpr int kMaxDev = 64;
-  static bool attr_set[kMaxDev] = {false};
-  static int sm_count[kMaxDev] = {0};
-  static int grid_per_sm[kMaxDev][MAXC + 1] = {};
+  static LaunchCache cache;
+  static std::atomic<int> grid_per_sm[kMaxDev][MAXC + 1];
+  if (maxc > MAXC) return SEED_ERR_CUDA;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev || maxc > MAXC) return SEED_ERR_CUDA;
-  if (!attr_set[dev]) {
-    const size_t smax = warp_stage_bytes(MAXC, DK, DV, sizeof(TS)) + coef_floats(MAXC) * sizeof(float) + 16;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smax) != cudaSuccess)
-      return SEED_ERR_CUDA;
-    if (cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return SEED_ERR_CUDA;
-    attr_set[dev] = true;
-  }
-  if (grid_per_sm[dev][maxc] == 0) {
+  const size_t smax = warp_stage_bytes(MAXC, DK, DV, sizeof(TS)) + coef_floats(MAXC) * sizeof(float) + 16;
+  if (const int rc = cache.prepare(reinterpret_cast<const void*>(kern), smax, &dev)) return rc;
+  int per_sm = grid_per_sm[dev][maxc].load(std::memory_order_relaxed);
+  if (per_sm == 0) {
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 32, smem) != cudaSuccess) return SEED_ERR_CUDA;
-    grid_per_sm[dev][maxc] = n > 0 ? n : 1;
+    per_sm = n > 0 ? n : 1;
+    grid_per_sm[dev][maxc].store(per_sm, std::memory_order_relaxed);
   }
   const int units = p.B * p.H;
-  int grid = grid_per_sm[dev][maxc] * sm_count[dev];
+  int grid = per_sm * cache.sm_count[dev].load(std::memory_order_relaxed);
   if (grid > units) grid = units;
   kern<<<grid, 32, smem, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? SEED_OK : SEED_ERR_CUDA;

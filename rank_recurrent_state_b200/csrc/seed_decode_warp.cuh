@@ -123,11 +123,13 @@ SEED_DEV void load_vecs(const DecodeParams& p, int u, int c, UnitVecs<FORM, DK, 
 // stage (U at sU, V at sV, in their stored type TS), completing on bar.  A unit
 // with an invalid column count gets no copies (the wait still ends).  A column is
 // d_k (d_v) values of at least 2 bytes, d >= 16: every copy is a multiple of 16 bytes.
+// withhold: announce the bytes but issue no copy (the injected wait fault).
 template <int DK, int DV, typename TS>
-SEED_DEV void issue_unit(const DecodeParams& p, TS* sU, TS* sV, uint64_t* bar, int u, int c, int m) {
+SEED_DEV void issue_unit(const DecodeParams& p, TS* sU, TS* sV, uint64_t* bar, int u, int c, int m,
+                         bool withhold = false) {
   const bool valid = c > 0 && c < m;
   mbar_arrive_expect_tx(bar, valid ? (uint32_t)(c * (DK + DV) * sizeof(TS)) : 0u);
-  if (!valid) return;
+  if (!valid || withhold) return;
   const long long unit = unit_index(p, u);
   bulk_g2s(sU, static_cast<const TS*>(p.U) + unit * (long long)m * DK, (uint32_t)(c * DK * sizeof(TS)), bar);
   bulk_g2s(sV, static_cast<const TS*>(p.V) + unit * (long long)m * DV, (uint32_t)(c * DV * sizeof(TS)), bar);
@@ -184,8 +186,9 @@ SEED_DEV void decode_warp_run(const DecodeParams& p, const FastParams* fp, const
   __syncwarp();
 
   // the first unit: its columns to the stage, its vectors to registers
+  const bool fault = wait_fault_injected(p.status);
   int c = p.ncols[unit_index(p, u0)];
-  if (lane == 0) issue_unit<DK, DV, TS>(p, sU, sV, full, u0, c, m);
+  if (lane == 0) issue_unit<DK, DV, TS>(p, sU, sV, full, u0, c, m, fault);
   Vecs cur, nxt;
   load_vecs<FORM, DK, DV>(p, u0, c, cur);
   int c_next = u0 + stride < n_units ? p.ncols[unit_index(p, u0 + stride)] : 0;
@@ -198,7 +201,8 @@ SEED_DEV void decode_warp_run(const DecodeParams& p, const FastParams* fp, const
     const int c_after = u_next + stride < n_units ? p.ncols[unit_index(p, u_next + stride)] : 0;
     const float g = cur.g, be = cur.be;
 
-    if (!__all_sync(0xffffffffu, mbar_wait_bounded(full, (uint32_t)i & 1u, kWaitLimitNs))) {
+    const uint64_t limit = (fault && i == 0) ? 0ull : kWaitLimitNs;
+    if (!__all_sync(0xffffffffu, mbar_wait_bounded(full, (uint32_t)i & 1u, limit))) {
       if (lane == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
       mbar_wait_bounded(full, (uint32_t)i & 1u, kWaitLimitNs);   // let the copies land before exit
       return;

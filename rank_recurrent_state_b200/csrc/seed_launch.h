@@ -2,15 +2,43 @@
 // Arguments are validated by seed_abi.cu before any of these is called.
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/seed.h"
 #include "../../include/seed_synth.h"
 
 namespace seed {
+
+constexpr int kMaxDev = 64;
+
+// Index (32-bit words from the status word) of the workspace word that turns on the
+// injected wait fault of the timeout tests (kWsWaitFaultWord in seed_common.cuh).
+constexpr int kWsWaitFaultWordHost = 8;
+
+// cuTensorMapEncodeTiled from the driver, looked up once (nullptr if unavailable).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+
+// Unique id of the calling thread's current CUDA context; 0 if there is none.
+unsigned long long current_context_id();
+
+// Per kernel instantiation and device: the SM count, and the context in which the
+// kernel's dynamic shared-memory opt-in was last set (a device reset loads the
+// module afresh, so the opt-in is set again in the new context).  Atomics: host
+// threads that launch at the same time for the first time store equal values.
+struct LaunchCache {
+  std::atomic<int> sm_count[kMaxDev];
+  std::atomic<unsigned long long> attr_ctx[kMaxDev];
+  // Current device into *dev; sets the opt-in for max_dyn_smem bytes when above
+  // the default 48 KB and not yet set in this context.
+  int prepare(const void* kernel, size_t max_dyn_smem, int* dev);
+};
 
 // Per-unit length of seed_state.scale: d_k for KDA (the decay product P), else
 // R + W rounded up to a multiple of 4 (column scales, 16-byte aligned per unit).

@@ -91,9 +91,11 @@ class DeviceRun:
                                   buf["q"], buf["k"], buf["v"], buf["alpha"], buf["beta"])
 
     def step(self, buf: dict, outs: list | None = None, sigma: torch.Tensor | None = None,
-             dense: bool = False) -> bool:
+             dense: bool = False, pre_compress=None) -> bool:
         """One decode step of every layer (inputs generated on the device), then the
-        compression if it is due.  Returns True when a compression ran."""
+        compression if it is due.  Returns True when a compression ran.  pre_compress:
+        called with no argument right before a separate compression launch (not with
+        the fused step), e.g. to read the states about to be compressed."""
         d = self.dims
         fuse = self.fused and (self.ragged or self.c + 1 == d.m)
         sig_l = None
@@ -120,10 +122,14 @@ class DeviceRun:
         self.t += 1
         if self.ragged:   # some request is due after every step: only its units compress
             if not fuse:
+                if pre_compress is not None:
+                    pre_compress()
                 S.seed_compress(d, self.state, S.SEED_ALL_LAYERS, self.ws, sigma_out=sigma)
             return True
         if self.c == d.m:
             if not fuse:
+                if pre_compress is not None:
+                    pre_compress()
                 S.seed_compress(d, self.state, S.SEED_ALL_LAYERS, self.ws, sigma_out=sigma)
             self.c = d.R
             return True

@@ -271,6 +271,11 @@ def seed_get_diagnostics(ws: Workspace, stream=None) -> dict:
             "compress_units": c[1] + c[4]}
 
 
+def seed_debug_wait_fault(ws: Workspace, enable: bool, stream=None) -> None:
+    _check("seed_debug_wait_fault",
+           _lib.load().seed_debug_wait_fault(ws.ptr, ws.nbytes, 1 if enable else 0, _stream(stream)))
+
+
 # ------------------------------------------------------------------ synthetic workloads
 
 def synth_key(cfg, b0: int = 0) -> _lib.seed_synth_key:

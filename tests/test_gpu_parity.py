@@ -10,7 +10,8 @@ import pytest
 
 from workloads import FORM_KDA, config, philox
 
-from parity_util import TOL, compare, ensure_lib, rel_fro, run_device, run_oracle
+from parity_util import TOL, compare, ensure_lib, record_set, rel_fro, run_device, run_oracle
+from workloads import KDA_SWEEP_R, KDA_SWEEP_W
 
 pytestmark = pytest.mark.gpu
 
@@ -80,11 +81,15 @@ def test_dense_prefill_matches_oracle(cid, batch, T):
 
 # --------------------------------------------------------------- whole decode path
 
-def _parity(cfg, sample, n_prefill, n_decode, batch=None):
-    dev = run_device(cfg, sample, n_prefill, n_decode, batch=batch)
+def _parity(cfg, sample, n_prefill, n_decode, batch=None, label=None):
+    c = cfg if batch is None else cfg.replace(batch=batch)
+    su = np.asarray(sample, dtype=np.int64)
+    b, rem = np.divmod(su, c.layers * c.heads)
+    l, h = np.divmod(rem, c.heads)
+    ref = run_oracle(cfg, {"b": b, "l": l, "h": h}, n_prefill, n_decode)
+    dev = run_device(cfg, sample, n_prefill, n_decode, batch=batch, record_units=record_set(cfg, ref))
     assert dev["flags"] == 0, hex(dev["flags"])
-    ref = run_oracle(cfg, dev, n_prefill, n_decode)
-    return compare(cfg, dev, ref)
+    return compare(cfg, dev, ref, label=label)
 
 
 def test_tiny_gdn_workload_full():
@@ -108,13 +113,14 @@ def test_mamba2_reduced():
     _parity(cfg, sample, 200, 2 * cfg.W + 3, batch=1)
 
 
-@pytest.mark.parametrize("R,W", [(8, 8), (16, 16), (16, 32), (32, 32), (32, 64), (8, 64)])
+@pytest.mark.parametrize("R,W", [(r, w) for r in KDA_SWEEP_R for w in KDA_SWEEP_W])
 def test_kda_sweep_reduced(R, W):
-    """KDA 128x128 with per-channel decay over the R, W sweep (one request, sampled heads)."""
+    """KDA 128x128 with per-channel decay over the whole R x W sweep, R in {8, 16, 32},
+    W in {8, 16, 32, 64} (one request, 24 sampled heads, two compressions)."""
     cfg = config(4, R=R, W=W)
     rng = np.random.default_rng(R * 100 + W)
     sample = np.sort(rng.choice(cfg.layers * cfg.heads, 24, replace=False))
-    _parity(cfg, sample, 150, 2 * W + 2, batch=1)
+    _parity(cfg, sample, 150, 2 * W + 2, batch=1, label=f"kda R{R} W{W} reduced")
 
 
 def test_odd_window_and_empty_prefill():

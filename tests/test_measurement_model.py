@@ -82,3 +82,22 @@ def test_kernel_launch_counts():
     assert bench.compress_kernel_launches(m2) == 1 and bench.compress_kernel_launches(tiny) == 1
     assert bench.fused_kernel_launches(gdn) == 2
     assert bench.fused_kernel_launches(m2) == 2 and bench.fused_kernel_launches(tiny) == 2
+
+
+def test_bench_steady_state_is_independent_of_the_timed_window():
+    """The headline step time is that of one compression window whatever K steps the
+    window held: t_step = (sum_c layers x t_dec(c) + t_cmp) / W, column counts the
+    window missed filled by the line through the measured ones."""
+    import bench
+    R, W, L = 16, 16, 36
+    t_dec = lambda c: 0.040 + 0.001 * c   # noqa: E731  (ms, linear in the columns)
+    t_cmp = 40.0
+    exact = (L * sum(t_dec(c) for c in range(R, R + W)) + t_cmp) / W
+    for warmup, steps in ((5, 20), (16, 320), (3, 7), (0, 16)):
+        dec = []
+        c = R + warmup % W
+        for s in range(steps):
+            dec += [(t_dec(c), c)] * L
+            c = R if c + 1 == R + W else c + 1
+        st = bench.steady_state(dec, [t_cmp], R, W, L)
+        assert abs(st["ms_per_step"] - exact) <= 1e-9 * exact, (warmup, steps, st)

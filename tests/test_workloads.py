@@ -80,3 +80,19 @@ def test_configs_are_the_five_workloads():
     assert sorted(CONFIGS) == [0, 1, 2, 3, 4]
     assert CONFIGS[2].units == 256 * 36 * 48
     assert [CONFIGS[i].form for i in range(5)] == [FORM_GDN] * 3 + [FORM_MAMBA2, FORM_KDA]
+
+
+def test_philox_matches_published_known_answer_vectors(golden_dir):
+    """The host generator against the published Philox4x32-10 known-answer vectors
+    (tests/golden/philox4x32_10_kat.txt); the device generator is tested equal to
+    the host one value by value, so this pins both."""
+    import os
+    rows = []
+    with open(os.path.join(golden_dir, "philox4x32_10_kat.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                rows.append([int(x, 16) for x in line.split()])
+    assert len(rows) == 3
+    for r in rows:
+        out = philox.philox4x32_10(*r[:4], *r[4:6])
+        assert [int(x) for x in out] == r[6:10]

@@ -11,8 +11,9 @@ no compression).  The CUDA library carries its own, independently written
 Philox generator for the same counters; the tests check that the two agree.
 """
 
-from .configs import CONFIGS, Config, FORM_GDN, FORM_KDA, FORM_MAMBA2, FORM_NAMES, config
+from .configs import (CONFIGS, Config, FORM_GDN, FORM_KDA, FORM_MAMBA2, FORM_NAMES, KDA_SWEEP_R,
+                      KDA_SWEEP_W, config)
 from . import philox
 
-__all__ = ["CONFIGS", "Config", "FORM_GDN", "FORM_KDA", "FORM_MAMBA2", "FORM_NAMES",
-           "config", "philox"]
+__all__ = ["CONFIGS", "Config", "FORM_GDN", "FORM_KDA", "FORM_MAMBA2", "FORM_NAMES", "KDA_SWEEP_R",
+           "KDA_SWEEP_W", "config", "philox"]
