@@ -36,16 +36,11 @@ METRIC = "decode head-steps/s and achieved HBM GB/s (% of B200 peak) at R=16,W=1
 UNIT = "head-steps/s"
 NOMINAL_HBM_GBS = 8000.0
 # DRAM bytes (read + write) of one decode launch, measured by ncu (dram__bytes_read.sum +
-# dram__bytes_write.sum; profiles/decode_warp_kernel_*gdn_stack_2layers.md) for a full
-# per-layer launch of the GDN stack shape (256 requests x 48 heads) at c = 19 stored
-# columns, per factor format.  Set an entry to None whenever that kernel changes, until
-# it is measured again.
-NCU_DECODE_TRAFFIC = [
-    {"kernel": "decode_warp_kernel", "form": 0, "d_k": 128, "d_v": 128, "R": 16, "W": 16, "factors": 0,
-     "units": 12288, "c": 19, "bytes": 266.032e6 + 20.088e6},
-    {"kernel": "decode_warp_kernel", "form": 0, "d_k": 128, "d_v": 128, "R": 16, "W": 16, "factors": 1,
-     "units": 12288, "c": 19, "bytes": 146.493e6 + 10.716e6},
-]
+# dram__bytes_write.sum; profiles/decode_ring_kernel_*gdn_stack_2layers.md) for a full
+# per-layer launch of the GDN stack shape (256 requests x 48 heads) at c stored columns,
+# per factor format.  Remove an entry whenever that kernel changes, until it is measured
+# again (no entry: the line's roofline.traffic is null).
+NCU_DECODE_TRAFFIC = []
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -338,7 +333,7 @@ def run_reference(args, world, rank):
 # ------------------------------------------------------------------ GPU arm
 
 def decode_kernel_name(d):
-    return "decode_warp_kernel" if d.R + d.W - 1 <= 64 else "decode_step_kernel"
+    return "decode_ring_kernel" if d.R + d.W - 1 <= 64 else "decode_step_kernel"
 
 
 def decode_traffic(d, units, cbar):
@@ -358,10 +353,13 @@ def decode_traffic(d, units, cbar):
 
 
 def compress_kernel_launches(d) -> int:
-    """Kernels one seed_compress call launches: the fast (Cholesky-QR) kernel where the
-    shape allows it, then the Householder scan over the units still due."""
-    fast = d.R + d.W <= 32 and d.R <= 16 and d.d_k in (64, 128) and d.d_v in (64, 128)
-    return 2 if fast else 1
+    """Kernels one seed_compress call launches: a Cholesky-QR kernel where the shape
+    allows one (R + W <= 32 with R <= 16, or 32 < R + W <= 64 with R <= 32; d_k, d_v in
+    {64, 128}), then the Householder scan over the units still due."""
+    dims_ok = d.d_k in (64, 128) and d.d_v in (64, 128)
+    fast = d.R + d.W <= 32 and d.R <= 16
+    wide = 32 < d.R + d.W <= 64 and d.R <= 32
+    return 2 if dims_ok and (fast or wide) else 1
 
 
 def fused_kernel_launches(d) -> int:

@@ -231,6 +231,34 @@ int seed_state_energy(const seed_dims* dims, const seed_state* state, int32_t la
                       const int32_t* units, int32_t n_units, float* out, void* ws, size_t ws_bytes,
                       void* stream);
 
+/* Singular spectra and the top output direction of the stored states (SEED figures &
+ * tables, Figure 3 (e): the spectra of the state and of the content, divided by the
+ * head's top singular value; Figure 3 (h): |cos| between the head's top output
+ * direction v* and vbar; Figure 13 (a): the energy share of the state's i-th
+ * singular direction, sigma_i^2 / sum_j sigma_j^2; Figure 13 (d): the rank that holds
+ * 90% and 99% of the content's energy).  For the listed units of `layer` (or all
+ * layers; units and n_units as in seed_state_to_dense, NULL = every unit in scope):
+ *   sigma_state    [n][R+W+1] float  the largest R+W+1 singular values of
+ *                                    S = a vbar^T + U V^T (true U), descending; S has
+ *                                    rank at most ncols + 1 <= R+W+1
+ *   sigma_content  [n][R+W+1] float  the same for the content C = U V^T
+ *   cos_top        [n] float         |v*^T vbar| / ||vbar||, v* the right singular vector
+ *                                    of S's largest singular value (o = S^T q lies in the
+ *                                    span of the right singular vectors)
+ *   ranks          [n][2] int32      the smallest k whose k largest singular values of C
+ *                                    hold 90% (ranks[.][0]) and 99% ([.][1]) of
+ *                                    ||C||_F^2; 0 for a zero content
+ * Computed in float32 by a one-sided Jacobi SVD of the explicit d_k x d_v matrices (a
+ * diagnostic: about a millisecond per hundred 128 x 128 units, not for the decode
+ * loop).  Reads the state only.  Device flags: SEED_FLAG_BADINDEX for a unit index
+ * outside the scope (its rows are not written), SEED_FLAG_BADCOLS for a column count
+ * outside [0, R+W] (the unit is taken as holding none), SEED_FLAG_NOCONVERGE if a
+ * Jacobi SVD reached its sweep cap.                                               */
+int seed_state_spectrum(const seed_dims* dims, const seed_state* state, int32_t layer,
+                        const int32_t* units, int32_t n_units, float* sigma_state,
+                        float* sigma_content, float* cos_top, int32_t* ranks, void* ws,
+                        size_t ws_bytes, void* stream);
+
 /* The dense-state step that SEED replaces, kept as the in-run comparison: every
  * decode step loads and stores whole recurrent states (SEED abstract, readsearch.ai).
  * One step of `layer` on a dense state S [B][L][H][d_k][d_v] with the form's dense

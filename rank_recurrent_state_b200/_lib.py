@@ -51,6 +51,9 @@ SIGNATURES = {
                                            c_void_p, c_int32, c_void_p, c_void_p, c_size_t, c_void_p]),
     "seed_state_energy": (ctypes.c_int, [ctypes.POINTER(seed_dims), ctypes.POINTER(seed_state), c_int32,
                                          c_void_p, c_int32, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "seed_state_spectrum": (ctypes.c_int, [ctypes.POINTER(seed_dims), ctypes.POINTER(seed_state), c_int32,
+                                           c_void_p, c_int32, c_void_p, c_void_p, c_void_p, c_void_p,
+                                           c_void_p, c_size_t, c_void_p]),
     "seed_dense_step": (ctypes.c_int, [ctypes.POINTER(seed_dims), c_void_p, c_int32, c_void_p, c_void_p,
                                        c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                        c_void_p]),

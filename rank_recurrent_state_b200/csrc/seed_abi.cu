@@ -183,6 +183,29 @@ int seed_state_energy(const seed_dims* dims, const seed_state* state, int32_t la
                                    as_stream(stream));
 }
 
+int seed_state_spectrum(const seed_dims* dims, const seed_state* state, int32_t layer, const int32_t* units,
+                        int32_t n_units, float* sigma_state, float* sigma_content, float* cos_top,
+                        int32_t* ranks, void* ws, size_t ws_bytes, void* stream) {
+  SEED_TRY(check_dims(dims));
+  SEED_TRY(check_layer(dims, layer, true));
+  SEED_TRY(check_state(state));
+  SEED_TRY(check_ptr(sigma_state));
+  SEED_TRY(check_ptr(sigma_content));
+  SEED_TRY(check_ptr(cos_top));
+  SEED_TRY(check_ptr(ranks));
+  SEED_TRY(check_ws(ws, ws_bytes));
+  const long long scope = (long long)dims->batch * dims->heads * (layer < 0 ? dims->layers : 1);
+  if (units) {
+    if (n_units < 0 || n_units > scope) return SEED_ERR_INVALID_ARG;
+    if (n_units == 0) return SEED_OK;
+    SEED_TRY(check_ptr(units));
+  } else {
+    n_units = (int32_t)scope;
+  }
+  return seed::launch_state_spectrum(*dims, *state, layer, units, n_units, sigma_state, sigma_content, cos_top,
+                                     ranks, status_word(ws), as_stream(stream));
+}
+
 int seed_dense_step(const seed_dims* dims, float* S, int32_t layer, const float* q, const float* k,
                     const float* v, const float* alpha, const float* beta, float* o, void* ws,
                     size_t ws_bytes, void* stream) {

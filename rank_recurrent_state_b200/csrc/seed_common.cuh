@@ -62,6 +62,13 @@ SEED_DEV T fac_from_f(float x) {
   else return x;
 }
 
+// One factor value stored with the streaming hint (evict first: not read again soon).
+template <typename T>
+SEED_DEV void fac_st_stream(T* p, float x) {
+  if constexpr (std::is_same<T, float>::value) __stcs(p, x);
+  else *p = fac_from_f<T>(x);
+}
+
 // The value x has once stored as T.
 template <typename T>
 SEED_DEV float fac_round(float x) { return fac_to_f(fac_from_f<T>(x)); }

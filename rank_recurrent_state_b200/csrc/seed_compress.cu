@@ -395,6 +395,9 @@ int launch_compress(const seed_dims& d, const seed_state& s, int layer, float* s
   if (compress_fast_supported(d)) {
     const int rc = launch_compress_fast(d, s, layer, sigma_out, status, st);
     if (rc != SEED_OK) return rc;
+  } else if (compress_wide_supported(d)) {
+    const int rc = launch_compress_wide(d, s, layer, sigma_out, status, st);
+    if (rc != SEED_OK) return rc;
   }
   return launch_compress_householder(d, s, layer, sigma_out, status, st);
 }

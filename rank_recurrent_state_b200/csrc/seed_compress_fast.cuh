@@ -9,8 +9,9 @@
 //      16-bit factors: cp.async into staging buffers, widened to float32 in the
 //      same layout); the Gram matrix G = U^T U accumulates on the tensor cores
 //      (mma.sync TF32 with a three-term hi/lo split, float32 accuracy), is
-//      equilibrated by the column norms and factored by Cholesky in registers
-//      (L_u); then the V panel the same way (L_v).  So U = Q_u R_u, V = Q_v R_v
+//      equilibrated by the column norms and factored by Cholesky in shared memory
+//      (L_u; right-looking, lane = row, each step's column broadcast from shared
+//      memory); then the V panel the same way (L_v).  So U = Q_u R_u, V = Q_v R_v
 //      with R = L^T D (D the column norms, and the lazy decay scales for GDN /
 //      Mamba-2);
 //   2. the core M = R_u R_v^T = L_u^T D_u D_v L_v (m x m);
@@ -96,53 +97,104 @@ SEED_DEV void gram_row(const float* P, float (&acc)[MP]) {
   }
 }
 
-// Equilibrate the Gram row held by lane i (divide by the column norms) and return
-// the norm of column i.  Row i of the result is Uhat^T Uhat restricted to row i.
-template <int MP>
-SEED_DEV float equilibrate_row(float (&g)[MP]) {
+// Equilibrate the Gram G (MP x MP, row-major, stride LG; columns at or beyond m are
+// zero) by its column norms and factor it by Cholesky in place, one warp, lane i
+// owning rows i and i + 32 (MP <= 64).  Right-looking: at step j the column below the pivot is
+// scaled and copied to colj, then every lane updates its rows below j against it
+// (whole rows, 128-bit accesses; the part above the diagonal is not read and is zeroed
+// at the end).  On return G[i * LG + j] = L[i][j] for j <= i, 0 above, and nrm holds
+// the column norms.  A zero column, or a non-positive pivot, gives a zero column of L;
+// a pivot below kCholPivotMin on a nonzero column also sets bad.
+template <int MP, int LG>
+SEED_DEV void cholesky_wide(float* G, int m, float* nrm, float* ninv, float* colj, bool& bad) {
   const int lane = threadIdx.x & 31;
-  float d = 0.f;
+  constexpr int RPL = (MP + 31) / 32;
 #pragma unroll
-  for (int i = 0; i < MP; ++i)
-    if (i == lane) d = g[i];
-  const float n = sqrtf(fmaxf(d, 0.f));
-  const float ninv = n > 0.f ? 1.f / n : 0.f;
+  for (int h = 0; h < RPL; ++h) {
+    const int i = lane + 32 * h;
+    if (i >= MP) continue;
+    const float n = i < m ? sqrtf(fmaxf(G[i * LG + i], 0.f)) : 0.f;
+    nrm[i] = n;
+    ninv[i] = n > 0.f ? 1.f / n : 0.f;
+  }
+  __syncwarp();
 #pragma unroll
-  for (int i = 0; i < MP; ++i) g[i] *= __shfl_sync(kFull, ninv, i) * ninv;
-  return lane < MP ? n : 0.f;
-}
-
-// Right-looking Cholesky of the equilibrated Gram, one warp, lane i holding row i
-// in registers; row i of L (lower, zero above the diagonal) is written to
-// L[i * LD ..].  The column loop is not unrolled, to keep the code small: after
-// step j every row is shifted down by one register, so that the current column is
-// always g[0].  Column j is dropped (zero) when column j of the panel is zero
-// (norm_j == 0) or the pivot is not positive; a pivot below kCholPivotMin on a
-// nonzero column sets `bad`.
-template <int MP, int LD>
-SEED_DEV void cholesky_rolled(float (&g)[MP], float norm_self, bool& bad, float* L) {
-  const int lane = threadIdx.x & 31;
+  for (int h = 0; h < RPL; ++h) {
+    const int i = lane + 32 * h;
+    if (i >= MP) continue;
+    const float fi = ninv[i];
+#pragma unroll
+    for (int j4 = 0; j4 < MP; j4 += 4) {
+      float4 g = ld4(G + i * LG + j4);
+      const float4 n4 = ld4(ninv + j4);
+      g.x *= fi * n4.x; g.y *= fi * n4.y; g.z *= fi * n4.z; g.w *= fi * n4.w;
+      st4(G + i * LG + j4, g);
+    }
+  }
+  __syncwarp();
 #pragma unroll 1
-  for (int j = 0; j < MP; ++j) {
-    const float d = __shfl_sync(kFull, g[0], j);
-    const bool zero = !(__shfl_sync(kFull, norm_self, j) > 0.f);
+  for (int j = 0; j < m; ++j) {
+    const float d = G[j * LG + j];
+    const bool zero = !(nrm[j] > 0.f);
     bool drop = zero || !(d > 0.f);
     if (!zero && d < kCholPivotMin) {
       drop = true;
       bad = true;
     }
     const float rs = drop ? 0.f : rsqrtf(d);
-    const float lij = lane > j ? g[0] * rs : 0.f;
-    if (lane < MP) L[lane * LD + j] = lane == j ? d * rs : lij;
+    __syncwarp();   // every lane has read the pivot before its row is rewritten
+    float l[RPL];
 #pragma unroll
-    for (int t = 1; t < MP; ++t) {   // column j + t of the rows below
-      const float lkj = __shfl_sync(kFull, lij, (j + t) & 31);
-      if (j + t <= lane) g[t] = fmaf(-lij, lkj, g[t]);
+    for (int h = 0; h < RPL; ++h) {
+      const int i = lane + 32 * h;
+      l[h] = 0.f;
+      if (i >= MP) continue;
+      if (i > j) {
+        l[h] = G[i * LG + j] * rs;
+        G[i * LG + j] = l[h];
+      } else if (i == j) {
+        G[i * LG + i] = drop ? 0.f : d * rs;
+      }
+      colj[i] = l[h];   // L[i][j] below the diagonal, 0 elsewhere
     }
+    __syncwarp();
+    const int c0 = (j + 1) & ~3;
 #pragma unroll
-    for (int t = 0; t + 1 < MP; ++t) g[t] = g[t + 1];
-    g[MP - 1] = 0.f;
+    for (int h = 0; h < RPL; ++h) {
+      const int i = lane + 32 * h;
+      if (i > j && i < m && l[h] != 0.f) {
+        const float lij = l[h];
+#pragma unroll 2
+        for (int c4 = c0; c4 < m; c4 += 4) {
+          const float4 lc = ld4(colj + c4);
+          float4 g = ld4(G + i * LG + c4);
+          g.x = fmaf(-lij, lc.x, g.x);
+          g.y = fmaf(-lij, lc.y, g.y);
+          g.z = fmaf(-lij, lc.z, g.z);
+          g.w = fmaf(-lij, lc.w, g.w);
+          st4(G + i * LG + c4, g);
+        }
+      }
+    }
+    __syncwarp();   // the updated rows, and colj free again
   }
+#pragma unroll
+  for (int h = 0; h < RPL; ++h) {
+    const int i = lane + 32 * h;
+    if (i >= MP) continue;
+#pragma unroll
+    for (int j4 = 0; j4 < MP; j4 += 4) {
+      float4 g = ld4(G + i * LG + j4);
+      if (j4 > i || i >= m) g = zero4();
+      else {
+        if (j4 + 1 > i) g.y = 0.f;
+        if (j4 + 2 > i) g.z = 0.f;
+        if (j4 + 3 > i) g.w = 0.f;
+      }
+      st4(G + i * LG + j4, g);
+    }
+  }
+  __syncwarp();
 }
 
 // Lanes of one column pair (LP lanes, aligned) sum their partial values.
@@ -302,16 +354,20 @@ SEED_DEV int jacobi_regs(float* sM, bool& conv) {
 // bar[c & 1].  Columns m .. MP-1 lie outside the tensor and arrive as zeros.  In
 // shared memory column j is a 128-byte row whose 16-byte pieces are permuted by
 // the 128-byte swizzle: piece f sits at f ^ (j & 7).
-// withhold: announce the bytes but issue no copy (the injected wait fault).
+// withhold: announce the bytes but issue no copy (the injected wait fault).  last:
+// the second pass, the panel's last read (evict_first); the first pass keeps its
+// lines in L2 (evict_last) for the second, which follows after the core SVD.
 template <int NCU, int CHUNK>
 SEED_DEV void issue_chunk(int c, float* sA, const CUtensorMap* tmU, const CUtensorMap* tmV, long long unit,
-                          uint64_t* bar, bool withhold = false) {
+                          uint64_t* bar, bool withhold = false, bool last = false) {
   const int bb = c & 1;
   const bool isU = c < NCU;
   const int r0 = 32 * (isU ? c : c - NCU);
   if ((threadIdx.x & 31) == 0) {
     mbar_arrive_expect_tx(&bar[bb], (uint32_t)(CHUNK * 4));
-    if (!withhold) tma_load_3d(sA + bb * CHUNK, isU ? tmU : tmV, r0, 0, (int)unit, &bar[bb]);
+    if (!withhold)
+      tma_load_3d_hint(sA + bb * CHUNK, isU ? tmU : tmV, r0, 0, (int)unit, &bar[bb],
+                       last ? l2_policy_evict_first() : l2_policy_evict_last());
   }
 }
 
@@ -537,10 +593,10 @@ struct FastLayout {
 // Chunks 0 and 1 of a stream.
 template <int DK, int DV, int MP, typename TS>
 SEED_DEV void start_stream(float* sA, const CUtensorMap* tmU, const CUtensorMap* tmV, const FastParams& p,
-                           long long unit, int m, uint64_t* bar, bool withhold = false) {
+                           long long unit, int m, uint64_t* bar, bool withhold = false, bool last = false) {
   if constexpr (std::is_same<TS, float>::value) {
-    issue_chunk<DK / 32, MP * 32>(0, sA, tmU, tmV, unit, bar, withhold);
-    issue_chunk<DK / 32, MP * 32>(1, sA, tmU, tmV, unit, bar);
+    issue_chunk<DK / 32, MP * 32>(0, sA, tmU, tmV, unit, bar, withhold, last);
+    issue_chunk<DK / 32, MP * 32>(1, sA, tmU, tmV, unit, bar, false, last);
   } else {
     issue_chunk16<DK, DV, MP, TS>(0, sA, p, unit, m);
     issue_chunk16<DK, DV, MP, TS>(1, sA, p, unit, m);
@@ -597,23 +653,16 @@ SEED_DEV bool compress_fast_unit(const FastParams& p, const CUtensorMap& tmU, co
     if (lane == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
     return false;
   }
-  {
-    const float n = equilibrate_row<MP>(g);
-    if (lane < MP) nu[lane] = n;
-    cholesky_rolled<MP, LG>(g, n, bad, sLu);
-  }
+  // equilibrated Cholesky in shared memory; nrm and du are free until after both
+  // factorisations and serve as its scratch
+  cholesky_wide<MP, LG>(sLu, m, nu, nrm, du, bad);
   // V: chunks NCU .. NCH-1; L_v over the chunk buffers once the last one is read
   if (!gram_stream<KDA, DK, DV, MP, LG, TS>(NCU, NCH, false, sA, &tmU, &tmV, p, unit, m, bar, uses, scl, sM,
                                             g, bad)) {
     if (lane == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
     return false;
   }
-  {
-    const float n = equilibrate_row<MP>(g);
-    if (lane < MP) nv[lane] = n;
-    __syncwarp();   // every lane has read the last V chunk before L_v overwrites it
-    cholesky_rolled<MP, LG>(g, n, bad, sM);
-  }
+  cholesky_wide<MP, LG>(sM, m, nv, nrm, du, bad);
   if (__any_sync(kFull, bad)) {
     if (lane == 0) atomicAdd(p.status + 6, 1u);
     return true;
@@ -803,7 +852,7 @@ SEED_DEV bool compress_fast_unit(const FastParams& p, const CUtensorMap& tmU, co
   //    holds them, so slots 0..R-1 can be overwritten in place.
   fence_proxy_async_smem();   // the chunk buffers were written with ordinary stores
   __syncwarp();
-  start_stream<DK, DV, MP, TS>(sA, &tmU, &tmV, p, unit, m, bar);
+  start_stream<DK, DV, MP, TS>(sA, &tmU, &tmV, p, unit, m, bar, false, true);
   bool nonfinite = false;
   TS* Uo = static_cast<TS*>(p.U) + unit * (long long)m * DK;
   TS* Vo = static_cast<TS*>(p.V) + unit * (long long)m * DV;
@@ -856,7 +905,8 @@ SEED_DEV bool compress_fast_unit(const FastParams& p, const CUtensorMap& tmU, co
       }
     }
     __syncwarp();   // every lane has read this chunk before the next copy overwrites it
-    if (std::is_same<TS, float>::value && c + 2 < NCH) issue_chunk<NCU, CHUNK>(c + 2, sA, &tmU, &tmV, unit, bar);
+    if (std::is_same<TS, float>::value && c + 2 < NCH)
+      issue_chunk<NCU, CHUNK>(c + 2, sA, &tmU, &tmV, unit, bar, false, true);
     TS* out = (isU ? Uo : Vo) + r0;
     const int ld = isU ? DK : DV;
 #pragma unroll
@@ -873,7 +923,7 @@ SEED_DEV bool compress_fast_unit(const FastParams& p, const CUtensorMap& tmU, co
             if (q < p.R) {
               const float v = acc[mt][nt][2 * hh + e] * rowf;
               nonfinite |= !isfinite(fac_round<TS>(v));
-              out[(long long)q * ld + r] = fac_from_f<TS>(v);
+              fac_st_stream<TS>(out + (long long)q * ld + r, v);
             }
           }
         }

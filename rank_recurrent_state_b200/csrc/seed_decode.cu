@@ -366,7 +366,7 @@ static int launch_cols_t(const DecodeParams& p, cudaStream_t st) {
 
 template <int FORM, int DK, int DV>
 static int launch_cols(const DecodeParams& p, int factors, cudaStream_t st) {
-  if (p.R + p.W - 1 <= 64) return launch_decode_warp(p, FORM, DK, DV, factors, st);
+  if (p.R + p.W - 1 <= 64) return launch_decode_ring(p, FORM, DK, DV, factors, st);
   switch (factors) {
     case SEED_FACTORS_F32: return launch_cols_t<FORM, DK, DV, float>(p, st);
     case SEED_FACTORS_F16: return launch_cols_t<FORM, DK, DV, __half>(p, st);

@@ -74,7 +74,8 @@ SEED_DEV float warp_xreduce(float (&v)[NV]) {
 template <int NV>
 SEED_DEV constexpr int log2c() { return NV <= 1 ? 0 : 1 + log2c<NV / 2>(); }
 
-// The one-warp-per-unit decode kernel (seed_decode_warp.cu), for R + W - 1 <= 64.
-int launch_decode_warp(const DecodeParams& p, int form, int dk, int dv, int factors, cudaStream_t st);
+// The one-warp-per-unit decode kernel with a ring of column chunks
+// (seed_decode_ring.cu), for R + W - 1 <= 64: the decode step's kernel there.
+int launch_decode_ring(const DecodeParams& p, int form, int dk, int dv, int factors, cudaStream_t st);
 
 }  // namespace seed

@@ -61,8 +61,7 @@ static int launch_fused_t(const DecodeParams& p, const FastParams& fp, cudaStrea
        !make_panel_map(&tmV, static_cast<const float*>(p.V), DV, m, all_units, MP)))
     return SEED_ERR_CUDA;
   const int units = p.B * p.H;
-  int grid = per_sm * cache.sm_count[dev].load(std::memory_order_relaxed);
-  if (grid > units) grid = units;
+  const int grid = balanced_grid(units, per_sm * cache.sm_count[dev].load(std::memory_order_relaxed));
   kern<<<grid, 32, smem, st>>>(p, fp, tmU, tmV);
   return cudaGetLastError() == cudaSuccess ? SEED_OK : SEED_ERR_CUDA;
 }

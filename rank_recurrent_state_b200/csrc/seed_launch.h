@@ -28,6 +28,18 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 // Unique id of the calling thread's current CUDA context; 0 if there is none.
 unsigned long long current_context_id();
 
+// Blocks of a persistent grid of at most max_blocks that deal `units` units round
+// robin so that every block takes the same number of units, up to one: with
+// k = ceil(units / max_blocks) units per block, ceil(units / k) blocks.  (A grid of
+// max_blocks itself would leave a last round in which only units mod max_blocks
+// blocks work.)
+inline int balanced_grid(int units, int max_blocks) {
+  if (units <= 0) return 1;
+  if (max_blocks < 1) max_blocks = 1;
+  const int k = (units + max_blocks - 1) / max_blocks;
+  return (units + k - 1) / k;
+}
+
 // Per kernel instantiation and device: the SM count, and the context in which the
 // kernel's dynamic shared-memory opt-in was last set (a device reset loads the
 // module afresh, so the opt-in is set again in the new context).  Atomics: host
@@ -70,6 +82,11 @@ bool compress_fast_supported(const seed_dims& d);
 int launch_compress_fast(const seed_dims& d, const seed_state& s, int layer, float* sigma_out,
                          uint32_t* status, cudaStream_t st);
 
+// 32 < R + W <= 64, R <= 32 (seed_compress_wide.cu).
+bool compress_wide_supported(const seed_dims& d);
+int launch_compress_wide(const seed_dims& d, const seed_state& s, int layer, float* sigma_out,
+                         uint32_t* status, cudaStream_t st);
+
 int launch_compress(const seed_dims& d, const seed_state& s, int layer, float* sigma_out,
                     uint32_t* status, cudaStream_t st);
 
@@ -92,6 +109,10 @@ int launch_to_dense(const seed_dims& d, const seed_state& s, int layer, const in
 
 int launch_state_energy(const seed_dims& d, const seed_state& s, int layer, const int32_t* units,
                         int n_units, float* out, uint32_t* status, cudaStream_t st);
+
+int launch_state_spectrum(const seed_dims& d, const seed_state& s, int layer, const int32_t* units, int n_units,
+                          float* sigma_state, float* sigma_content, float* cos_top, int32_t* ranks,
+                          uint32_t* status, cudaStream_t st);
 
 int launch_dense_step(const seed_dims& d, float* S, int layer, const float* q, const float* k,
                       const float* v, const float* alpha, const float* beta, float* o,

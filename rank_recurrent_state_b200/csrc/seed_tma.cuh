@@ -44,6 +44,12 @@ SEED_DEV void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar
       : "memory");
 }
 
+// Bulk prefetch of [src, src + bytes) from global memory into L2 (no shared memory, no
+// completion to wait for); src 16-byte aligned, bytes a multiple of 16.
+SEED_DEV void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Ampere-style asynchronous 16-byte copy global -> shared (no mbarrier): groups
 // are committed in order and waited for by count; each thread waits for its own.
 SEED_DEV void cp_async16(void* dst, const void* src) {
@@ -61,6 +67,29 @@ SEED_DEV void tma_load_3d(void* dst, const void* tmap, int x, int y, int z, uint
       "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
           smem_addr(dst)),
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// L2 eviction priorities for the cache_hint forms of the copies: evict_last keeps
+// the lines in L2 ahead of normal traffic (data read again soon), evict_first lets
+// them go first (data read for the last time).
+SEED_DEV uint64_t l2_policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+SEED_DEV uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// tma_load_3d with an L2 eviction policy (from l2_policy_*).
+SEED_DEV void tma_load_3d_hint(void* dst, const void* tmap, int x, int y, int z, uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(
+          smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar)), "l"(policy)
       : "memory");
 }
 

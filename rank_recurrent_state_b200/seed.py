@@ -249,6 +249,20 @@ def seed_state_energy(dims: Dims, state: State, layer: int, out: torch.Tensor, w
         _stream(stream)))
 
 
+def seed_state_spectrum(dims: Dims, state: State, layer: int, sigma_state: torch.Tensor,
+                        sigma_content: torch.Tensor, cos_top: torch.Tensor, ranks: torch.Tensor,
+                        ws: Workspace, units: torch.Tensor | None = None, stream=None) -> None:
+    """sigma_state, sigma_content [n][R+W+1], cos_top [n] (float32); ranks [n][2] int32 (see seed.h)."""
+    _check_state(dims, state)
+    if ranks.dtype != torch.int32:
+        raise ValueError("ranks must be int32")
+    d, s = dims.c(), state.c()
+    n = 0 if units is None else int(units.numel())
+    _check("seed_state_spectrum", _lib.load().seed_state_spectrum(
+        ctypes.byref(d), ctypes.byref(s), layer, _ptr(units), n, _ptr(sigma_state), _ptr(sigma_content),
+        _ptr(cos_top), _ptr(ranks), ws.ptr, ws.nbytes, _stream(stream)))
+
+
 def seed_dense_step(dims: Dims, S: torch.Tensor, layer: int, q, k, v, alpha, beta, o,
                     ws: Workspace, stream=None) -> None:
     d = dims.c()

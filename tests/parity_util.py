@@ -150,6 +150,16 @@ _UNIT_AXIS1 = ("o", "a_t", "sigma", "gap", "tail", "err_open", "sink_dev")
 _SHARED = ("ncols", "comp_steps")
 
 
+def _one_blas_thread():
+    """Pool initializer: one BLAS thread per oracle worker (the workers already use
+    every core)."""
+    try:
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(1)
+    except Exception:   # pragma: no cover - speed only
+        pass
+
+
 def _oracle_chunk(args):
     from oracle import run as orun
     cfg, b, l, h, n_prefill, n_decode = args
@@ -163,7 +173,7 @@ def run_oracle_units(cfg, b, l, h, n_prefill, n_decode, workers=8, chunk=8):
     b, l, h = (np.asarray(x, dtype=np.int64) for x in (b, l, h))
     parts = [(cfg, b[i:i + chunk], l[i:i + chunk], h[i:i + chunk], n_prefill, n_decode)
              for i in range(0, b.size, chunk)]
-    with mp.get_context("spawn").Pool(min(workers, len(parts))) as pool:
+    with mp.get_context("spawn").Pool(min(workers, len(parts)), initializer=_one_blas_thread) as pool:
         outs = pool.map(_oracle_chunk, parts)
     merged = {}
     for key in outs[0]:

@@ -1,9 +1,10 @@
 """seed_compress on factor states built on the host, against the oracle's truncation.
 
 The states are inputs (uploaded), so nothing the device computes reaches the
-oracle.  Covers every form, the fast path (R + W <= 32, d in {64, 128}), the
-Householder path (larger windows, 16-wide heads), a key repeated inside one window
-(the fast path declines it), and exactly zero columns.
+oracle.  Covers every form, the Cholesky-QR paths (R + W <= 32 with R <= 16, and
+32 < R + W <= 64 with R <= 32, for d in {64, 128}), the Householder path (larger
+windows, 16-wide heads), a key repeated inside one window (the Cholesky-QR paths
+decline it), and exactly zero columns.
 """
 
 import numpy as np
@@ -80,24 +81,32 @@ def _run(form, dk, dv, R, W, repeat=False, zero_cols=0, n=24, seed=0):
 @pytest.mark.parametrize("form", [FORM_GDN, FORM_KDA, FORM_MAMBA2])
 @pytest.mark.parametrize("dk,dv,R,W", [(128, 128, 16, 16), (128, 64, 8, 8), (64, 64, 4, 12),
                                        (128, 128, 8, 16), (64, 128, 12, 8), (128, 128, 32, 64),
-                                       (16, 16, 4, 4), (128, 64, 8, 32)])
+                                       (16, 16, 4, 4), (128, 64, 8, 32),
+                                       # the wide Cholesky-QR path, 32 < R + W <= 64
+                                       (128, 128, 32, 32), (128, 128, 16, 32), (128, 128, 3, 30),
+                                       (128, 128, 21, 12), (64, 128, 20, 20), (64, 64, 16, 24),
+                                       (128, 64, 32, 17)])
 def test_compress_matches_truncated_svd(form, dk, dv, R, W):
     _run(form, dk, dv, R, W, seed=dk + R + W + form)
 
 
-def test_repeated_key_takes_the_householder_path():
-    diag = _run(FORM_GDN, 128, 128, 16, 16, repeat=True, n=8, seed=7)
+@pytest.mark.parametrize("R,W", [(16, 16), (8, 32), (32, 32)], ids=["fast", "wide-40", "wide-64"])
+def test_repeated_key_takes_the_householder_path(R, W):
+    diag = _run(FORM_GDN, 128, 128, R, W, repeat=True, n=8, seed=7)
     assert diag["cholqr_declined"] == 8 and diag["householder_units"] == 8
 
 
-def test_well_conditioned_units_take_the_cholesky_qr_path():
-    diag = _run(FORM_GDN, 128, 128, 16, 16, n=16, seed=11)
-    assert diag["cholqr_units"] == 16 and diag["householder_units"] == 0
+@pytest.mark.parametrize("form,dk,dv,R,W", [(FORM_GDN, 128, 128, 16, 16), (FORM_MAMBA2, 128, 64, 8, 32),
+                                            (FORM_KDA, 128, 128, 32, 32), (FORM_GDN, 128, 128, 16, 48)])
+def test_well_conditioned_units_take_the_cholesky_qr_path(form, dk, dv, R, W):
+    diag = _run(form, dk, dv, R, W, n=16, seed=11)
+    assert diag["cholqr_units"] == 16 and diag["householder_units"] == 0, diag
 
 
-def test_zero_columns_are_dropped_exactly():
-    _run(FORM_GDN, 128, 128, 16, 16, zero_cols=5, n=8, seed=9)
-    _run(FORM_KDA, 128, 128, 16, 16, zero_cols=16, n=8, seed=10)
+@pytest.mark.parametrize("R,W", [(16, 16), (8, 32), (32, 32)], ids=["fast", "wide-40", "wide-64"])
+def test_zero_columns_are_dropped_exactly(R, W):
+    _run(FORM_GDN, 128, 128, R, W, zero_cols=5, n=8, seed=9)
+    _run(FORM_KDA, 128, 128, R, W, zero_cols=min(16, R), n=8, seed=10)
 
 
 def _graded_state(form, n, dk, dv, R, W, rng, lazy):
@@ -120,7 +129,7 @@ def _graded_state(form, n, dk, dv, R, W, rng, lazy):
 
 
 @pytest.mark.parametrize("lazy", [False, True])
-@pytest.mark.parametrize("dk,dv,R,W", [(128, 128, 16, 16), (128, 64, 8, 32)])
+@pytest.mark.parametrize("dk,dv,R,W", [(128, 128, 16, 16), (128, 64, 8, 32), (128, 128, 32, 32)])
 def test_graded_spectrum_with_long_decayed_columns(lazy, dk, dv, R, W):
     import torch
     from rank_recurrent_state_b200 import seed as S

@@ -49,12 +49,14 @@ def test_compress_flop_model():
     assert rf.fp32_peak_tflops(1965.0) == pytest.approx(148 * 128 * 2 * 1.965e9 / 1e12)
 
 
-def test_traffic_capture_scales_by_the_byte_model():
+def test_traffic_capture_scales_by_the_byte_model(monkeypatch):
     import bench
     from rank_recurrent_state_b200.seed import Dims
     d = Dims(0, 256, 36, 48, 128, 128, 16, 16)
+    cap = {"kernel": bench.decode_kernel_name(d), "form": 0, "d_k": 128, "d_v": 128, "R": 16, "W": 16,
+           "factors": 0, "units": 12288, "c": 19, "bytes": 2.9e8}
+    monkeypatch.setattr(bench, "NCU_DECODE_TRAFFIC", [cap])
     t = bench.decode_traffic(d, 12288, 19)
-    cap = [x for x in bench.NCU_DECODE_TRAFFIC if x["factors"] == 0][0]
     assert t == pytest.approx(cap["bytes"])                       # same units, same column count
     assert bench.decode_traffic(d, 2 * 12288, 19) == pytest.approx(2 * cap["bytes"])
     assert bench.decode_traffic(d, 12288, 23.5) > t                # more columns, more bytes
@@ -76,12 +78,13 @@ def test_kernel_launch_counts():
     import bench
     from rank_recurrent_state_b200.seed import Dims
     gdn = Dims(0, 256, 36, 48, 128, 128, 16, 16)
-    m2 = Dims(2, 256, 40, 64, 128, 64, 8, 32)          # R + W = 40: Householder only
+    m2 = Dims(2, 256, 40, 64, 128, 64, 8, 32)          # R + W = 40: wide Cholesky QR + Householder
+    kda96 = Dims(1, 512, 20, 32, 128, 128, 32, 64)      # R + W = 96: Householder only
     tiny = Dims(0, 1, 1, 2, 16, 16, 4, 4)               # d = 16: Householder only
-    assert bench.compress_kernel_launches(gdn) == 2
-    assert bench.compress_kernel_launches(m2) == 1 and bench.compress_kernel_launches(tiny) == 1
+    assert bench.compress_kernel_launches(gdn) == 2 and bench.compress_kernel_launches(m2) == 2
+    assert bench.compress_kernel_launches(kda96) == 1 and bench.compress_kernel_launches(tiny) == 1
     assert bench.fused_kernel_launches(gdn) == 2
-    assert bench.fused_kernel_launches(m2) == 2 and bench.fused_kernel_launches(tiny) == 2
+    assert bench.fused_kernel_launches(m2) == 3 and bench.fused_kernel_launches(tiny) == 2
 
 
 def test_bench_steady_state_is_independent_of_the_timed_window():
