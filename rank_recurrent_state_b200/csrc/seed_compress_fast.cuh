@@ -105,8 +105,10 @@ SEED_DEV void gram_row(const float* P, float (&acc)[MP]) {
 // at the end).  On return G[i * LG + j] = L[i][j] for j <= i, 0 above, and nrm holds
 // the column norms.  A zero column, or a non-positive pivot, gives a zero column of L;
 // a pivot below kCholPivotMin on a nonzero column also sets bad.
+// Not inlined: each compression factors two Grams with it, and one copy of the code
+// keeps the kernel within the instruction cache.
 template <int MP, int LG>
-SEED_DEV void cholesky_wide(float* G, int m, float* nrm, float* ninv, float* colj, bool& bad) {
+__device__ __noinline__ void cholesky_wide(float* G, int m, float* nrm, float* ninv, float* colj, bool& bad) {
   const int lane = threadIdx.x & 31;
   constexpr int RPL = (MP + 31) / 32;
 #pragma unroll
@@ -211,29 +213,19 @@ SEED_DEV float warp_max(float v) {
   return v;
 }
 
-// One-sided Jacobi on the MP x MP matrix in sM (column-major, stride LM), in
-// registers.  Slot s = lane / LP holds the column pair (x, y); lane part h holds
-// rows h*NR .. h*NR+NR-1 of both.  The matrix must be scaled so that its squared
-// column norms stay far from the float32 range limits (entries of order one).
-// Returns the sweeps run; `conv` is set when the last sweep rotated nothing.  On
-// return sM holds M Z (columns in place).
-template <int MP, int LM>
-SEED_DEV int jacobi_regs(float* sM, bool& conv) {
+// One-sided Jacobi (Hestenes) on MP columns held in registers, as described at
+// jacobi_regs below: lane (slot s, part h) holds rows h*NR .. h*NR+NR-1 of the pair
+// (x, y) whose column indices are (ix, iy), initially (s, s + MP/2).  On return x, y
+// hold the rotated columns now at (ix, iy).
+template <int MP>
+SEED_DEV int jacobi_core(float (&x)[(MP / (64 / MP))], float (&y)[(MP / (64 / MP))], int& ix, int& iy,
+                         bool& conv) {
   constexpr int LP = 64 / MP;   // lanes per pair
   constexpr int NR = MP / LP;   // rows per lane
   constexpr int NS = MP / 2;    // pair slots
   static_assert(NR % 4 == 0, "rows per lane must be whole float4s");
   const int lane = threadIdx.x & 31;
   const int slot = lane / LP, h = lane % LP;
-  int ix = slot, iy = slot + NS;
-  float x[NR], y[NR];
-#pragma unroll
-  for (int f = 0; f < NR / 4; ++f) {
-    const float4 a = ld4(sM + ix * LM + h * NR + 4 * f);
-    const float4 b = ld4(sM + iy * LM + h * NR + 4 * f);
-    x[4 * f] = a.x; x[4 * f + 1] = a.y; x[4 * f + 2] = a.z; x[4 * f + 3] = a.w;
-    y[4 * f] = b.x; y[4 * f + 1] = b.y; y[4 * f + 2] = b.z; y[4 * f + 3] = b.w;
-  }
   const float tol = 8.f * sqrtf((float)MP) * 5.9604645e-8f;
   const float tol2 = tol * tol;
   float tiny = 0.f;
@@ -339,6 +331,32 @@ SEED_DEV int jacobi_regs(float* sM, bool& conv) {
       break;
     }
   }
+  return sweeps;
+}
+
+// One-sided Jacobi on the MP x MP matrix in sM (column-major, stride LM), in
+// registers.  Slot s = lane / LP holds the column pair (x, y); lane part h holds
+// rows h*NR .. h*NR+NR-1 of both.  The matrix must be scaled so that its squared
+// column norms stay far from the float32 range limits (entries of order one).
+// Returns the sweeps run; `conv` is set when the last sweep rotated nothing.  On
+// return sM holds M Z (columns in place).
+template <int MP, int LM>
+SEED_DEV int jacobi_regs(float* sM, bool& conv) {
+  constexpr int LP = 64 / MP;   // lanes per pair
+  constexpr int NR = MP / LP;   // rows per lane
+  constexpr int NS = MP / 2;    // pair slots
+  const int lane = threadIdx.x & 31;
+  const int slot = lane / LP, h = lane % LP;
+  int ix = slot, iy = slot + NS;
+  float x[NR], y[NR];
+#pragma unroll
+  for (int f = 0; f < NR / 4; ++f) {
+    const float4 a = ld4(sM + ix * LM + h * NR + 4 * f);
+    const float4 b = ld4(sM + iy * LM + h * NR + 4 * f);
+    x[4 * f] = a.x; x[4 * f + 1] = a.y; x[4 * f + 2] = a.z; x[4 * f + 3] = a.w;
+    y[4 * f] = b.x; y[4 * f + 1] = b.y; y[4 * f + 2] = b.z; y[4 * f + 3] = b.w;
+  }
+  const int sweeps = jacobi_core<MP>(x, y, ix, iy, conv);
   __syncwarp();
 #pragma unroll
   for (int f = 0; f < NR / 4; ++f) {

@@ -60,8 +60,10 @@ struct WideLayout {
 // triangle whose columns lie below m (the rest is zero: those columns are).  fold
 // (KDA's U): entries weighted by P.  Checks the column scale.  Returns false if a copy
 // did not arrive in time (after waiting for those in flight).
+// Not inlined (both Grams use it): one copy of the code keeps the kernel closer to the
+// instruction cache.
 template <bool KDA, int DK, int DV, int MP, int LG, typename TS>
-SEED_DEV bool gram_wide(int c0, int c1, bool fold, float* sA, const CUtensorMap* tmU, const CUtensorMap* tmV,
+__device__ __noinline__ bool gram_wide(int c0, int c1, bool fold, float* sA, const CUtensorMap* tmU, const CUtensorMap* tmV,
                         const FastParams& p, long long unit, int m, uint64_t* bar, uint32_t (&uses)[2],
                         const float* scl, float* Gs, bool& bad, bool fault) {
   constexpr int NCU = DK / 32, NCH = (DK + DV) / 32, CHUNK = MP * 32;
@@ -500,9 +502,8 @@ SEED_DEV bool compress_wide_unit(const FastParams& p, const CUtensorMap& tmU, co
       for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
-#pragma unroll
-    for (int ks = 0; ks < MP / 8; ++ks) {
-      if (ks >= ks_end) break;
+#pragma unroll 1
+    for (int ks = 0; ks < ks_end; ++ks) {
       const int k = ks * 8 + tq;
       uint32_t bh[4][2], bl[4][2];
 #pragma unroll

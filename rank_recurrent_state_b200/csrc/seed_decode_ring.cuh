@@ -201,7 +201,7 @@ SEED_DEV void decode_ring_run(const DecodeParams& p) {
   Vecs cur, nxt;
   if (u < n_units) ring_load_vecs<FORM, DK, DV, MAXC>(p, u, c_cur, cur);
 
-  for (; u < n_units; u += stride) {
+  while (u < n_units) {
     const long long unit = ring_unit(p, u);
     const int u_next = u + stride;
     // the next unit's vectors and the column count two units ahead, while this one runs
@@ -349,13 +349,15 @@ SEED_DEV void decode_ring_run(const DecodeParams& p) {
         if (__any_sync(0xffffffffu, bad) && lane == 0) raise_flag(p.status, SEED_FLAG_NONFINITE);
       }
     }
-    // the next unit: its chunks follow this unit's in the sequence
+    // the next unit: its chunks follow this unit's in the sequence.  u moves on before
+    // the ring is refilled: fill() names the current unit u and the next u + stride
     base += n_cur;
     n_cur = n_nxt;
     c_cur = c_nxt;
     c_nxt = c_aft;
     n_nxt = u_next + stride < n_units ? ring_chunks(c_aft, m) : 0;
     cur = nxt;
+    u = u_next;
     fill();
   }
 }

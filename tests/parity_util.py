@@ -11,7 +11,7 @@ from __future__ import annotations
 import numpy as np
 
 TOL = 1e-4          # relative Frobenius error, fp32 device vs fp64 oracle
-GAP_TOL = 1e-5      # units with a relative singular gap at R below this are near-ties
+U32 = 2.0 ** -24    # float32 unit roundoff
 
 
 def rel_fro(x, y) -> float:
@@ -202,15 +202,28 @@ SUMMARY: list[dict] = []
 
 def first_near_tie(cfg, ref, tol=TOL):
     """Per sampled unit, the first truncation of the oracle's trajectory that is a
-    near-tie (event 0 the conversion, i >= 1 compression i), -1 if none: the relative
-    gap (sigma_R - sigma_{R+1}) / sigma_1 below GAP_TOL while sigma_R / sigma_1 is above
-    the tolerance (below it, any choice moves the state by less than the tolerance)."""
+    near-tie (event 0 the conversion, i >= 1 compression i), -1 if none.
+
+    A truncation to rank R is ill-conditioned when the singular values sigma_R and
+    sigma_{R+1} nearly coincide: a perturbation of relative size u of the matrix turns
+    the kept subspace by about u sigma_1 / (sigma_R - sigma_{R+1}) and moves the
+    truncated matrix by about that times sigma_R.  Any float32 computation perturbs it
+    by the unit roundoff u = 2^-24 at least, so where the predicted error
+        u (sigma_R / sigma_1) / g,   g = (sigma_R - sigma_{R+1}) / sigma_1,
+    exceeds 0.3 of the tolerance, float32 cannot be expected to reproduce the float64
+    truncation to the tolerance, and several truncations are correct to working
+    precision: a near-tie.  (On the GDN layer workload at full size -- 3,072 units, 17
+    truncations each -- the one unit whose error exceeded the tolerance had a predicted
+    error of 3.4e-4, at most twice below its measured 6.9e-4; every unit predicted below
+    0.3 of the tolerance stayed within 0.6 of it.)"""
     gaps = [ref["conv_gap"]] + [ref["gap"][i] for i in range(ref["gap"].shape[0])]
     sigs = [ref["conv_sigma"]] + [ref["sigma"][i] for i in range(ref["sigma"].shape[0])]
     first = np.full(gaps[0].shape[0], -1)
     for ev_i, (g, sg) in enumerate(zip(gaps, sigs)):
         top = np.where(sg[:, 0] > 0, sg[:, 0], 1.0)
-        hit = (g < GAP_TOL) & (sg[:, -1] > tol * top) & (first < 0)
+        ratio = sg[:, -1] / top
+        predicted = U32 * ratio / np.maximum(g, 1e-300)
+        hit = (predicted > 0.3 * tol) & (first < 0)
         first[hit] = ev_i
     return first
 
@@ -259,12 +272,11 @@ def check_compressions(dev, R, tol=TOL):
     return worst
 
 
-def compare(cfg, dev, ref, tol=TOL, max_tie_frac=0.25, label=None):
+def compare(cfg, dev, ref, tol=TOL, max_tie_frac=0.1, label=None):
     """Device against oracle.
 
-    Units whose relative singular gap (sigma_R - sigma_{R+1}) / sigma_1 falls below
-    GAP_TOL at the conversion or at a compression where sigma_R / sigma_1 exceeds the
-    tolerance are near-ties: several truncations are correct there.  For them, what is
+    Units with an ill-conditioned truncation (first_near_tie) at the conversion or at a
+    compression are near-ties: several truncations are correct there.  For them, what is
     unique is compared: the sink coefficient a (no truncation touches it), and the
     trajectory up to the first ambiguous truncation -- the outputs o of every step up
     to it, and the kept singular values of every compression up to and including it.

@@ -123,6 +123,22 @@ def test_kda_sweep_reduced(R, W):
     _parity(cfg, sample, 150, 2 * W + 2, batch=1, label=f"kda R{R} W{W} reduced")
 
 
+@pytest.mark.parametrize("cid,over,batch", [(3, {}, 64), (4, {"R": 8, "W": 8}, 64), (0, {}, 2048),
+                                             (1, {"R": 4, "W": 4}, 64)],
+                         ids=["mamba2-b64", "kda-R8-W8-b64", "tiny-b2048", "gdn-R4-W4-b64"])
+def test_several_units_per_warp(cid, over, batch):
+    """Batches large enough that every warp of the persistent decode grid steps several
+    units in turn, at column counts of one or two chunks per factor, so that the ring
+    of each warp streams one unit's chunks while it still holds the previous one's
+    (sampled units, two compressions)."""
+    cfg = config(cid, **over)
+    c = cfg.replace(batch=batch)
+    rng = np.random.default_rng(cid * 7 + batch)
+    n = c.units
+    sample = np.unique(np.concatenate([rng.choice(n, 40, replace=False), np.arange(n - 8, n)]))
+    _parity(cfg, sample, 64, 2 * cfg.W + 3, batch=batch, label=f"cfg{cid} batch {batch} (several units per warp)")
+
+
 def test_odd_window_and_empty_prefill():
     """R + W odd (the core SVD pads a zero column) and a zero prefill state (rank 0)."""
     cfg = config(0, R=3, W=4)
