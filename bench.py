@@ -712,11 +712,11 @@ def run_ours(args, world, rank, local):
             one_step(s_next, ev2)
             s_next += 1
             if due:
-                cmp_ms = [a.elapsed_time(b) for a, b in ev2["cmp"]]
-                fus_ms = [a.elapsed_time(b) for a, b in ev2["fus"]]
-                extra_cmp = True
                 break
         torch.cuda.synchronize()
+        cmp_ms = [a.elapsed_time(b) for a, b in ev2["cmp"]]
+        fus_ms = [a.elapsed_time(b) for a, b in ev2["fus"]]
+        extra_cmp = True
         diag2 = S.seed_get_diagnostics(run.ws)
         for key in diag:
             diag[key] += diag2[key]

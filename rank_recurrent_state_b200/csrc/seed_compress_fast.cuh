@@ -492,16 +492,18 @@ SEED_DEV void mma3_tf32(float (&d)[4], const uint32_t (&ah)[4], const uint32_t (
 // (chunk c + 2 is issued into a buffer once chunk c is read) with tensor-core tiles:
 // G = P^T P as (MP x 32-row chunk) x (32-row chunk x MP) products, the upper block
 // triangle only (m16n8 tiles with n-tile >= 2 m-tile), mirrored when written to Gs
-// (row-major, stride LG); then lane i loads row i of G into g.  The A operand of
+// (row-major, stride LG).  The A operand of
 // an m-tile is made of the B operands of n-tiles 2 mt and 2 mt + 1 (the same panel
 // columns).  fold (KDA's U): entries weighted by P (true U = Diag(P) U).  Also
 // checks the column scale.  Returns false if a copy did not arrive in time (after
 // waiting for those in flight).
+// Not inlined: both Grams use it, and one copy of the code keeps the kernel closer to
+// the instruction cache.
 template <bool KDA, int DK, int DV, int MP, int LG, typename TS>
-SEED_DEV bool gram_stream(int c0, int c1, bool fold, float* sA, const CUtensorMap* tmU,
-                          const CUtensorMap* tmV, const FastParams& p, long long unit, int m, uint64_t* bar,
-                          uint32_t (&uses)[2], const float* scl, float* Gs, float (&g)[MP], bool& bad,
-                          bool fault = false) {
+__device__ __noinline__ bool gram_stream(int c0, int c1, bool fold, float* sA, const CUtensorMap* tmU,
+                                         const CUtensorMap* tmV, const FastParams& p, long long unit, int m,
+                                         uint64_t* bar, uint32_t (&uses)[2], const float* scl, float* Gs,
+                                         bool& bad, bool fault) {
   constexpr int NCU = DK / 32, NCH = (DK + DV) / 32, CHUNK = MP * 32;
   constexpr int NT = MP / 8, MT = MP / 16;
   const int lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
@@ -573,13 +575,6 @@ SEED_DEV bool gram_stream(int c0, int c1, bool fold, float* sA, const CUtensorMa
     }
   }
   __syncwarp();
-  const int i = lane < MP ? lane : 0;
-#pragma unroll
-  for (int k = 0; k < MP; k += 4) {
-    const float4 v = ld4(Gs + i * LG + k);
-    g[k] = v.x; g[k + 1] = v.y; g[k + 2] = v.z; g[k + 3] = v.w;
-  }
-  __syncwarp();   // every lane has its row before Gs is overwritten
   return true;
 }
 
@@ -662,11 +657,10 @@ SEED_DEV bool compress_fast_unit(const FastParams& p, const CUtensorMap& tmU, co
   const bool fault = std::is_same<TS, float>::value && wait_fault_injected(p.status);
   start_stream<DK, DV, MP, TS>(sA, &tmU, &tmV, p, unit, m, bar, fault);
   bool bad = false;   // ill-conditioned or badly scaled: left for the Householder kernel
-  float g[MP];
   // U: chunks 0 .. NCU-1, then its Cholesky factor (to its own region); a copy that
   // does not arrive here leaves the unit untouched at R + W columns, for the
   // Householder kernel
-  if (!gram_stream<KDA, DK, DV, MP, LG, TS>(0, NCU, true, sA, &tmU, &tmV, p, unit, m, bar, uses, scl, sLu, g,
+  if (!gram_stream<KDA, DK, DV, MP, LG, TS>(0, NCU, true, sA, &tmU, &tmV, p, unit, m, bar, uses, scl, sLu,
                                             bad, fault)) {
     if (lane == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
     return false;
@@ -676,7 +670,7 @@ SEED_DEV bool compress_fast_unit(const FastParams& p, const CUtensorMap& tmU, co
   cholesky_wide<MP, LG>(sLu, m, nu, nrm, du, bad);
   // V: chunks NCU .. NCH-1; L_v over the chunk buffers once the last one is read
   if (!gram_stream<KDA, DK, DV, MP, LG, TS>(NCU, NCH, false, sA, &tmU, &tmV, p, unit, m, bar, uses, scl, sM,
-                                            g, bad)) {
+                                            bad, false)) {
     if (lane == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
     return false;
   }
