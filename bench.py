@@ -40,7 +40,12 @@ NOMINAL_HBM_GBS = 8000.0
 # per-layer launch of the GDN stack shape (256 requests x 48 heads) at c stored columns,
 # per factor format.  Remove an entry whenever that kernel changes, until it is measured
 # again (no entry: the line's roofline.traffic is null).
-NCU_DECODE_TRAFFIC = []
+NCU_DECODE_TRAFFIC = [
+    # decode_ring_kernel, float32 factors, layer 0 of step 3 after the conversion (c = 19):
+    # dram__bytes_read.sum 266.12 MB + dram__bytes_write.sum 17.83 MB
+    {"kernel": "decode_ring_kernel", "form": 0, "d_k": 128, "d_v": 128, "R": 16, "W": 16, "factors": 0,
+     "units": 12288, "c": 19, "bytes": 283.95e6},
+]
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -69,6 +74,10 @@ def parse_args(argv=None):
     ap.add_argument("--dense-steps", type=int, default=8)
     ap.add_argument("--e2e-steps", type=int, default=None,
                     help="end-to-end steps (default: one compression window, W)")
+    ap.add_argument("--e2e-copy", default="step", choices=["step", "layer"],
+                    help="end-to-end copy granularity: one copy per input tensor per step (all "
+                         "layers, into a ring of device slots) and o out once per step, or five "
+                         "copies in and one out per layer")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--reference-units", type=int, default=384,
                     help="units of the workload the reference arm (the fp64 oracle) steps")
@@ -333,7 +342,9 @@ def run_reference(args, world, rank):
 # ------------------------------------------------------------------ GPU arm
 
 def decode_kernel_name(d):
-    return "decode_ring_kernel" if d.R + d.W - 1 <= 64 else "decode_step_kernel"
+    if d.R + d.W - 1 > 64:
+        return "decode_step_kernel"
+    return "decode_ring_kernel" if d.factors == 0 else "decode_warp_kernel"
 
 
 def decode_traffic(d, units, cbar):
@@ -452,8 +463,18 @@ def run_e2e(args, run, d, L, BH, q, k, v, alpha, beta, o, kda, stream, dev, worl
     old_aff = os.sched_getaffinity(0)
     if aff:
         os.sched_setaffinity(0, aff)
+    # the host pool cycles as many distinct steps as the device pool (3 W by default),
+    # so that the W columns a window appends are distinct keys as in the timed loop; a
+    # pool of a few steps repeats keys inside a window, and the compression then meets
+    # rank-deficient factors (the Householder fallback) that the workload never has
+    step_bytes = (q[0].numel() + k[0].numel() + v[0].numel() + alpha[0].numel() + beta[0].numel()) * 4
     try:
-        Ph = 2
+        import psutil
+        avail = psutil.virtual_memory().available
+    except ImportError:
+        avail = 64 << 30
+    Ph = max(2, min(q.shape[0], int(0.25 * avail) // step_bytes))
+    try:
         hq = torch.empty(Ph, L, BH, d.d_k, dtype=torch.float32, pin_memory=True)
         hk = torch.empty_like(hq, pin_memory=True)
         hv = torch.empty(Ph, L, BH, d.d_v, dtype=torch.float32, pin_memory=True)
@@ -465,18 +486,24 @@ def run_e2e(args, run, d, L, BH, q, k, v, alpha, beta, o, kda, stream, dev, worl
             os.sched_setaffinity(0, old_aff)
     for t in range(Ph):
         hq[t].copy_(q[t]); hk[t].copy_(k[t]); hv[t].copy_(v[t]); ha[t].copy_(alpha[t]); hb[t].copy_(beta[t])
-    # inputs copied in on their own stream into two alternating device buffers, each
-    # layer's o copied out on a third stream as soon as it is written, so that the
-    # transfers (host memory and PCIe bound) overlap the decode launches
-    nb = 2
-    bufs = [(torch.empty_like(q[0, 0]), torch.empty_like(k[0, 0]), torch.empty_like(v[0, 0]),
-             torch.empty_like(alpha[0, 0]), torch.empty_like(beta[0, 0])) for _ in range(nb)]
+    # inputs copied in on their own stream into a ring of device slots, outputs copied
+    # out on a third, so that the transfers (host memory and PCIe bound) overlap the
+    # decode launches.  "step": one slot holds a whole step (all layers); "layer": one
+    # layer's inputs, with each layer's o copied out as soon as it is written
+    per_step = args.e2e_copy == "step"
+    nb = 3 if per_step else 2
+    if per_step:
+        bufs = [(torch.empty_like(q[0]), torch.empty_like(k[0]), torch.empty_like(v[0]),
+                 torch.empty_like(alpha[0]), torch.empty_like(beta[0]), torch.empty_like(o)) for _ in range(nb)]
+    else:
+        bufs = [(torch.empty_like(q[0, 0]), torch.empty_like(k[0, 0]), torch.empty_like(v[0, 0]),
+                 torch.empty_like(alpha[0, 0]), torch.empty_like(beta[0, 0])) for _ in range(nb)]
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     ev_in = [torch.cuda.Event() for _ in range(nb)]
     ev_free = [torch.cuda.Event() for _ in range(nb)]
     ev_dec = [torch.cuda.Event() for _ in range(L)]
-    ev_out = [torch.cuda.Event() for _ in range(L)]
-    h2d = L * sum(x.numel() for x in bufs[0]) * 4   # as copied
+    ev_out = [torch.cuda.Event() for _ in range(max(L, nb))]
+    h2d = (1 if per_step else L) * sum(x.numel() for x in bufs[0][:5]) * 4   # as copied
     d2h = o.numel() * 4
 
     # the host link alone: one step's inputs in (all layers, one copy per tensor), the
@@ -521,69 +548,112 @@ def run_e2e(args, run, d, L, BH, q, k, v, alpha, beta, o, kda, stream, dev, worl
                                   v[1, l], al, beta[1, l, :BH])
     bound_ms = max(t_both, step_ms)   # copies overlapped with the device work at best
 
-    # align to the start of a window (the step after a compression), untimed
+    # align to the start of a window (the step after a compression), untimed, cycling
+    # the device pool's steps
+    P = q.shape[0]
     while run.c != d.R and not args.ragged:
+        t = s_next % P
         for l in range(L):
-            S.seed_decode_step(d, run.state, l, q[0, l], k[0, l], v[0, l],
-                               alpha[0, l] if kda else alpha[0, l, :BH], beta[0, l, :BH], o[l], run.ws, stream)
+            S.seed_decode_step(d, run.state, l, q[t, l], k[t, l], v[t, l],
+                               alpha[t, l] if kda else alpha[t, l, :BH], beta[t, l, :BH], o[l], run.ws, stream)
+        s_next += 1
         run.c += 1
         if run.c == d.m:
             S.seed_compress(d, run.state, S.SEED_ALL_LAYERS, run.ws, stream=stream)
             run.c = d.R
     n_steps = args.e2e_steps if args.e2e_steps else d.W
     torch.cuda.synchronize()
+    diag0 = S.seed_get_diagnostics(run.ws)
+    cmp_ev = []
     barrier(world, dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     s_in.wait_stream(stream)
     s_out.wait_stream(stream)
     n = 0
+    t_host = time.perf_counter()
     for s in range(n_steps):
-        t = s % Ph
+        t = (s_next + s) % Ph   # the pool's steps in the order the timed loop left them
         fuse = args.fused and (args.ragged or run.c + 1 == d.m)
-        for l in range(L):
-            bi = n % nb
-            bq, bk, bv, ba, bb = bufs[bi]
+        step_fn = S.seed_decode_step_compress if fuse else S.seed_decode_step
+        if per_step:
+            j = s % nb
+            bq, bk, bv, ba, bb, bo = bufs[j]
             with torch.cuda.stream(s_in):
-                if n >= nb:
-                    s_in.wait_event(ev_free[bi])
-                bq.copy_(hq[t, l], non_blocking=True); bk.copy_(hk[t, l], non_blocking=True)
-                bv.copy_(hv[t, l], non_blocking=True); ba.copy_(ha[t, l], non_blocking=True)
-                bb.copy_(hb[t, l], non_blocking=True)
-                ev_in[bi].record(s_in)
-            stream.wait_event(ev_in[bi])
-            if s > 0:
-                stream.wait_event(ev_out[l])   # last step's o of this layer is out
-            step_fn = S.seed_decode_step_compress if fuse else S.seed_decode_step
-            step_fn(d, run.state, l, bq, bk, bv, ba if kda else ba[:BH], bb[:BH], o[l], run.ws, stream=stream)
-            ev_free[bi].record(stream)
-            ev_dec[l].record(stream)
+                if s >= nb:
+                    s_in.wait_event(ev_free[j])   # step s - nb's launches have read the slot
+                bq.copy_(hq[t], non_blocking=True); bk.copy_(hk[t], non_blocking=True)
+                bv.copy_(hv[t], non_blocking=True); ba.copy_(ha[t], non_blocking=True)
+                bb.copy_(hb[t], non_blocking=True)
+                ev_in[j].record(s_in)
+            stream.wait_event(ev_in[j])
+            if s >= nb:
+                stream.wait_event(ev_out[j])   # step s - nb's o has left the slot
+            for l in range(L):
+                step_fn(d, run.state, l, bq[l], bk[l], bv[l], ba[l] if kda else ba[l, :BH], bb[l, :BH], bo[l],
+                        run.ws, stream=stream)
+            ev_free[j].record(stream)
             with torch.cuda.stream(s_out):
-                s_out.wait_event(ev_dec[l])
-                ho[l].copy_(o[l], non_blocking=True)
-                ev_out[l].record(s_out)
-            n += 1
+                s_out.wait_event(ev_free[j])
+                ho.copy_(bo, non_blocking=True)
+                ev_out[j].record(s_out)
+            n += L
+        else:
+            for l in range(L):
+                bi = n % nb
+                bq, bk, bv, ba, bb = bufs[bi]
+                with torch.cuda.stream(s_in):
+                    if n >= nb:
+                        s_in.wait_event(ev_free[bi])
+                    bq.copy_(hq[t, l], non_blocking=True); bk.copy_(hk[t, l], non_blocking=True)
+                    bv.copy_(hv[t, l], non_blocking=True); ba.copy_(ha[t, l], non_blocking=True)
+                    bb.copy_(hb[t, l], non_blocking=True)
+                    ev_in[bi].record(s_in)
+                stream.wait_event(ev_in[bi])
+                if s > 0:
+                    stream.wait_event(ev_out[l])   # last step's o of this layer is out
+                step_fn(d, run.state, l, bq, bk, bv, ba if kda else ba[:BH], bb[:BH], o[l], run.ws, stream=stream)
+                ev_free[bi].record(stream)
+                ev_dec[l].record(stream)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(ev_dec[l])
+                    ho[l].copy_(o[l], non_blocking=True)
+                    ev_out[l].record(s_out)
+                n += 1
         run.c += 1
         if run.c == d.m or args.ragged:   # ragged: some request is due after every step
             if not fuse:
+                cmp_ev.append((torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)))
+                cmp_ev[-1][0].record(stream)
                 S.seed_compress(d, run.state, S.SEED_ALL_LAYERS, run.ws, stream=stream)
+                cmp_ev[-1][1].record(stream)
             run.c = d.R
+    host_ms = (time.perf_counter() - t_host) * 1e3
     stream.wait_stream(s_out)
     stream.wait_stream(s_in)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(world, dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    per_step = e2e_ms / n_steps
+    step_e2e = e2e_ms / n_steps
+    diag1 = S.seed_get_diagnostics(run.ws)
+    e2e_cmp = {"launches": len(cmp_ev),
+               "ms_per_launch": (sum(a.elapsed_time(b) for a, b in cmp_ev) / len(cmp_ev)) if cmp_ev else None,
+               "cholqr_units": diag1["cholqr_units"] - diag0["cholqr_units"],
+               "householder_units": diag1["householder_units"] - diag0["householder_units"]}
     return {"value": n_steps * units * world / (e2e_ms / 1e3), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_steps,
-            "ms_per_step": per_step,
-            "h2d_GBps_achieved": h2d / (per_step / 1e3) / 1e9, "d2h_GBps_achieved": d2h / (per_step / 1e3) / 1e9,
+            "ms_per_step": step_e2e,
+            "h2d_GBps_achieved": h2d / (step_e2e / 1e3) / 1e9, "d2h_GBps_achieved": d2h / (step_e2e / 1e3) / 1e9,
+            "copies": args.e2e_copy, "host_enqueue_ms_per_step": host_ms / n_steps,
+            "host_pool_steps": Ph, "compress": e2e_cmp,
             "host_link": link,
             "host_link_bound_value": units * world / (bound_ms / 1e3),
-            "frac_of_host_link_bound": (units * world / (per_step / 1e3)) / (units * world / (bound_ms / 1e3)),
+            "frac_of_host_link_bound": bound_ms / step_e2e,
             "note": "pinned host buffers; every step copies its inputs in and its o out (copies on their own "
-                    "streams, overlapping the decode launches); timed over whole compression windows "
+                    "streams, overlapping the decode launches; 'copies' = step: one copy per tensor for all "
+                    "layers into a ring of three device slots, layer: per layer into two); timed over whole "
+                    "compression windows "
                     "starting right after a compression; host_link_bound_value = units / max(device "
                     "step, one step's input and output copies run alone and together)"}
 

@@ -216,14 +216,14 @@ SEED_DEV float warp_max(float v) {
 // One-sided Jacobi (Hestenes) on MP columns held in registers, as described at
 // jacobi_regs below: lane (slot s, part h) holds rows h*NR .. h*NR+NR-1 of the pair
 // (x, y) whose column indices are (ix, iy), initially (s, s + MP/2).  On return x, y
-// hold the rotated columns now at (ix, iy).
-template <int MP>
-SEED_DEV int jacobi_core(float (&x)[(MP / (64 / MP))], float (&y)[(MP / (64 / MP))], int& ix, int& iy,
-                         bool& conv) {
+// hold the rotated columns now at (ix, iy).  NR * (64 / MP) may be below MP when the
+// rows beyond it are zero in every column: rotations keep them zero, so they are
+// not held.
+template <int MP, int NR = MP / (64 / MP)>
+SEED_DEV int jacobi_core(float (&x)[NR], float (&y)[NR], int& ix, int& iy, bool& conv) {
   constexpr int LP = 64 / MP;   // lanes per pair
-  constexpr int NR = MP / LP;   // rows per lane
   constexpr int NS = MP / 2;    // pair slots
-  static_assert(NR % 4 == 0, "rows per lane must be whole float4s");
+  static_assert(NR % 4 == 0 && NR * LP <= MP, "rows per lane: whole float4s, at most MP in all");
   const int lane = threadIdx.x & 31;
   const int slot = lane / LP, h = lane % LP;
   const float tol = 8.f * sqrtf((float)MP) * 5.9604645e-8f;
@@ -336,14 +336,14 @@ SEED_DEV int jacobi_core(float (&x)[(MP / (64 / MP))], float (&y)[(MP / (64 / MP
 
 // One-sided Jacobi on the MP x MP matrix in sM (column-major, stride LM), in
 // registers.  Slot s = lane / LP holds the column pair (x, y); lane part h holds
-// rows h*NR .. h*NR+NR-1 of both.  The matrix must be scaled so that its squared
+// rows h*NR .. h*NR+NR-1 of both (NR below MP / LP: the rows from NR * LP on are
+// zero and left as they are).  The matrix must be scaled so that its squared
 // column norms stay far from the float32 range limits (entries of order one).
 // Returns the sweeps run; `conv` is set when the last sweep rotated nothing.  On
 // return sM holds M Z (columns in place).
-template <int MP, int LM>
+template <int MP, int LM, int NR = MP / (64 / MP)>
 SEED_DEV int jacobi_regs(float* sM, bool& conv) {
   constexpr int LP = 64 / MP;   // lanes per pair
-  constexpr int NR = MP / LP;   // rows per lane
   constexpr int NS = MP / 2;    // pair slots
   const int lane = threadIdx.x & 31;
   const int slot = lane / LP, h = lane % LP;
@@ -356,7 +356,7 @@ SEED_DEV int jacobi_regs(float* sM, bool& conv) {
     x[4 * f] = a.x; x[4 * f + 1] = a.y; x[4 * f + 2] = a.z; x[4 * f + 3] = a.w;
     y[4 * f] = b.x; y[4 * f + 1] = b.y; y[4 * f + 2] = b.z; y[4 * f + 3] = b.w;
   }
-  const int sweeps = jacobi_core<MP>(x, y, ix, iy, conv);
+  const int sweeps = jacobi_core<MP, NR>(x, y, ix, iy, conv);
   __syncwarp();
 #pragma unroll
   for (int f = 0; f < NR / 4; ++f) {

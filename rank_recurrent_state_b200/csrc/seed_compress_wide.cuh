@@ -15,7 +15,8 @@
 //      broadcast column j);
 //   3. M = L_u^T diag(w) L_v is formed in place of L_v, lane j holding columns j and
 //      j + 32;
-//   4. one-sided Jacobi on M in registers, one column pair per lane (jacobi_regs);
+//   4. one-sided Jacobi on M in registers, one column pair per lane (jacobi_regs),
+//      each lane holding the first R + W rows rounded up to 8 (the rest are zero);
 //   5. the R leading left vectors X_R (re-orthonormalised when some of them belong to
 //      numerically negligible columns), T_v = D_u L_u X_R Sigma^{-1} and, by back
 //      substitution in place of L_u, T_u = diag(1/nu) L_u^{-T} X_R;
@@ -255,9 +256,15 @@ SEED_DEV bool compress_wide_unit(const FastParams& p, const CUtensorMap& tmU, co
     __syncwarp();
   }
 
-  // 4. one-sided Jacobi on M
+  // 4. one-sided Jacobi on M; its rows from m on are zero, so the lanes hold only the
+  //    first m rounded up to 8 (one copy of the sweep code per row count; m is the
+  //    same for every unit of a launch)
   bool converged;
-  const int sweeps = jacobi_regs<MP, LG>(sM, converged);
+  int sweeps;
+  if (m <= 40) sweeps = jacobi_regs<MP, LG, 40>(sM, converged);
+  else if (m <= 48) sweeps = jacobi_regs<MP, LG, 48>(sM, converged);
+  else if (m <= 56) sweeps = jacobi_regs<MP, LG, 56>(sM, converged);
+  else sweeps = jacobi_regs<MP, LG, 64>(sM, converged);
   if (lane == 0) {
     atomicAdd(p.status + 1, (uint32_t)sweeps);
     atomicAdd(p.status + 5, 1u);

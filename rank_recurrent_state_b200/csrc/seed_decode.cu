@@ -357,8 +357,10 @@ static int launch_one(const DecodeParams& p, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? SEED_OK : SEED_ERR_CUDA;
 }
 
-// Up to 64 stored columns: one warp per unit (seed_decode_warp.cu); above (up to
-// SEED_MAX_COLS - 1), this kernel with four consumer warps per unit.
+// Up to 64 stored columns: one warp per unit (float32 factors through a ring of
+// column chunks, seed_decode_ring.cu; 16-bit factors with a whole-unit stage,
+// seed_decode_warp.cu); above (up to SEED_MAX_COLS - 1), this kernel with four
+// consumer warps per unit.
 template <int FORM, int DK, int DV, typename TS>
 static int launch_cols_t(const DecodeParams& p, cudaStream_t st) {
   return launch_one<FORM, DK, DV, 96, TS>(p, st);
@@ -366,7 +368,9 @@ static int launch_cols_t(const DecodeParams& p, cudaStream_t st) {
 
 template <int FORM, int DK, int DV>
 static int launch_cols(const DecodeParams& p, int factors, cudaStream_t st) {
-  if (p.R + p.W - 1 <= 64) return launch_decode_ring(p, FORM, DK, DV, factors, st);
+  if (p.R + p.W - 1 <= 64)
+    return factors == SEED_FACTORS_F32 ? launch_decode_ring(p, FORM, DK, DV, factors, st)
+                                       : launch_decode_warp16(p, FORM, DK, DV, factors, st);
   switch (factors) {
     case SEED_FACTORS_F32: return launch_cols_t<FORM, DK, DV, float>(p, st);
     case SEED_FACTORS_F16: return launch_cols_t<FORM, DK, DV, __half>(p, st);

@@ -77,5 +77,7 @@ SEED_DEV constexpr int log2c() { return NV <= 1 ? 0 : 1 + log2c<NV / 2>(); }
 // The one-warp-per-unit decode kernel with a ring of column chunks
 // (seed_decode_ring.cu), for R + W - 1 <= 64: the decode step's kernel there.
 int launch_decode_ring(const DecodeParams& p, int form, int dk, int dv, int factors, cudaStream_t st);
+// The whole-unit one-warp kernel for 16-bit factors (seed_decode_warp.cu).
+int launch_decode_warp16(const DecodeParams& p, int form, int dk, int dv, int factors, cudaStream_t st);
 
 }  // namespace seed

@@ -23,7 +23,9 @@
 //   4. the sink update, the new column pair and the read-out, written from registers.
 // The per-unit vectors (k, q, a, v, vbar, the decay scales, g, beta) go from HBM to
 // each lane's registers with coalesced loads one unit ahead.  16-bit factors travel
-// and sit in the slots as stored and are widened as they are read.
+// and sit in the slots as stored and are widened as they are read (the library
+// launches this kernel for float32 factors; 16-bit factors decode with the whole-unit
+// stage of seed_decode_warp.cu, which costs fewer instructions per byte).
 #pragma once
 
 #include "seed_common.cuh"
