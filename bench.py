@@ -36,7 +36,7 @@ METRIC = "decode head-steps/s and achieved HBM GB/s (% of B200 peak) at R=16,W=1
 UNIT = "head-steps/s"
 NOMINAL_HBM_GBS = 8000.0
 # DRAM bytes (read + write) of one decode launch, measured by ncu (dram__bytes_read.sum +
-# dram__bytes_write.sum; profiles/decode_ring_kernel_*gdn_stack_2layers.md) for a full
+# dram__bytes_write.sum, one captured launch on one B200) for a full
 # per-layer launch of the GDN stack shape (256 requests x 48 heads) at c stored columns,
 # per factor format.  Remove an entry whenever that kernel changes, until it is measured
 # again (no entry: the line's roofline.traffic is null).
@@ -45,6 +45,9 @@ NCU_DECODE_TRAFFIC = [
     # dram__bytes_read.sum 266.12 MB + dram__bytes_write.sum 17.83 MB
     {"kernel": "decode_ring_kernel", "form": 0, "d_k": 128, "d_v": 128, "R": 16, "W": 16, "factors": 0,
      "units": 12288, "c": 19, "bytes": 283.95e6},
+    # decode_warp_kernel, float16 factors, the same launch: 146.49 MB + 10.27 MB
+    {"kernel": "decode_warp_kernel", "form": 0, "d_k": 128, "d_v": 128, "R": 16, "W": 16, "factors": 1,
+     "units": 12288, "c": 19, "bytes": 156.76e6},
 ]
 FALLBACK_HBM_GBS = 6650.0
 
@@ -68,6 +71,10 @@ def parse_args(argv=None):
     ap.add_argument("--fused", action="store_true",
                     help="compress inside the decode launch of the step that fills R + W "
                          "(seed_decode_step_compress) instead of a separate compression launch")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="launch every layer's decode step plainly (seed_decode_step) instead of "
+                         "letting it begin during the previous layer's (seed_decode_step_overlapped); "
+                         "also times every launch with its own CUDA events")
     ap.add_argument("--ragged", action="store_true",
                     help="ragged compression schedules: requests joined at different times, a "
                          "compression launch after every step compresses the units that are due")
@@ -245,7 +252,7 @@ def cpu_oracle_rate(cfg, seconds: float, rank_seed: int = 0) -> dict:
             "affinity_cores": len(os.sched_getaffinity(0))}
 
 
-def config_obj(cfg, batch, world, prefill, ragged=False, factors="f32", fused=False):
+def config_obj(cfg, batch, world, prefill, ragged=False, factors="f32", fused=False, overlap=False):
     schedule = ("ragged: request b joined W-1-floor(bW/B) steps before the others; a compression "
                 "launch after every step compresses the units that are due" if ragged else
                 "lockstep: every unit compresses after steps W, 2W, ...")
@@ -260,7 +267,10 @@ def config_obj(cfg, batch, world, prefill, ragged=False, factors="f32", fused=Fa
                             else "a separate launch over all units after the step that fills R + W"),
             "factors": factors + (" (U and V stored in 16 bits, rounded to nearest when written)"
                                   if factors != "f32" else ""),
-            "l2": "inputs and state larger than L2 (no flush needed)"}
+            "l2": "inputs and state larger than L2 (no flush needed)",
+            "layer_launches": ("layers after the first begin during the previous layer's launch "
+                               "(seed_decode_step_overlapped, programmatic dependent launch)" if overlap
+                               else "one after another (seed_decode_step)")}
 
 
 def run_reference(args, world, rank):
@@ -451,9 +461,9 @@ def gpu_numa_affinity(local: int):
 
 def run_e2e(args, run, d, L, BH, q, k, v, alpha, beta, o, kda, stream, dev, world, local, units, step_ms, s_next):
     """The same metric through the public API with host buffers: every step copies its
-    inputs from pinned host memory to the device and each layer's o back, inside the
-    timed region.  Timed over whole compression windows that start right after a
-    compression (steady state); also measures the host link alone in the same run."""
+    inputs from pinned host memory to the device and its o back, inside the timed
+    region.  Timed over W steps (one compression) from the middle of a compression
+    window; also measures the host link alone in the same run."""
     import torch
 
     from rank_recurrent_state_b200 import seed as S
@@ -492,6 +502,7 @@ def run_e2e(args, run, d, L, BH, q, k, v, alpha, beta, o, kda, stream, dev, worl
     # layer's inputs, with each layer's o copied out as soon as it is written
     per_step = args.e2e_copy == "step"
     nb = 3 if per_step else 2
+    overlap = per_step and not (args.no_overlap or args.fused or args.ragged)   # as in the timed loop
     if per_step:
         bufs = [(torch.empty_like(q[0]), torch.empty_like(k[0]), torch.empty_like(v[0]),
                  torch.empty_like(alpha[0]), torch.empty_like(beta[0]), torch.empty_like(o)) for _ in range(nb)]
@@ -548,10 +559,13 @@ def run_e2e(args, run, d, L, BH, q, k, v, alpha, beta, o, kda, stream, dev, worl
                                   v[1, l], al, beta[1, l, :BH])
     bound_ms = max(t_both, step_ms)   # copies overlapped with the device work at best
 
-    # align to the start of a window (the step after a compression), untimed, cycling
-    # the device pool's steps
+    # align, untimed, to the middle of a compression window (c = R + W/2), cycling the
+    # device pool's steps: the W timed steps then hold one compression, in their middle,
+    # where the next steps' input copies overlap it as they do in a long run (a window
+    # that ends with its compression leaves nothing to overlap it)
     P = q.shape[0]
-    while run.c != d.R and not args.ragged:
+    c_start = d.R + d.W // 2
+    while run.c != c_start and not args.ragged:
         t = s_next % P
         for l in range(L):
             S.seed_decode_step(d, run.state, l, q[t, l], k[t, l], v[t, l],
@@ -590,8 +604,9 @@ def run_e2e(args, run, d, L, BH, q, k, v, alpha, beta, o, kda, stream, dev, worl
             if s >= nb:
                 stream.wait_event(ev_out[j])   # step s - nb's o has left the slot
             for l in range(L):
-                step_fn(d, run.state, l, bq[l], bk[l], bv[l], ba[l] if kda else ba[l, :BH], bb[l, :BH], bo[l],
-                        run.ws, stream=stream)
+                fn = S.seed_decode_step_overlapped if (overlap and not fuse and l > 0) else step_fn
+                fn(d, run.state, l, bq[l], bk[l], bv[l], ba[l] if kda else ba[l, :BH], bb[l, :BH], bo[l],
+                   run.ws, stream=stream)
             ev_free[j].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_free[j])
@@ -652,9 +667,9 @@ def run_e2e(args, run, d, L, BH, q, k, v, alpha, beta, o, kda, stream, dev, worl
             "frac_of_host_link_bound": bound_ms / step_e2e,
             "note": "pinned host buffers; every step copies its inputs in and its o out (copies on their own "
                     "streams, overlapping the decode launches; 'copies' = step: one copy per tensor for all "
-                    "layers into a ring of three device slots, layer: per layer into two); timed over whole "
-                    "compression windows "
-                    "starting right after a compression; host_link_bound_value = units / max(device "
+                    "layers into a ring of three device slots, layer: per layer into two); timed over W steps "
+                    "(default) from the middle of a compression window, so that they hold one compression "
+                    "with copies around it; host_link_bound_value = units / max(device "
                     "step, one step's input and output copies run alone and together)"}
 
 
@@ -713,6 +728,10 @@ def run_ours(args, world, rank, local):
     def inputs(t, l):
         return (q[t, l], k[t, l], v[t, l], alpha[t, l] if kda else alpha[t, l, :BH], beta[t, l, :BH])
 
+    # layers after the first step through seed_decode_step_overlapped: the launch before
+    # each is the previous layer's step, which writes none of its state
+    overlap = not (args.no_overlap or args.fused or args.ragged)
+
     def one_step(s, ev=None):
         t = s % P
         fuse = args.fused and (args.ragged or run.c + 1 == d.m)
@@ -726,12 +745,16 @@ def run_ours(args, world, rank, local):
                 if ev is not None:
                     ev["fus"][-1][1].record(stream)
                 continue
-            if ev is not None:
+            # overlapped launches: an event between two launches would serialise them,
+            # so one event pair spans the step's L launches (n = L in the record)
+            timed_here = ev is not None and (not overlap or l == 0)
+            if timed_here:
                 ev["dec"].append((torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-                                  roofline.mean_columns(d.R, d.W) if args.ragged else run.c))
+                                  roofline.mean_columns(d.R, d.W) if args.ragged else run.c, L if overlap else 1))
                 ev["dec"][-1][0].record(stream)
-            S.seed_decode_step(d, run.state, l, qq, kk, vv, aa, bb, o[l], run.ws, stream)
-            if ev is not None:
+            step_fn = S.seed_decode_step_overlapped if (overlap and l > 0) else S.seed_decode_step
+            step_fn(d, run.state, l, qq, kk, vv, aa, bb, o[l], run.ws, stream)
+            if ev is not None and (not overlap or l == L - 1):
                 ev["dec"][-1][1].record(stream)
         run.c += 1
         if fuse:
@@ -769,7 +792,9 @@ def run_ours(args, world, rank, local):
     s_next = args.warmup + args.steps
 
     units = d.units
-    dec_pairs = [(a.elapsed_time(b), c) for a, b, c in ev["dec"]]
+    dec_pairs = []   # per launch: (ms, column count); a step-wide pair gives each launch its share
+    for a, b, c, n in ev["dec"]:
+        dec_pairs += [(a.elapsed_time(b) / n, c)] * n
     cmp_ms = [a.elapsed_time(b) for a, b in ev["cmp"]]
     fus_ms = [a.elapsed_time(b) for a, b in ev["fus"]]
     extra_cmp = False
@@ -829,7 +854,7 @@ def run_ours(args, world, rank, local):
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded Philox4x32-10 inputs and prefill, generated on the device)",
-        "config": config_obj(cfg, B, world, prefill, args.ragged, args.factors, args.fused),
+        "config": config_obj(cfg, B, world, prefill, args.ragged, args.factors, args.fused, overlap),
         "steady_state": (None if steady is None else dict(
             steady, how="value = units / t_step with t_step = (sum over the window's column counts "
                         "c = R .. R+W-1 of layers x t_decode(c) + t_compress) / W, every t the mean "
@@ -848,7 +873,9 @@ def run_ours(args, world, rank, local):
                      "algorithmic_bytes_per_head_step_mean": roofline.lazy_bytes(d.form, d.d_k, d.d_v, cbar, fb),
                      "algorithmic_bytes_per_launch": dec_bytes,
                      "avg_launch_us": 1e3 * dec_launch_ms if dec_launch_ms else None,
-                     "launches": len(dec_ms)},
+                     "launches": len(dec_ms),
+                     "timing": ("CUDA events around each step's L overlapped launches, divided by L"
+                                if overlap else "CUDA events around each launch")},
         "decode_only": {"head_steps_per_s": BH * world / (dec_launch_ms / 1e3) if dec_launch_ms else None,
                         "GBps": dec_gbs},
         "compress": {"launches": len(cmp_ms), "ms_per_launch": t_cmp,

@@ -173,6 +173,20 @@ int seed_decode_step(const seed_dims* dims, const seed_state* state, int32_t lay
                      const float* q, const float* k, const float* v, const float* alpha,
                      const float* beta, float* o, void* ws, size_t ws_bytes, void* stream);
 
+/* seed_decode_step, with the same arguments and results, for a stream on which the
+ * launch just before this call does not write this layer's stored state (a, U, V,
+ * scale, ncols), e.g. the decode step of another layer.  The step may then begin
+ * streaming this layer's stored columns while that launch finishes (programmatic
+ * dependent launch, float32 factors with R + W <= 65; other shapes launch as
+ * seed_decode_step does).  It reads q, k, v, alpha, beta and the state's scalars,
+ * and writes anything, only after that launch has completed, so the inputs may be
+ * its outputs.  The caller owns the guarantee: if the launch before writes this
+ * layer's state (a seed_compress or a conversion of this layer, for instance), call
+ * seed_decode_step instead.                                                          */
+int seed_decode_step_overlapped(const seed_dims* dims, const seed_state* state, int32_t layer,
+                                const float* q, const float* k, const float* v, const float* alpha,
+                                const float* beta, float* o, void* ws, size_t ws_bytes, void* stream);
+
 /* Periodic compression (SEED figures & tables, Figure 1(b): every W steps the
  * factors are compressed back to rank R; SEED summary, Corollary 4 bounds its
  * open-loop error).  For every unit of `layer` (or all layers) whose ncols equals

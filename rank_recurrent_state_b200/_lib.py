@@ -42,6 +42,9 @@ SIGNATURES = {
     "seed_decode_step": (ctypes.c_int, [ctypes.POINTER(seed_dims), ctypes.POINTER(seed_state), c_int32,
                                         c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                         c_void_p, c_size_t, c_void_p]),
+    "seed_decode_step_overlapped": (ctypes.c_int, [ctypes.POINTER(seed_dims), ctypes.POINTER(seed_state), c_int32,
+                                                   c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                                   c_void_p, c_size_t, c_void_p]),
     "seed_compress": (ctypes.c_int, [ctypes.POINTER(seed_dims), ctypes.POINTER(seed_state), c_int32,
                                      c_void_p, c_void_p, c_size_t, c_void_p]),
     "seed_decode_step_compress": (ctypes.c_int, [ctypes.POINTER(seed_dims), ctypes.POINTER(seed_state), c_int32,

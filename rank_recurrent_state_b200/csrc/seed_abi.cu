@@ -115,6 +115,23 @@ int seed_decode_step(const seed_dims* dims, const seed_state* state, int32_t lay
                                   as_stream(stream));
 }
 
+int seed_decode_step_overlapped(const seed_dims* dims, const seed_state* state, int32_t layer, const float* q,
+                                const float* k, const float* v, const float* alpha, const float* beta,
+                                float* o, void* ws, size_t ws_bytes, void* stream) {
+  SEED_TRY(check_dims(dims));
+  SEED_TRY(check_layer(dims, layer, false));
+  SEED_TRY(check_state(state));
+  SEED_TRY(check_ptr(q));
+  SEED_TRY(check_ptr(k));
+  SEED_TRY(check_ptr(v));
+  SEED_TRY(check_ptr(alpha));
+  SEED_TRY(check_ptr(beta));
+  SEED_TRY(check_ptr(o));
+  SEED_TRY(check_ws(ws, ws_bytes));
+  return seed::launch_decode_step(*dims, *state, layer, q, k, v, alpha, beta, o, status_word(ws),
+                                  as_stream(stream), true);
+}
+
 int seed_decode_step_compress(const seed_dims* dims, const seed_state* state, int32_t layer, const float* q,
                               const float* k, const float* v, const float* alpha, const float* beta, float* o,
                               float* sigma_out, void* ws, size_t ws_bytes, void* stream) {

@@ -32,6 +32,14 @@ SEED_DEV bool wait_fault_injected(const uint32_t* status) {
   return *reinterpret_cast<const volatile uint32_t*>(status + kWsWaitFaultWord) != 0u;
 }
 
+// Programmatic dependent launch (sm_90 and later).  griddep_wait: block until the
+// grids this launch depends on have completed and their writes are visible (returns
+// at once for a launch made without the programmatic-serialization attribute).
+// griddep_launch_dependents: let the launch that depends on this grid begin; its
+// blocks take SM slots as this grid's blocks retire.
+SEED_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+SEED_DEV void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ vector helpers
 SEED_DEV float4 ld_stream4(const float* p) { return __ldcs(reinterpret_cast<const float4*>(p)); }
 SEED_DEV float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }

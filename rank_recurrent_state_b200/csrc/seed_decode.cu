@@ -395,9 +395,9 @@ static int launch_dims(const DecodeParams& p, int dk, int dv, int factors, cudaS
 
 int launch_decode_step(const seed_dims& d, const seed_state& s, int layer, const float* q,
                        const float* k, const float* v, const float* alpha, const float* beta,
-                       float* o, uint32_t* status, cudaStream_t st) {
+                       float* o, uint32_t* status, cudaStream_t st, bool overlap) {
   DecodeParams p{q, k, v, alpha, beta, o, s.a, s.U, s.V, s.scale, s.ncols, s.vbar, status,
-                 d.batch, d.layers, d.heads, layer, d.R, d.W, scale_len(d)};
+                 d.batch, d.layers, d.heads, layer, d.R, d.W, scale_len(d), overlap ? 1 : 0};
   switch (d.form) {
     case SEED_GDN: return launch_dims<SEED_GDN>(p, d.d_k, d.d_v, d.factors, st);
     case SEED_KDA: return launch_dims<SEED_KDA>(p, d.d_k, d.d_v, d.factors, st);

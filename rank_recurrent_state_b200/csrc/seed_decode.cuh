@@ -21,6 +21,7 @@ struct DecodeParams {
   const float* vbar;
   uint32_t* status;
   int B, L, H, layer, R, W, slen;
+  int overlap;   // host side only: launch with programmatic stream serialization
 };
 
 // One pipeline stage: everything a unit's step reads (U and V in their stored type).

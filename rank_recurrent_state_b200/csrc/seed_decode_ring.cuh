@@ -199,6 +199,13 @@ SEED_DEV void decode_ring_run(const DecodeParams& p) {
     return false;
   };
   fill();
+  // Up to here the launch has read only this layer's stored state (column counts, and
+  // the first chunks now in flight).  An overlapped launch (seed_decode_step_overlapped)
+  // may have begun while the launch before it on the stream was still running, which
+  // by the caller's guarantee writes none of that state but may write this step's
+  // inputs: everything else waits for it.  Then the next launch may begin.
+  griddep_wait();
+  griddep_launch_dependents();
 
   Vecs cur, nxt;
   if (u < n_units) ring_load_vecs<FORM, DK, DV, MAXC>(p, u, c_cur, cur);

@@ -74,9 +74,11 @@ int with_factor_type(const seed_dims& d, F&& f) {
 
 bool decode_dims_supported(int dk, int dv);
 
+// overlap: seed_decode_step_overlapped (the float32 ring kernel is then launched with
+// programmatic stream serialization; the other decode kernels launch as usual).
 int launch_decode_step(const seed_dims& d, const seed_state& s, int layer, const float* q,
                        const float* k, const float* v, const float* alpha, const float* beta,
-                       float* o, uint32_t* status, cudaStream_t st);
+                       float* o, uint32_t* status, cudaStream_t st, bool overlap = false);
 
 bool compress_fast_supported(const seed_dims& d);
 int launch_compress_fast(const seed_dims& d, const seed_state& s, int layer, float* sigma_out,

@@ -24,7 +24,7 @@ class DeviceRun:
 
     def __init__(self, cfg, batch: int | None = None, b0: int = 0, device: str = "cuda",
                  n_prefill: int | None = None, keep_dense: bool = False, ragged: bool = False,
-                 factors: int = S.SEED_FACTORS_F32, fused: bool = False):
+                 factors: int = S.SEED_FACTORS_F32, fused: bool = False, overlap: bool = False):
         self.cfg = cfg
         self.dims = S.Dims.from_config(cfg, batch, factors)
         self.key = S.synth_key(cfg, b0)
@@ -45,6 +45,10 @@ class DeviceRun:
         # requests still in their lead-in at lead-in step j are a prefix of the batch
         self.ragged = ragged
         self.fused = fused
+        # layers after the first use seed_decode_step_overlapped: the launch before
+        # each is the previous layer's step, which writes none of its state (the
+        # first layer may follow a compression)
+        self.overlap = overlap
         gb = torch.arange(b0, b0 + self.dims.batch)
         self.phase = (cfg.W - 1 - (gb * cfg.W) // cfg.batch).clamp(min=0) if ragged else torch.zeros_like(gb)
 
@@ -111,8 +115,8 @@ class DeviceRun:
                 if sig_l is not None:
                     sigma.view(d.batch, d.layers, d.heads, d.R)[:, l] = sig_l.view(d.batch, d.heads, d.R)
             else:
-                S.seed_decode_step(d, self.state, l, buf["q"], buf["k"], buf["v"], buf["alpha"],
-                                   buf["beta"], buf["o"], self.ws)
+                step = S.seed_decode_step_overlapped if (self.overlap and l > 0) else S.seed_decode_step
+                step(d, self.state, l, buf["q"], buf["k"], buf["v"], buf["alpha"], buf["beta"], buf["o"], self.ws)
             if dense and self.dense is not None:
                 S.seed_dense_step(d, self.dense, l, buf["q"], buf["k"], buf["v"], buf["alpha"],
                                   buf["beta"], buf["o_dense"], self.ws)

@@ -194,6 +194,18 @@ def seed_decode_step(dims: Dims, state: State, layer: int, q, k, v, alpha, beta,
         _ptr(o), ws.ptr, ws.nbytes, _stream(stream)))
 
 
+def seed_decode_step_overlapped(dims: Dims, state: State, layer: int, q, k, v, alpha, beta, o,
+                                ws: Workspace, stream=None) -> None:
+    """seed_decode_step for a stream whose previous launch does not write this layer's
+    state (e.g. another layer's step): the step may begin streaming the state while
+    that launch finishes, and reads its inputs after it."""
+    _check_state(dims, state)
+    d, s = dims.c(), state.c()
+    _check("seed_decode_step_overlapped", _lib.load().seed_decode_step_overlapped(
+        ctypes.byref(d), ctypes.byref(s), layer, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+        _ptr(o), ws.ptr, ws.nbytes, _stream(stream)))
+
+
 def seed_decode_step_noalloc(dims: Dims, state: State, layer: int, q, k, v, alpha, beta, o,
                              status_out: torch.Tensor | None = None, stream=None) -> None:
     """seed_decode_step with the library's own fixed device workspace; status_out, if

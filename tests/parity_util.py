@@ -29,11 +29,12 @@ def ensure_lib():
 
 
 def run_device(cfg, sample_units, n_prefill, n_decode, batch=None, factors=0, fused=False,
-               record_compress=True, record_units=None):
+               record_compress=True, record_units=None, overlap=False):
     """Run prefill, conversion and n_decode steps of every unit of (cfg, batch) on the
     device; return the trajectories of the sampled global units as numpy arrays.
     factors: storage format of U and V (seed_factors); fused: compress inside the
-    decode launch of the step that fills R + W (seed_decode_step_compress).
+    decode launch of the step that fills R + W (seed_decode_step_compress); overlap:
+    layers after the first step through seed_decode_step_overlapped.
     record_compress: also return, per compression, the sampled units' dense states
     right before and right after it (``S_pre``, ``S_post``; not with fused) and their
     sink a x vbar^T, for the optimality check of compare(); record_units: positions in
@@ -42,7 +43,7 @@ def run_device(cfg, sample_units, n_prefill, n_decode, batch=None, factors=0, fu
     from rank_recurrent_state_b200 import seed as S
     from rank_recurrent_state_b200.pipeline import DeviceRun
 
-    run = DeviceRun(cfg, batch=batch, n_prefill=n_prefill, factors=factors, fused=fused)
+    run = DeviceRun(cfg, batch=batch, n_prefill=n_prefill, factors=factors, fused=fused, overlap=overlap)
     d = run.dims
     run.prefill_and_convert()
     su = np.asarray(sample_units, dtype=np.int64)
