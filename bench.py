@@ -42,12 +42,12 @@ NOMINAL_HBM_GBS = 8000.0
 # again (no entry: the line's roofline.traffic is null).
 NCU_DECODE_TRAFFIC = [
     # decode_ring_kernel, float32 factors, layer 0 of step 3 after the conversion (c = 19):
-    # dram__bytes_read.sum 266.12 MB + dram__bytes_write.sum 17.83 MB
+    # dram__bytes_read.sum 266.10 MB + dram__bytes_write.sum 18.97 MB
     {"kernel": "decode_ring_kernel", "form": 0, "d_k": 128, "d_v": 128, "R": 16, "W": 16, "factors": 0,
-     "units": 12288, "c": 19, "bytes": 283.95e6},
-    # decode_warp_kernel, float16 factors, the same launch: 146.49 MB + 10.27 MB
+     "units": 12288, "c": 19, "bytes": 285.08e6},
+    # decode_warp_kernel, float16 factors, the same launch: 146.50 MB + 10.29 MB
     {"kernel": "decode_warp_kernel", "form": 0, "d_k": 128, "d_v": 128, "R": 16, "W": 16, "factors": 1,
-     "units": 12288, "c": 19, "bytes": 156.76e6},
+     "units": 12288, "c": 19, "bytes": 156.79e6},
 ]
 FALLBACK_HBM_GBS = 6650.0
 

@@ -177,8 +177,7 @@ int seed_decode_step(const seed_dims* dims, const seed_state* state, int32_t lay
  * launch just before this call does not write this layer's stored state (a, U, V,
  * scale, ncols), e.g. the decode step of another layer.  The step may then begin
  * streaming this layer's stored columns while that launch finishes (programmatic
- * dependent launch, float32 factors with R + W <= 65; other shapes launch as
- * seed_decode_step does).  It reads q, k, v, alpha, beta and the state's scalars,
+ * dependent launch, R + W <= 65; larger shapes launch as seed_decode_step does).  It reads q, k, v, alpha, beta and the state's scalars,
  * and writes anything, only after that launch has completed, so the inputs may be
  * its outputs.  The caller owns the guarantee: if the launch before writes this
  * layer's state (a seed_compress or a conversion of this layer, for instance), call

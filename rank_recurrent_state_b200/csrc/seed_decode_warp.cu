@@ -36,8 +36,21 @@ static int launch_warp_t(const DecodeParams& p, cudaStream_t st) {
   }
   const int units = p.B * p.H;
   const int grid = balanced_grid(units, per_sm * cache.sm_count[dev].load(std::memory_order_relaxed));
-  kern<<<grid, 32, smem, st>>>(p);
-  return cudaGetLastError() == cudaSuccess ? SEED_OK : SEED_ERR_CUDA;
+  if (!p.overlap) {
+    kern<<<grid, 32, smem, st>>>(p);
+    return cudaGetLastError() == cudaSuccess ? SEED_OK : SEED_ERR_CUDA;
+  }
+  cudaLaunchConfig_t cfg = {};   // programmatic stream serialization, as the ring kernel
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p) == cudaSuccess ? SEED_OK : SEED_ERR_CUDA;
 }
 
 template <int FORM, int DK, int DV, typename TS>

@@ -189,6 +189,10 @@ SEED_DEV void decode_warp_run(const DecodeParams& p, const FastParams* fp, const
   const bool fault = wait_fault_injected(p.status);
   int c = p.ncols[unit_index(p, u0)];
   if (lane == 0) issue_unit<DK, DV, TS>(p, sU, sV, full, u0, c, m, fault);
+  // as in the ring kernel: an overlapped launch has read only this layer's stored
+  // state so far; the step's inputs wait for the launch before it
+  griddep_wait();
+  griddep_launch_dependents();
   Vecs cur, nxt;
   load_vecs<FORM, DK, DV>(p, u0, c, cur);
   int c_next = u0 + stride < n_units ? p.ncols[unit_index(p, u0 + stride)] : 0;

@@ -74,8 +74,8 @@ int with_factor_type(const seed_dims& d, F&& f) {
 
 bool decode_dims_supported(int dk, int dv);
 
-// overlap: seed_decode_step_overlapped (the float32 ring kernel is then launched with
-// programmatic stream serialization; the other decode kernels launch as usual).
+// overlap: seed_decode_step_overlapped (the one-warp kernels, R + W <= 65, are then
+// launched with programmatic stream serialization; the four-warp kernel as usual).
 int launch_decode_step(const seed_dims& d, const seed_state& s, int layer, const float* q,
                        const float* k, const float* v, const float* alpha, const float* beta,
                        float* o, uint32_t* status, cudaStream_t st, bool overlap = false);
