@@ -99,16 +99,22 @@ SEED_DEV void gram_row(const float* P, float (&acc)[MP]) {
 
 // Equilibrate the Gram G (MP x MP, row-major, stride LG; columns at or beyond m are
 // zero) by its column norms and factor it by Cholesky in place, one warp, lane i
-// owning rows i and i + 32 (MP <= 64).  Right-looking: at step j the column below the pivot is
-// scaled and copied to colj, then every lane updates its rows below j against it
-// (whole rows, 128-bit accesses; the part above the diagonal is not read and is zeroed
-// at the end).  On return G[i * LG + j] = L[i][j] for j <= i, 0 above, and nrm holds
-// the column norms.  A zero column, or a non-positive pivot, gives a zero column of L;
-// a pivot below kCholPivotMin on a nonzero column also sets bad.
+// owning rows i and i + 32 (MP <= 64).  Right-looking in panels of four columns: the
+// lanes hold their rows' four panel entries in registers and factor the panel column
+// by column (the pivot and the column below it travel by warp shuffles), store it,
+// and then every row below the panel takes the panel's rank-4 update of its columns
+// to the right, four at a time, the panel rows of L read back from G (128-bit
+// accesses; the part above the diagonal is not read and is zeroed at the end).  Every
+// entry receives the same fused multiply-adds in the same order as a column-by-column
+// factorisation, with two warp barriers per panel instead of per column.  On return
+// G[i * LG + j] = L[i][j] for j <= i, 0 above, and nrm holds the column norms.  A
+// zero column, or a non-positive pivot, gives a zero column of L; a pivot below
+// kCholPivotMin on a nonzero column also sets bad.  ninv: MP floats of scratch.
 // Not inlined: each compression factors two Grams with it, and one copy of the code
 // keeps the kernel within the instruction cache.
 template <int MP, int LG>
-__device__ __noinline__ void cholesky_wide(float* G, int m, float* nrm, float* ninv, float* colj, bool& bad) {
+__device__ __noinline__ void cholesky_wide(float* G, int m, float* nrm, float* ninv, bool& bad) {
+  static_assert(MP % 4 == 0, "whole panels");
   const int lane = threadIdx.x & 31;
   constexpr int RPL = (MP + 31) / 32;
 #pragma unroll
@@ -135,50 +141,84 @@ __device__ __noinline__ void cholesky_wide(float* G, int m, float* nrm, float* n
   }
   __syncwarp();
 #pragma unroll 1
-  for (int j = 0; j < m; ++j) {
-    const float d = G[j * LG + j];
-    const bool zero = !(nrm[j] > 0.f);
-    bool drop = zero || !(d > 0.f);
-    if (!zero && d < kCholPivotMin) {
-      drop = true;
-      bad = true;
-    }
-    const float rs = drop ? 0.f : rsqrtf(d);
-    __syncwarp();   // every lane has read the pivot before its row is rewritten
-    float l[RPL];
+  for (int jb = 0; jb < m; jb += 4) {
+    // the panel: columns jb .. jb + 3 of the lane's rows
+    float p[RPL][4];
 #pragma unroll
     for (int h = 0; h < RPL; ++h) {
       const int i = lane + 32 * h;
-      l[h] = 0.f;
-      if (i >= MP) continue;
-      if (i > j) {
-        l[h] = G[i * LG + j] * rs;
-        G[i * LG + j] = l[h];
-      } else if (i == j) {
-        G[i * LG + i] = drop ? 0.f : d * rs;
+      const float4 t = i < MP ? ld4(G + i * LG + jb) : zero4();
+      p[h][0] = t.x; p[h][1] = t.y; p[h][2] = t.z; p[h][3] = t.w;
+    }
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int j = jb + t;
+      if (j >= m) break;
+      const float pj = (RPL > 1 && (j >> 5) == 1) ? p[RPL - 1][t] : p[0][t];
+      const float d = __shfl_sync(kFull, pj, j & 31);
+      const bool zero = !(nrm[j] > 0.f);
+      bool drop = zero || !(d > 0.f);
+      if (!zero && d < kCholPivotMin) {
+        drop = true;
+        bad = true;
       }
-      colj[i] = l[h];   // L[i][j] below the diagonal, 0 elsewhere
+      const float rs = drop ? 0.f : rsqrtf(d);
+      float l[RPL];
+#pragma unroll
+      for (int h = 0; h < RPL; ++h) {
+        const int i = lane + 32 * h;
+        l[h] = 0.f;
+        if (i >= MP) continue;
+        if (i > j) {
+          l[h] = p[h][t] * rs;
+          p[h][t] = l[h];
+        } else if (i == j) {
+          p[h][t] = drop ? 0.f : d * rs;
+        }
+      }
+      // the panel's columns after j: L[c][j] comes from the lane owning row c
+#pragma unroll
+      for (int t2 = t + 1; t2 < 4; ++t2) {
+        const int c = jb + t2;
+        const float lsrc = (RPL > 1 && (c >> 5) == 1) ? l[RPL - 1] : l[0];
+        const float lc = __shfl_sync(kFull, lsrc, c & 31);
+#pragma unroll
+        for (int h = 0; h < RPL; ++h) {
+          const int i = lane + 32 * h;
+          if (i > j && i < m && l[h] != 0.f) p[h][t2] = fmaf(-l[h], lc, p[h][t2]);
+        }
+      }
     }
-    __syncwarp();
-    const int c0 = (j + 1) & ~3;
 #pragma unroll
     for (int h = 0; h < RPL; ++h) {
       const int i = lane + 32 * h;
-      if (i > j && i < m && l[h] != 0.f) {
-        const float lij = l[h];
+      if (i < MP) st4(G + i * LG + jb, make_float4(p[h][0], p[h][1], p[h][2], p[h][3]));
+    }
+    __syncwarp();   // the panel's rows of L are in G
+    // rows below the panel: columns jb + 4 .. m - 1 against the panel (the rows of the
+    // panel itself have nothing left below the diagonal to the right of it)
+    const int c0 = jb + 4;
+#pragma unroll
+    for (int h = 0; h < RPL; ++h) {
+      const int i = lane + 32 * h;
+      if (i >= c0 && i < m) {
+        const float a0 = p[h][0], a1 = p[h][1], a2 = p[h][2], a3 = p[h][3];
 #pragma unroll 2
         for (int c4 = c0; c4 < m; c4 += 4) {
-          const float4 lc = ld4(colj + c4);
           float4 g = ld4(G + i * LG + c4);
-          g.x = fmaf(-lij, lc.x, g.x);
-          g.y = fmaf(-lij, lc.y, g.y);
-          g.z = fmaf(-lij, lc.z, g.z);
-          g.w = fmaf(-lij, lc.w, g.w);
+          const float4 r0 = ld4(G + c4 * LG + jb);          // L[c4][jb .. jb + 3]
+          const float4 r1 = ld4(G + (c4 + 1) * LG + jb);
+          const float4 r2 = ld4(G + (c4 + 2) * LG + jb);
+          const float4 r3 = ld4(G + (c4 + 3) * LG + jb);
+          g.x = fmaf(-a0, r0.x, g.x); g.x = fmaf(-a1, r0.y, g.x); g.x = fmaf(-a2, r0.z, g.x); g.x = fmaf(-a3, r0.w, g.x);
+          g.y = fmaf(-a0, r1.x, g.y); g.y = fmaf(-a1, r1.y, g.y); g.y = fmaf(-a2, r1.z, g.y); g.y = fmaf(-a3, r1.w, g.y);
+          g.z = fmaf(-a0, r2.x, g.z); g.z = fmaf(-a1, r2.y, g.z); g.z = fmaf(-a2, r2.z, g.z); g.z = fmaf(-a3, r2.w, g.z);
+          g.w = fmaf(-a0, r3.x, g.w); g.w = fmaf(-a1, r3.y, g.w); g.w = fmaf(-a2, r3.z, g.w); g.w = fmaf(-a3, r3.w, g.w);
           st4(G + i * LG + c4, g);
         }
       }
     }
-    __syncwarp();   // the updated rows, and colj free again
+    __syncwarp();   // the updated rows, before the next panel reads them
   }
 #pragma unroll
   for (int h = 0; h < RPL; ++h) {
@@ -665,16 +705,16 @@ SEED_DEV bool compress_fast_unit(const FastParams& p, const CUtensorMap& tmU, co
     if (lane == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
     return false;
   }
-  // equilibrated Cholesky in shared memory; nrm and du are free until after both
-  // factorisations and serve as its scratch
-  cholesky_wide<MP, LG>(sLu, m, nu, nrm, du, bad);
+  // equilibrated Cholesky in shared memory; nrm is free until after both
+  // factorisations and serves as its scratch
+  cholesky_wide<MP, LG>(sLu, m, nu, nrm, bad);
   // V: chunks NCU .. NCH-1; L_v over the chunk buffers once the last one is read
   if (!gram_stream<KDA, DK, DV, MP, LG, TS>(NCU, NCH, false, sA, &tmU, &tmV, p, unit, m, bar, uses, scl, sM,
                                             bad, false)) {
     if (lane == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
     return false;
   }
-  cholesky_wide<MP, LG>(sM, m, nv, nrm, du, bad);
+  cholesky_wide<MP, LG>(sM, m, nv, nrm, bad);
   if (__any_sync(kFull, bad)) {
     if (lane == 0) atomicAdd(p.status + 6, 1u);
     return true;

@@ -11,8 +11,8 @@
 //      matrices accumulate on the tensor cores (split TF32, float32 accuracy), only
 //      the tiles of columns below R + W;
 //   2. each Gram is equilibrated and factored by Cholesky in shared memory,
-//      right-looking, lane i holding rows i and i + 32 (a row-major update against the
-//      broadcast column j);
+//      right-looking in panels of four columns, lane i holding rows i and i + 32 (the
+//      panel in registers, then a rank-4 update of the rows below it);
 //   3. M = L_u^T diag(w) L_v is formed in place of L_v, lane j holding columns j and
 //      j + 32;
 //   4. one-sided Jacobi on M in registers, one column pair per lane (jacobi_regs),
@@ -48,8 +48,8 @@ struct WideLayout {
   static constexpr int LU = A;
   static constexpr int SMALL = LU + MP * LG;
   static constexpr int SL = FORM == SEED_KDA ? DK : MP;
-  // nu nv du wk sg ninv colj (7 x MP), fu fv (2 x 32), scl
-  static constexpr int FLOATS = SMALL + 7 * MP + 2 * kWideMaxR + SL;
+  // nu nv du wk sg ninv (6 x MP), fu fv (2 x 32), scl
+  static constexpr int FLOATS = SMALL + 6 * MP + 2 * kWideMaxR + SL;
   static constexpr size_t BAR_OFF = (FLOATS * sizeof(float) + kWideMaxR * sizeof(int) + 7) & ~size_t(7);
   static constexpr size_t bytes = BAR_OFF + 2 * sizeof(uint64_t);
   static_assert(MP * XS <= A, "the transposed left vectors fit region A");
@@ -166,8 +166,7 @@ SEED_DEV bool compress_wide_unit(const FastParams& p, const CUtensorMap& tmU, co
   float* wk = du + MP;
   float* sg = wk + MP;
   float* ninv = sg + MP;
-  float* colj = ninv + MP;
-  float* fu = colj + MP;
+  float* fu = ninv + MP;
   float* fv = fu + kWideMaxR;
   float* scl = fv + kWideMaxR;
   int* sel = reinterpret_cast<int*>(scl + Lay::SL);
@@ -193,13 +192,13 @@ SEED_DEV bool compress_wide_unit(const FastParams& p, const CUtensorMap& tmU, co
     if (lane == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
     return false;
   }
-  cholesky_wide<MP, LG>(sLu, m, nu, ninv, colj, bad);
+  cholesky_wide<MP, LG>(sLu, m, nu, ninv, bad);
   if (!gram_wide<KDA, DK, DV, MP, LG, TS>(NCU, NCH, false, sA, &tmU, &tmV, p, unit, m, bar, uses, scl, sM, bad,
                                           false)) {
     if (lane == 0) raise_flag(p.status, SEED_FLAG_TIMEOUT);
     return false;
   }
-  cholesky_wide<MP, LG>(sM, m, nv, ninv, colj, bad);
+  cholesky_wide<MP, LG>(sM, m, nv, ninv, bad);
   if (__any_sync(kFull, bad)) {
     if (lane == 0) atomicAdd(p.status + 6, 1u);
     return true;
