@@ -407,6 +407,17 @@ def compress_rate(d, diag, cmp_ms, clk):
             "frac_fp32_peak": tflops / peak}
 
 
+def per_launch_times(records):
+    """Decode timings per launch, (ms, column count), from the timed region's event
+    records (start, end, c, n): n = 1 for a launch timed alone; n = L for one event
+    pair around a step's L overlapped launches (an event between two launches would
+    serialise them), which gives each of the L launches an equal share."""
+    out = []
+    for a, b, c, n in records:
+        out += [(a.elapsed_time(b) / n, c)] * n
+    return out
+
+
 def steady_state(dec, cmp_ms, R, W, layers):
     """Steady-state step time from the run's own per-launch CUDA-event times.
 
@@ -792,9 +803,7 @@ def run_ours(args, world, rank, local):
     s_next = args.warmup + args.steps
 
     units = d.units
-    dec_pairs = []   # per launch: (ms, column count); a step-wide pair gives each launch its share
-    for a, b, c, n in ev["dec"]:
-        dec_pairs += [(a.elapsed_time(b) / n, c)] * n
+    dec_pairs = per_launch_times(ev["dec"])
     cmp_ms = [a.elapsed_time(b) for a, b in ev["cmp"]]
     fus_ms = [a.elapsed_time(b) for a, b in ev["fus"]]
     extra_cmp = False

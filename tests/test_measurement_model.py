@@ -104,3 +104,34 @@ def test_bench_steady_state_is_independent_of_the_timed_window():
             c = R if c + 1 == R + W else c + 1
         st = bench.steady_state(dec, [t_cmp], R, W, L)
         assert abs(st["ms_per_step"] - exact) <= 1e-9 * exact, (warmup, steps, st)
+
+
+def test_step_wide_decode_timing_gives_the_same_steady_state():
+    """With overlapped layer launches the bench times each step's L decode launches
+    with one event pair; per_launch_times spreads it over the L launches, so the
+    steady state equals that of per-launch events with the same total per step."""
+    import bench
+
+    class Ev:
+        def __init__(self, t):
+            self.t = t
+
+        def elapsed_time(self, other):
+            return other.t - self.t
+
+    R, W, L = 16, 16, 36
+    per_launch, per_step = [], []
+    clock, c = 0.0, R
+    for s in range(2 * W):
+        t0 = clock
+        for _ in range(L):
+            per_launch.append((Ev(clock), Ev(clock + 0.04 + 0.001 * c), c, 1))
+            clock += 0.04 + 0.001 * c
+        per_step.append((Ev(t0), Ev(clock), c, L))
+        c = R if c + 1 == R + W else c + 1
+    a = bench.per_launch_times(per_launch)
+    b = bench.per_launch_times(per_step)
+    assert len(a) == len(b) == 2 * W * L
+    sa = bench.steady_state(a, [40.0], R, W, L)
+    sb = bench.steady_state(b, [40.0], R, W, L)
+    assert abs(sa["ms_per_step"] - sb["ms_per_step"]) <= 1e-9 * sa["ms_per_step"]
