@@ -494,7 +494,9 @@ def run_e2e(args, run, d, L, BH, q, k, v, alpha, beta, o, kda, stream, dev, worl
         avail = psutil.virtual_memory().available
     except ImportError:
         avail = 64 << 30
-    Ph = max(2, min(q.shape[0], int(0.25 * avail) // step_bytes))
+    # a quarter of the host memory, shared by the ranks on this node
+    ranks_here = max(1, int(os.environ.get("LOCAL_WORLD_SIZE", world)))
+    Ph = max(2, min(q.shape[0], int(0.25 * avail / ranks_here) // step_bytes))
     try:
         hq = torch.empty(Ph, L, BH, d.d_k, dtype=torch.float32, pin_memory=True)
         hk = torch.empty_like(hq, pin_memory=True)
