@@ -252,7 +252,7 @@ def cpu_oracle_rate(cfg, seconds: float, rank_seed: int = 0) -> dict:
             "affinity_cores": len(os.sched_getaffinity(0))}
 
 
-def config_obj(cfg, batch, world, prefill, ragged=False, factors="f32", fused=False, overlap=False):
+def config_obj(cfg, batch, world, prefill, ragged=False, factors="f32", fused=False):
     schedule = ("ragged: request b joined W-1-floor(bW/B) steps before the others; a compression "
                 "launch after every step compresses the units that are due" if ragged else
                 "lockstep: every unit compresses after steps W, 2W, ...")
@@ -267,10 +267,7 @@ def config_obj(cfg, batch, world, prefill, ragged=False, factors="f32", fused=Fa
                             else "a separate launch over all units after the step that fills R + W"),
             "factors": factors + (" (U and V stored in 16 bits, rounded to nearest when written)"
                                   if factors != "f32" else ""),
-            "l2": "inputs and state larger than L2 (no flush needed)",
-            "layer_launches": ("layers after the first begin during the previous layer's launch "
-                               "(seed_decode_step_overlapped, programmatic dependent launch)" if overlap
-                               else "one after another (seed_decode_step)")}
+            "l2": "inputs and state larger than L2 (no flush needed)"}
 
 
 def run_reference(args, world, rank):
@@ -865,7 +862,7 @@ def run_ours(args, world, rank, local):
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded Philox4x32-10 inputs and prefill, generated on the device)",
-        "config": config_obj(cfg, B, world, prefill, args.ragged, args.factors, args.fused, overlap),
+        "config": config_obj(cfg, B, world, prefill, args.ragged, args.factors, args.fused),
         "steady_state": (None if steady is None else dict(
             steady, how="value = units / t_step with t_step = (sum over the window's column counts "
                         "c = R .. R+W-1 of layers x t_decode(c) + t_compress) / W, every t the mean "
@@ -886,7 +883,10 @@ def run_ours(args, world, rank, local):
                      "avg_launch_us": 1e3 * dec_launch_ms if dec_launch_ms else None,
                      "launches": len(dec_ms),
                      "timing": ("CUDA events around each step's L overlapped launches, divided by L"
-                                if overlap else "CUDA events around each launch")},
+                                if overlap else "CUDA events around each launch"),
+                     "layer_launches": ("layers after the first begin during the previous layer's launch "
+                                        "(seed_decode_step_overlapped, programmatic dependent launch)"
+                                        if overlap else "one after another (seed_decode_step)")},
         "decode_only": {"head_steps_per_s": BH * world / (dec_launch_ms / 1e3) if dec_launch_ms else None,
                         "GBps": dec_gbs},
         "compress": {"launches": len(cmp_ms), "ms_per_launch": t_cmp,
