@@ -23,17 +23,19 @@ def _lib():
     ensure_lib()
 
 
-def _run(cid=1, batch=2, n_prefill=64):
+def _run(cid=1, batch=2, n_prefill=64, factors=0):
     from rank_recurrent_state_b200.pipeline import DeviceRun
-    run = DeviceRun(config(cid, batch=batch), n_prefill=n_prefill)
+    run = DeviceRun(config(cid, batch=batch), n_prefill=n_prefill, factors=factors)
     run.prefill_and_convert()
     return run
 
 
-def test_decode_wait_runs_out_and_leaves_the_state_unchanged():
+# float32 factors: the ring kernel; 16-bit: the whole-unit stage kernel
+@pytest.mark.parametrize("factors", [0, 1], ids=["f32-ring", "f16-whole-unit"])
+def test_decode_wait_runs_out_and_leaves_the_state_unchanged(factors):
     import torch
     from rank_recurrent_state_b200 import seed as S
-    run, twin = _run(), _run()
+    run, twin = _run(factors=factors), _run(factors=factors)
     d = run.dims
     buf = S.alloc_step_inputs(d)
     run.gen_inputs(0, 0, buf)
