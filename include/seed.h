@@ -194,8 +194,9 @@ int seed_decode_step_overlapped(const seed_dims* dims, const seed_state* state, 
  * (Q_u X_R) Sigma_R (Q_v Y_R)^T written to slots 0..R-1; ncols <- R.  The sink a
  * is not touched.  Units with ncols != R+W are left unchanged.
  * How Sigma_R is stored depends on the path a unit takes (both represent the same
- * state): R + W <= 32, R <= 16, d_k, d_v in {64, 128} and a well-conditioned,
- * well-scaled unit take Cholesky QR, which for GDN and Mamba-2 stores the unit
+ * state): with d_k, d_v in {64, 128} and either R + W <= 32 and R <= 16, or
+ * 32 < R + W <= 64 and R <= 32, a well-conditioned, well-scaled unit takes
+ * Cholesky QR, which for GDN and Mamba-2 stores the unit
  * columns Q_u X_R, Q_v Y_R and scale_r = sigma_r (scale 1 beyond R), and for KDA
  * Sigma^{1/2} on each side with P <- 1; every other unit takes Householder QR,
  * which stores Sigma^{1/2} on each side and resets the scales to 1.
