@@ -44,12 +44,6 @@ SEED_DEV void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar
       : "memory");
 }
 
-// Bulk prefetch of [src, src + bytes) from global memory into L2 (no shared memory, no
-// completion to wait for); src 16-byte aligned, bytes a multiple of 16.
-SEED_DEV void bulk_prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-
 // Ampere-style asynchronous 16-byte copy global -> shared (no mbarrier): groups
 // are committed in order and waited for by count; each thread waits for its own.
 SEED_DEV void cp_async16(void* dst, const void* src) {
