@@ -8,6 +8,13 @@
    per sweep, whatever the arrangement a sweep starts from.
 2. The transposed warp reduction (warp_xreduce<NV>): after it, lane l holds the
    total of value (l >> (5 - log2 NV)) & (NV - 1).
+3. The decode ring's chunk sequence (decode_ring_run): a warp's units u0, u0 +
+   stride, ... pass through NSLOT slots as chunks (its U chunks, then its V chunks);
+   lane 0 refills a slot with the next chunk of the sequence, which after the current
+   unit's last chunk belongs to the next unit.  Every chunk the warp reads must be
+   the one issued into that position for that unit, at most NSLOT may be in flight,
+   none may be left in flight when the warp exits, and a unit's chunks must cover
+   its stored columns exactly.
 """
 
 import itertools
@@ -126,3 +133,94 @@ def test_16bit_chunk_widening_lands_in_the_swizzled_layout(mp, m):
     for j in range(mp):
         for e in range(32):
             assert chunk[_swz(j, e)] == ((1000 * j + e) if j < m else 0.0)
+
+
+RING_CHUNK = 8
+
+
+def _ring_chunks(c, m):
+    return 2 * ((c + RING_CHUNK - 1) // RING_CHUNK) if 0 < c < m else 0
+
+
+def _ring_issue(c, kidx):
+    """Columns of chunk kidx of a unit holding c columns: (is V, first column, count)."""
+    n = (c + RING_CHUNK - 1) // RING_CHUNK
+    is_v = kidx >= n
+    col0 = (kidx - n if is_v else kidx) * RING_CHUNK
+    return is_v, col0, min(c - col0, RING_CHUNK)
+
+
+def _ring_warp(ncols, n_units, stride, u0, nslot, m):
+    """The control flow of one warp of decode_ring_run: returns the chunks issued
+    (sequence number -> (unit, kidx)) and read ((unit, kidx) in order), checking
+    the in-flight bound as it goes."""
+    issued_log, read = {}, []
+    st = {"u": u0, "base": 0, "issued": 0, "consumed": 0}
+    st["c_cur"] = ncols[u0] if u0 < n_units else 0
+    st["c_nxt"] = ncols[u0 + stride] if u0 + stride < n_units else 0
+    st["n_cur"] = _ring_chunks(st["c_cur"], m)
+    st["n_nxt"] = _ring_chunks(st["c_nxt"], m) if u0 + stride < n_units else 0
+
+    def fill():
+        while st["issued"] < st["consumed"] + nslot:
+            i, base = st["issued"], st["base"]
+            if i < base + st["n_cur"]:
+                uu, kk = st["u"], i - base
+            elif i < base + st["n_cur"] + st["n_nxt"]:
+                uu, kk = st["u"] + stride, i - base - st["n_cur"]
+            else:
+                break
+            issued_log[i] = (uu, kk)
+            st["issued"] += 1
+            assert st["issued"] - st["consumed"] <= nslot
+
+    def consume(unit, kidx):
+        assert st["consumed"] < st["issued"], "a read with no chunk issued"
+        assert issued_log[st["consumed"]] == (unit, kidx), (st["consumed"], issued_log[st["consumed"]], unit, kidx)
+        read.append((unit, kidx))
+        st["consumed"] += 1
+        fill()
+
+    fill()
+    while st["u"] < n_units:
+        u = st["u"]
+        u_next = u + stride
+        c_aft = ncols[u_next + stride] if u_next + stride < n_units else 0
+        c = st["c_cur"]
+        if 0 <= c < m:
+            nch = st["n_cur"] // 2
+            for ch in range(nch):        # U chunks
+                consume(u, ch)
+            for ch in range(nch):        # V chunks
+                consume(u, nch + ch)
+        st["base"] += st["n_cur"]
+        st["n_cur"], st["c_cur"], st["c_nxt"] = st["n_nxt"], st["c_nxt"], c_aft
+        st["n_nxt"] = _ring_chunks(c_aft, m) if u_next + stride < n_units else 0
+        st["u"] = u_next
+        fill()
+    assert st["issued"] == st["consumed"], "copies left in flight at exit"
+    return issued_log, read
+
+
+@pytest.mark.parametrize("m,nslot", [(32, 4), (32, 3), (40, 4), (65, 8), (17, 5)])
+@pytest.mark.parametrize("stride,n_units", [(1, 7), (3, 23), (7, 23), (30, 23)])
+def test_decode_ring_reads_every_unit_chunk_in_order(m, nslot, stride, n_units):
+    rng = np.random.default_rng(m * 1000 + nslot * 100 + stride * 10 + n_units)
+    R = max(1, m // 2)
+    ncols = list(rng.integers(R, m, size=n_units))      # R .. m - 1 columns held
+    for i in rng.choice(n_units, size=min(3, n_units), replace=False):
+        ncols[i] = int(rng.choice([0, m, -1]))          # empty, full and invalid units
+    for u0 in range(min(stride, n_units)):
+        _, read = _ring_warp(ncols, n_units, stride, u0, nslot, m)
+        for u in range(u0, n_units, stride):
+            c = ncols[u]
+            got = [k for uu, k in read if uu == u]
+            n = _ring_chunks(c, m)
+            assert got == list(range(n)), (u, c, got)
+            cols = {False: [], True: []}
+            for k in got:
+                is_v, col0, cnt = _ring_issue(c, k)
+                assert 0 < cnt <= RING_CHUNK
+                cols[is_v] += list(range(col0, col0 + cnt))
+            if n:
+                assert cols[False] == list(range(c)) and cols[True] == list(range(c)), (u, c)
