@@ -15,6 +15,11 @@
    the one issued into that position for that unit, at most NSLOT may be in flight,
    none may be left in flight when the warp exits, and a unit's chunks must cover
    its stored columns exactly.
+4. The compression's Cholesky in panels of four columns (cholesky_wide): every
+   entry must receive the same multiply-adds in the same order as a column-by-column
+   right-looking factorisation (emulated in float32 with the same operation for
+   both, so the two agree bit for bit exactly when the orders agree), with the same
+   dropped columns and the same rejection of small pivots.
 """
 
 import itertools
@@ -224,3 +229,109 @@ def test_decode_ring_reads_every_unit_chunk_in_order(m, nslot, stride, n_units):
                 cols[is_v] += list(range(col0, col0 + cnt))
             if n:
                 assert cols[False] == list(range(c)) and cols[True] == list(range(c)), (u, c)
+
+
+PIVOT_MIN = np.float32(1e-2)   # kCholPivotMin
+
+
+def _madd(a, b, c):
+    # the same float32 operation for both orders (the device fuses it; only the order
+    # of the updates is under test here)
+    return np.float32(np.float32(a * b) + c)
+
+
+def _equilibrate(G, m):
+    G = G.astype(np.float32).copy()
+    mp = G.shape[0]
+    nrm = np.zeros(mp, np.float32)
+    for i in range(m):
+        nrm[i] = np.sqrt(max(G[i, i], np.float32(0)))
+    ninv = np.array([np.float32(1) / n if n > 0 else np.float32(0) for n in nrm], np.float32)
+    for i in range(mp):
+        for j in range(mp):
+            G[i, j] = np.float32(G[i, j] * np.float32(ninv[i] * ninv[j]))
+    return G, nrm
+
+
+def _pivot(d, n):
+    zero = not (n > 0)
+    drop = zero or not (d > 0)
+    bad = False
+    if not zero and d < PIVOT_MIN:
+        drop, bad = True, True
+    rs = np.float32(0) if drop else np.float32(1) / np.sqrt(d)
+    return drop, bad, np.float32(rs)
+
+
+def _chol_columns(G0, m):
+    G, nrm = _equilibrate(G0, m)
+    mp, bad = G.shape[0], False
+    for j in range(m):
+        d = G[j, j]
+        drop, b, rs = _pivot(d, nrm[j])
+        bad |= b
+        col = np.zeros(mp, np.float32)
+        for i in range(j + 1, mp):
+            col[i] = np.float32(G[i, j] * rs)
+            G[i, j] = col[i]
+        G[j, j] = np.float32(0) if drop else np.float32(d * rs)
+        for i in range(j + 1, m):
+            if col[i] != 0:
+                for c in range(j + 1, m):
+                    G[i, c] = _madd(-col[i], col[c], G[i, c])
+    return np.tril(G[:m, :m]), bad
+
+
+def _chol_panels(G0, m):
+    G, nrm = _equilibrate(G0, m)
+    mp, bad = G.shape[0], False
+    for jb in range(0, m, 4):
+        p = G[:, jb:jb + 4].copy()                   # every row's panel entries
+        for t in range(4):
+            j = jb + t
+            if j >= m:
+                break
+            d = p[j, t]
+            drop, b, rs = _pivot(d, nrm[j])
+            bad |= b
+            l = np.zeros(mp, np.float32)
+            for i in range(j + 1, mp):
+                l[i] = np.float32(p[i, t] * rs)
+                p[i, t] = l[i]
+            p[j, t] = np.float32(0) if drop else np.float32(d * rs)
+            for t2 in range(t + 1, 4):
+                lc = l[jb + t2]
+                for i in range(j + 1, m):
+                    if l[i] != 0:
+                        p[i, t2] = _madd(-l[i], lc, p[i, t2])
+        G[:, jb:jb + 4] = p
+        for i in range(jb + 4, m):                   # rank-4 update of the rows below
+            for c4 in range(jb + 4, m, 4):
+                for e in range(4):
+                    c = c4 + e
+                    g = G[i, c]
+                    for t in range(4):
+                        g = _madd(-p[i, t], G[c, jb + t], g)
+                    G[i, c] = g
+    return np.tril(G[:m, :m]), bad
+
+
+@pytest.mark.parametrize("m,mp", [(7, 16), (16, 16), (23, 32), (32, 32), (40, 64), (61, 64)])
+@pytest.mark.parametrize("kind", ["random", "zero-column", "near-parallel"])
+def test_panel_cholesky_matches_the_column_order(m, mp, kind):
+    rng = np.random.default_rng(m * 7 + mp)
+    A = rng.standard_normal((3 * m, m))
+    if kind == "zero-column":
+        A[:, m // 2] = 0
+    if kind == "near-parallel":
+        A[:, m - 1] = A[:, 0] + 1e-3 * rng.standard_normal(3 * m)   # pivot below the minimum
+    G = np.zeros((mp, mp))
+    G[:m, :m] = A.T @ A
+    L1, bad1 = _chol_columns(G, m)
+    L2, bad2 = _chol_panels(G, m)
+    assert bad1 == bad2 == (kind == "near-parallel")
+    np.testing.assert_array_equal(L1, L2)
+    if kind == "random":   # and it is the Cholesky factor of the equilibrated Gram
+        d = np.sqrt(np.diag(G[:m, :m]))
+        ref = np.linalg.cholesky(G[:m, :m] / np.outer(d, d))
+        np.testing.assert_allclose(L1, ref, rtol=0, atol=1e-4)
