@@ -89,16 +89,18 @@ def test_scale_len_and_workspace(lib):
     (_dims(d_k=16, d_v=16, R=8, W=16), -2),     # R + W > d
     (_dims(R=64, W=64), -2),                    # R + W > SEED_MAX_COLS
 ])
-def test_decode_step_rejects_bad_dims(lib, dims, code):
+@pytest.mark.parametrize("entry", ["seed_decode_step", "seed_decode_step_overlapped"])
+def test_decode_step_rejects_bad_dims(lib, dims, code, entry):
     d = ctypes.byref(dims) if dims is not None else None
     s = _state()
-    rc = lib.seed_decode_step(d, ctypes.byref(s), 0, A, A, A, A, A, A, A, 256, None)
+    rc = getattr(lib, entry)(d, ctypes.byref(s), 0, A, A, A, A, A, A, A, 256, None)
     assert rc == code
 
 
-def test_decode_step_rejects_bad_pointers_and_layer(lib):
+@pytest.mark.parametrize("entry", ["seed_decode_step", "seed_decode_step_overlapped"])
+def test_decode_step_rejects_bad_pointers_and_layer(lib, entry):
     d, s = _dims(), _state()
-    call = lambda layer=0, st=s, q=A, ws=A, wsb=256: lib.seed_decode_step(  # noqa: E731
+    call = lambda layer=0, st=s, q=A, ws=A, wsb=256: getattr(lib, entry)(  # noqa: E731
         ctypes.byref(d), ctypes.byref(st), layer, q, A, A, A, A, A, ws, wsb, None)
     assert call(layer=3) == -1
     assert call(layer=-1) == -1                  # all layers is not a decode step
