@@ -1,15 +1,20 @@
 #!/usr/bin/env python
 """Throughput of the SEED decode hot path on B200: head-steps/s and HBM GB/s.
 
-A step is one pass of the whole hot path over one batch: seed_decode_step for
-every layer (one launch per layer), and seed_compress over all layers after the
-step that fills R + W columns.  Default workload: 36 GDN layers x 48 heads of
-128 x 128, R = W = 16, batch 256 requests per GPU (the full recurrent stack).
+A step is one pass of the whole hot path over one batch: the decode step of
+every layer (one launch per layer; layers after the first through
+seed_decode_step_overlapped, so that each starts during the previous one's tail),
+and seed_compress over all layers after the step that fills R + W columns.
+Default workload: 36 GDN layers x 48 heads of 128 x 128, R = W = 16, batch 256
+requests per GPU (the full recurrent stack).
 
 Timing: W untimed warm-up steps, then K steps between barriers and device
-synchronisations, CUDA events on the launching stream (max over ranks).  Inputs
-(q, k, v, alpha, beta of a pool of distinct steps) are generated on the device
-before the timed region and are larger than L2, as is the 15 GB state.
+synchronisations, CUDA events on the launching stream (max over ranks).  The
+headline is the steady state of a compression window, from the events of each
+step's decode launches and of each compression.  Inputs (q, k, v, alpha, beta of
+a pool of distinct steps) are generated on the device before the timed region
+and are larger than L2, as is the 15 GB state.  The end-to-end figure copies a
+step's inputs from pinned host memory and its o back inside its own timed region.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
